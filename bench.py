@@ -1,0 +1,501 @@
+"""Benchmark of the MX block-quantization hot path on one or more B200s.
+
+Workload: a Llama-3-8B-shaped linear layer, A = 8192 x 4096 bf16 activations
+(Laplace(0,1)), W = 14336 x 4096 bf16 weights (N(0, 0.02)), synthetic and
+seeded.  One step = every memory-bound row of the path on A and W:
+MXFP4 quantize+pack with fused fidelity stats, NVFP4 (tensor amax pre-pass +
+UE4M3 quantize), 32-point Hadamard + MXFP4, MBS + OAS MXFP4, and dequantize
+to bf16; launches alternate between A and W so that consecutive kernels read
+different tensors (A + W = 176 MiB > the 126 MB L2).  ``value`` is the
+step's algorithmic bytes (inputs read once, codes/scales/outputs written
+once; the NVFP4 amax pre-pass is time, not bytes) over the step time, summed
+over ranks.  The block-scaled FP4 GEMM (A^Q W^Q^T, FP32 accumulate) is timed
+as its own leg in the same run and reported under ``gemm``.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+(N > 1: launched by torchrun, one process per GPU, weak scaling: every rank
+quantizes its own copy of the layer, no data-path collective.)
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M_TOK, K_DIM, N_OUT = 8192, 4096, 14336
+WORKLOAD = ("Llama-3-8B-shaped linear layer: A 8192x4096 bf16 Laplace(0,1) seed 6, "
+            "W 14336x4096 bf16 N(0,0.02) seed 7 (W stored out x in, product A W^T)")
+METRIC = "MX quantize+pack GB/s (% of ~8 TB/s HBM); block-scaled FP4 GEMM TFLOPS"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-gemm", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d, "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# --------------------------------------------------------------- the step --
+def step_plan(mx):
+    """(name, tensor, config, kind) for every launch of one step."""
+    mxfp4 = mx.MXFP4
+    nvfp4 = mx.NVFP4
+    had = mx.Config(hadamard=32)
+    mbs = mx.Config(macro_block=128, rule=mx.RULE_OAS, oas_tau=7.0)
+    return [
+        ("mxfp4_row", "A", mxfp4, "q"), ("mxfp4_row", "W", mxfp4, "q"),
+        ("nvfp4_row", "A", nvfp4, "q"), ("nvfp4_row", "W", nvfp4, "q"),
+        ("had32_mxfp4", "A", had, "q"), ("had32_mxfp4", "W", had, "q"),
+        ("mbs_oas_mxfp4", "A", mbs, "q"), ("mbs_oas_mxfp4", "W", mbs, "q"),
+        ("dequant_mxfp4_bf16", "A", mxfp4, "d"), ("dequant_mxfp4_bf16", "W", mxfp4, "d"),
+    ]
+
+
+def algo_bytes(cfg, rows, cols, kind, in_bytes=2):
+    n = rows * cols
+    code = n if cfg.elem in (2, 3) else n // 2
+    nb = n // cfg.block if cfg.axis != 2 else n // 1024
+    macro = n // 128 if cfg.macro_block else 0
+    offs = 2 * nb if cfg.asymmetric else 0
+    if kind == "q":
+        return in_bytes * n + code + nb + macro + offs
+    return code + nb + macro + offs + 2 * n       # dequantize to bf16
+
+
+def launches_per_call(cfg, kind):
+    if kind == "d":
+        return 1
+    k = 2                                  # quantize + stats finalisation
+    if cfg.tensor_scale == 1:
+        k += 2                             # amax pre-pass + tensor-scale kernel
+    return k
+
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for ln in f:
+                    parts = [p.strip() for p in ln.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        except OSError:
+            pass
+        finally:
+            if self.path:
+                os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx_ = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx_) if mx_ else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def traffic_record(kernel_key: str):
+    """dram read+write bytes per launch from the committed ncu summary, or None
+    when the kernel sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel_key)
+    except (OSError, ValueError):
+        return None
+    if not rec:
+        return None
+    h = hashlib.sha256()
+    for rel in rec.get("sources", []):
+        try:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+        except OSError:
+            return None
+    if h.hexdigest()[:16] != rec.get("sources_sha256_16"):
+        return None
+    return rec.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------ our arm ------
+def run_ours(args, rank, world, device):
+    import microscaling_block_quantization_b200 as mx
+    from microscaling_block_quantization_b200 import inputs
+
+    A_cpu, W_cpu = inputs.llama_linear(M_TOK, K_DIM, N_OUT)
+    A = A_cpu.to(device)
+    W = W_cpu.to(device)
+    T = {"A": A, "W": W}
+    plan = step_plan(mx)
+    stream = torch.cuda.current_stream(device)
+
+    # pre-allocated outputs per launch (no allocation inside the timed region)
+    outs = {}
+    for name, t, cfg, kind in plan:
+        key = (name, t)
+        x = T[t]
+        if kind == "q":
+            outs[key] = mx.alloc_outputs(cfg, *x.shape, device, stats=True)
+        else:
+            src = outs[("mxfp4_row", t)]
+            outs[key] = torch.empty(x.shape, dtype=torch.bfloat16, device=device)
+            outs[(key, "src")] = src
+
+    def run_call(name, t, cfg, kind):
+        key = (name, t)
+        if kind == "q":
+            mx.quantize(T[t], cfg, out=outs[key], stream=stream)
+        else:
+            mx.dequantize(outs[(key, "src")], out=outs[key], stream=stream)
+
+    step_bytes = sum(algo_bytes(cfg, *T[t].shape, kind) for _, t, cfg, kind in plan)
+    launches = sum(launches_per_call(cfg, kind) for _, _, cfg, kind in plan)
+
+    # warm-up
+    for _ in range(args.warmup):
+        for call in plan:
+            run_call(*call)
+    torch.cuda.synchronize(device)
+
+    # timed region: events around every call (same stream)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in plan] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index) as clk:
+        start.record(stream)
+        for s in range(args.steps):
+            for i, call in enumerate(plan):
+                ev[s][i][0].record(stream)
+                run_call(*call)
+                ev[s][i][1].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize(device)
+    elapsed_ms = start.elapsed_time(stop)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+        torch.distributed.barrier()
+    ms_per_step = elapsed_ms / args.steps
+    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+
+    # per-row throughput from the events
+    rows = {}
+    for i, (name, t, cfg, kind) in enumerate(plan):
+        d = [ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)]
+        r = rows.setdefault(name, {"bytes": 0, "ms": 0.0})
+        r["bytes"] += algo_bytes(cfg, *T[t].shape, kind)
+        r["ms"] += statistics.mean(d)
+    for r in rows.values():
+        r["GB_per_s"] = round(r["bytes"] / (r["ms"] * 1e-3) / 1e9, 1)
+        r["us"] = round(r["ms"] * 1e3, 2)
+        del r["ms"]
+
+    pk, pk_src = peaks()
+    dom = rows["mxfp4_row"]
+    achieved = dom["GB_per_s"]
+    traffic = traffic_record("mxfp4_row_W")
+    roofline = {"bound": "hbm", "kernel": "k_quant_row<bf16,fast> + stats finalisation (mx_quantize MXFP4, A and W)",
+                "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk_src,
+                "traffic": traffic,
+                "algorithmic_bytes_per_launch": {"A": algo_bytes(mx.MXFP4, M_TOK, K_DIM, "q"),
+                                                 "W": algo_bytes(mx.MXFP4, N_OUT, K_DIM, "q")}}
+
+    # end to end through the public API with host buffers
+    e2e = run_e2e(mx, A_cpu, W_cpu, plan, outs, device, args, step_bytes, world)
+
+    # fidelity of the step (sanity: the stats the kernels produced)
+    fid = {f"{name}_{t}_qsnr_db": round(float(outs[(name, t)].stats[7].item()), 4)
+           for name, t, cfg, kind in plan if kind == "q"}
+
+    gemm = None if args.no_gemm else run_gemm(mx, A, W, device, args, world)
+    return dict(value=value, ms_per_step=ms_per_step, step_bytes=step_bytes, launches=launches,
+                rows=rows, roofline=roofline, e2e=e2e, fidelity=fid, gemm=gemm,
+                clocks=clk.summary())
+
+
+def run_e2e(mx, A_cpu, W_cpu, plan, outs, device, args, step_bytes, world):
+    """Same step through the public API, inputs copied from pinned host memory
+    and the codes, scales and stats read back, inside the timed region."""
+    stream = torch.cuda.current_stream(device)
+    hA = A_cpu.pin_memory()
+    hW = W_cpu.pin_memory()
+    dA = torch.empty_like(hA, device=device)
+    dW = torch.empty_like(hW, device=device)
+    T = {"A": dA, "W": dW}
+    back = []
+    for name, t, cfg, kind in plan:
+        if kind == "q":
+            o = outs[(name, t)]
+            back.append((o.codes, torch.empty(o.codes.shape, dtype=torch.uint8).pin_memory()))
+            back.append((o.scales, torch.empty(o.scales.shape, dtype=torch.uint8).pin_memory()))
+            back.append((o.stats, torch.empty(o.stats.shape, dtype=torch.float64).pin_memory()))
+    h2d = hA.numel() * 2 + hW.numel() * 2
+    d2h = sum(d.numel() * d.element_size() for d, _ in back)
+
+    def one():
+        dA.copy_(hA, non_blocking=True)
+        dW.copy_(hW, non_blocking=True)
+        for name, t, cfg, kind in plan:
+            if kind == "q":
+                mx.quantize(T[t], cfg, out=outs[(name, t)], stream=stream)
+            else:
+                mx.dequantize(outs[("mxfp4_row", t)], out=outs[(name, t)], stream=stream)
+        for d, h in back:
+            h.copy_(d, non_blocking=True)
+
+    steps = max(3, args.steps // 4)
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        one()
+    e.record(stream)
+    torch.cuda.synchronize(device)
+    ms = s.elapsed_time(e) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(world * step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3),
+            "steps": steps}
+
+
+def run_gemm(mx, A, W, device, args, world):
+    """Block-scaled FP4 GEMM C = A^Q W^Q^T (MXFP4 and NVFP4) and QSNR(AB)."""
+    out = {}
+    pk, pk_src = peaks()
+    fp4_peak = pk["bf16_tflops"] * 4.0      # nominal dense ratio fp4 : bf16 = 9 : 2.25
+    stream = torch.cuda.current_stream(device)
+    flop = 2.0 * M_TOK * N_OUT * K_DIM
+    for name, cfg in (("mxfp4", mx.MXFP4), ("nvfp4", mx.NVFP4)):
+        qa = mx.quantize(A, cfg, stats=False)
+        qw = mx.quantize(W, cfg, stats=False)
+        C = torch.empty((M_TOK, N_OUT), dtype=torch.bfloat16, device=device)
+        try:
+            mx.gemm(qa, qw, out=C, stream=stream)
+        except mx.MXError as e:
+            out[name] = {"unavailable": str(e)}
+            continue
+        for _ in range(args.warmup):
+            mx.gemm(qa, qw, out=C, stream=stream)
+        torch.cuda.synchronize(device)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        steps = max(5, args.steps)
+        s.record(stream)
+        for _ in range(steps):
+            mx.gemm(qa, qw, out=C, stream=stream)
+        e.record(stream)
+        torch.cuda.synchronize(device)
+        ms = s.elapsed_time(e) / steps
+        tf = flop / (ms * 1e-3) / 1e12
+        rec = {"TFLOPS": round(tf, 1), "ms": round(ms, 4), "unit": "TFLOP/s",
+               "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(fp4_peak, 1),
+                            "unit": "TFLOP/s", "frac": round(tf / fp4_peak, 4),
+                            "peak_source": f"{pk_src} bf16 x 4 (nominal fp4:bf16 dense ratio)"}}
+        try:
+            st = mx.gemm_qsnr(A, W, qa, qw, stream=stream)
+            torch.cuda.synchronize(device)
+            rec["qsnr_ab_db"] = round(float(st[2].item()), 4)
+        except mx.MXError as e:
+            rec["qsnr_ab"] = f"unavailable: {e}"
+        out[name] = rec
+    return out
+
+
+# ------------------------------------------------------------ CPU oracle ---
+def oracle_sample(rows_a=512, rows_w=512):
+    """The oracle on a bounded sample of the step: the first rows of A and W
+    through every launch of the step (same configs)."""
+    import oracle as O
+    import microscaling_block_quantization_b200 as mx
+    from microscaling_block_quantization_b200 import inputs
+
+    A, W = inputs.llama_linear(M_TOK, K_DIM, N_OUT)
+    T = {"A": A[:rows_a], "W": W[:rows_w]}
+    plan = step_plan(mx)
+
+    def ocfg(c):
+        return O.Cfg(elem=c.elem, scale_fmt=c.scale_fmt, rule=c.rule, oas_tau=c.oas_tau,
+                     block=c.block, axis=c.axis, round_mode=c.round, asymmetric=c.asymmetric,
+                     tensor_scale=c.tensor_scale, macro_block=c.macro_block, hadamard=c.hadamard,
+                     seed=c.seed)
+
+    nbytes = sum(algo_bytes(cfg, *T[t].shape, kind) for _, t, cfg, kind in plan)
+
+    def run():
+        keep = {}
+        for name, t, cfg, kind in plan:
+            oc = ocfg(cfg)
+            if kind == "q":
+                r = O.quantize(oc, T[t])
+                xh = O.dequantize(oc, r["packed"], r["scales"], r["tensor_scale"], r["macro"],
+                                  r["offsets"], *T[t].shape)
+                O.stats(r["y"], xh)
+                keep[(name, t)] = r
+            else:
+                r = keep[("mxfp4_row", t)]
+                O.dequantize(oc, r["packed"], r["scales"], None, None, None, *T[t].shape)
+    return run, nbytes, f"first {rows_a} rows of A and {rows_w} rows of W through every launch of the step"
+
+
+def cpu_baseline(target_s=10.0):
+    run, nbytes, sample = oracle_sample()
+    t0 = time.perf_counter()
+    run()
+    one = time.perf_counter() - t0
+    reps = max(1, int(target_s / max(one, 1e-3)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        run()
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{sample}; {reps} repetitions, {dt:.3f} s each, single-threaded scalar C"}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle, as it stands, on the host cores; each
+    step a bounded sample of the workload."""
+    if rank != 0:
+        return None
+    run, nbytes, sample = oracle_sample(rows_a=256, rows_w=256)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = nbytes / dt / 1e9
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": sample},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    r = run_ours(args, rank, world, device)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline()
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    pk, _ = peaks()
+    line = {
+        "metric": METRIC,
+        "value": round(r["value"], 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(r["ms_per_step"], 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "step": [f"{n}:{t}" for n, t, _, _ in step_plan(__import__("microscaling_block_quantization_b200"))],
+                   "step_algorithmic_bytes": r["step_bytes"], "hbm_frac_of_8TBs": round(r["value"] / world / 8000, 4),
+                   "l2": "inputs larger than L2 (A+W 176 MiB > 126 MB); consecutive launches alternate tensors",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": r["roofline"],
+        "cpu_baseline": cpu,
+        "e2e": r["e2e"],
+        "gpu_launches": r["launches"] * args.steps,
+        "clocks": r["clocks"],
+        "rows": r["rows"],
+        "gemm": r["gemm"],
+        "fidelity": r["fidelity"],
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,245 @@
+/*
+ * mx.h -- C ABI of the B200 (sm_100a) microscaling block-quantization library.
+ *
+ * Plain C: every argument is a pointer (host or device, as stated), an
+ * integer or a float.  Every call is asynchronous on the CUDA stream passed
+ * as `stream` (a cudaStream_t passed as void*, NULL = legacy default stream),
+ * returns MX_OK (0) on success or a negative MX_ERR_* code, never prints and
+ * never traps.  Arguments are validated on the host before any launch.
+ *
+ * Ownership: the caller owns every buffer.  The library allocates no device
+ * memory; scratch space ("workspace") is passed in by the caller, sized by
+ * mx_query_sizes() / mx_qsnr_workspace_bytes() / mx_gemm_workspace_bytes().
+ * Buffers must stay alive until the stream reaches the end of the call.
+ *
+ * Sources (the pages this library follows):
+ *   [MXFP4-OAS] "Unveiling the Potential of Quantization with MXFP4:
+ *               Strategies for Quantization Error Reduction" (Qiita
+ *               explainer / nubint review): Sec.2 MXFP4 and NVFP4 formats,
+ *               Sec.3 QSNR Eq. (1) and Eq. (2), Sec.4 block granularity,
+ *               Overflow-Aware Scaling (OAS), Macro Block Scaling (MBS),
+ *               Fig. 5 (the AB^T product with macro scales).
+ *   [FINER]     "Is Finer Better? The Limits of Microscaling Formats in
+ *               Large Language Models": UE4M3 / UE5M3 block scales, FP32
+ *               per-tensor scale, per-block and per-tensor MSE.
+ *   [BRIDGING]  "Bridging the Gap Between Promise and Performance for
+ *               Microscaling FP4 Quantization": block-wise Hadamard
+ *               rotation fused with quantization (sec. 2.1-2.3), block-scaled
+ *               FP4 GEMM on Blackwell (sec. 2.3).
+ *   [MX-TRAIN]  fmread summary of Yang et al., MX quantization for LLM
+ *               training (ARITH 2025): E2M1/E3M0/INT4 elements, RTNE / Ceil /
+ *               stochastic rounding, asymmetric scaling, row-wise,
+ *               column-wise and 2D blocks, R-MSE.
+ */
+#ifndef MX_H_
+#define MX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define MX_OK                0
+#define MX_ERR_INVALID      -1   /* bad pointer, shape, enum value or combination */
+#define MX_ERR_UNSUPPORTED  -2   /* valid per the pages but not implemented here */
+#define MX_ERR_ALIGN        -3   /* a pointer is not 16-byte aligned */
+#define MX_ERR_CUDA         -4   /* a CUDA launch or runtime call failed */
+#define MX_ERR_WORKSPACE    -5   /* workspace missing or too small */
+#define MX_ERR_NO_DEVICE    -6   /* no sm_100 device is current */
+#define MX_ERR_TIMEOUT      -7   /* a bounded in-kernel wait gave up (device status) */
+
+/* ---- element formats ([MXFP4-OAS] Sec.2, [MX-TRAIN]) -------------------- */
+#define MX_E2M1 0   /* FP4: magnitudes {0,0.5,1,1.5,2,3,4,6}, sign-magnitude nibble */
+#define MX_E3M0 1   /* FP4 exponent-only: {0, 2^-2 .. 2^4}, sign-magnitude nibble */
+#define MX_E2M3 2   /* FP6 (OCP MXFP6), max 7.5, one code per byte (low 6 bits) */
+#define MX_E3M2 3   /* FP6 (OCP MXFP6), max 28, one code per byte (low 6 bits) */
+#define MX_INT4 4   /* symmetric: -7..7 two's-complement nibble; asymmetric: 0..15 */
+
+/* ---- block-scale formats ([MXFP4-OAS] Sec.2, [FINER]) -------------------- */
+#define MX_SCALE_E8M0  0   /* 2^(code-127); 0xFF = NaN */
+#define MX_SCALE_UE4M3 1   /* unsigned E4M3, bias 7: 2^-9 .. 448; 0x7F = NaN */
+#define MX_SCALE_UE5M3 2   /* unsigned E5M3, bias 15: 2^-17 .. 1.75*2^16; 0xFF = NaN */
+
+/* ---- shared-scale rules ----------------------------------------------- */
+/* FLOOR: 2^(floor(log2 amax) - emax_elem) (OCP MX).  CEIL: smallest power of
+ * two with amax <= max_elem * 2^k (no overflow).  OAS: FLOOR, doubled when
+ * amax / 2^k_floor > oas_tau ([MXFP4-OAS] Sec.4).  NEAREST: UE4M3/UE5M3 scale
+ * = RTNE((amax / max_elem) / s_T), saturating (NVFP4-style).  FLOOR / CEIL /
+ * OAS with a UE4M3 / UE5M3 format store power-of-two scales in that format
+ * ([MXFP4-OAS] Sec.4: E4M3 used as power-of-two scales for block 16). */
+#define MX_RULE_FLOOR   0
+#define MX_RULE_CEIL    1
+#define MX_RULE_OAS     2
+#define MX_RULE_NEAREST 3
+
+/* ---- element rounding ([MX-TRAIN]) ------------------------------------- */
+#define MX_ROUND_RTNE       0   /* nearest, ties to the even code, saturating */
+#define MX_ROUND_CEIL       1   /* next grid point up in magnitude, saturating */
+#define MX_ROUND_STOCHASTIC 2   /* up with probability (|v|-lo)/(hi-lo); Philox4x32-10 */
+
+/* ---- block axis ([MX-TRAIN]: row-wise, column-wise, 2D) ----------------- */
+#define MX_AXIS_ROW 0   /* 1 x B blocks along a row (the contiguous dimension) */
+#define MX_AXIS_COL 1   /* B x 1 blocks along a column */
+#define MX_AXIS_2D  2   /* 32 x 32 tiles */
+
+/* ---- dtypes ------------------------------------------------------------- */
+#define MX_DT_BF16 0
+#define MX_DT_FP32 1
+
+/* ---- per-tensor FP32 scale (NVFP4, UE*-S; [FINER]) ----------------------- */
+#define MX_TS_NONE    0   /* s_T = 1 */
+#define MX_TS_COMPUTE 1   /* s_T = amax_T / (max_elem * max_scale), written to *tensor_scale */
+#define MX_TS_GIVEN   2   /* s_T read from *tensor_scale (device) */
+
+typedef struct {
+    int32_t elem;          /* MX_E2M1 ... MX_INT4 */
+    int32_t scale_fmt;     /* MX_SCALE_* */
+    int32_t rule;          /* MX_RULE_* */
+    float   oas_tau;       /* OAS threshold on amax / 2^k_floor (E2M1: 6 = ceil, 8 = floor) */
+    int32_t block;         /* elements per block along the axis: 8,16,32,64,128,256 (row);
+                              8,16,32 (col); 32 (2D) */
+    int32_t axis;          /* MX_AXIS_* */
+    int32_t round;         /* MX_ROUND_* */
+    int32_t asymmetric;    /* 1: per-block bf16 offset (INT4: min; FP: (max+min)/2) */
+    int32_t tensor_scale;  /* MX_TS_* (UE4M3/UE5M3 with MX_RULE_NEAREST only) */
+    int32_t macro_block;   /* 0 or 128: MBS macro scale per 1x128 along the axis */
+    int32_t hadamard;      /* 0, 16 or 32: block Hadamard rotation (mx_hadamard_quantize) */
+    int32_t reserved;      /* must be 0 */
+    uint64_t seed;         /* stochastic-rounding key */
+} mx_config;
+
+typedef struct {
+    int64_t codes_bytes;     /* packed element codes */
+    int64_t n_scales;        /* one byte per block */
+    int64_t n_macro;         /* one E4M3 byte per macro block (0 without MBS) */
+    int64_t n_offsets;       /* one bf16 per block (0 unless asymmetric) */
+    int64_t workspace_bytes; /* scratch for mx_quantize / mx_hadamard_quantize */
+    int64_t n_blocks;
+} mx_sizes;
+
+/* Length of every `stats` buffer (binary64, device):
+ * [0] sum x^2   [1] sum (x - x_hat)^2   [2] sum (x_hat - x)   [3] #flushed
+ * (x != 0, x_hat == 0)   [4] #nonzero x   [5] MSE   [6] R-MSE   [7] QSNR dB
+ * (Eq. (1) of [MXFP4-OAS] Sec.3)   [8] mean bias   [9] flush-to-zero share
+ * [10] element count   [11..15] reserved (0).
+ * A zero signal gives QSNR NaN; a zero error gives +inf. */
+#define MX_STATS_LEN 16
+
+/* Sizes of the outputs of mx_quantize for a rows x cols input. */
+int mx_query_sizes(const mx_config *cfg, int64_t rows, int64_t cols, mx_sizes *out);
+
+/*
+ * mx_quantize -- block quantization of a row-major rows x cols tensor
+ * ([MXFP4-OAS] Sec.2/Sec.4, [FINER], [MX-TRAIN]).
+ *   x          device, bf16 or fp32 (x_dtype), row-major, 16-byte aligned.
+ *   codes      device out.  4-bit formats: rows x cols/2 bytes, element (r, 2j)
+ *              in the low nibble of byte (r, j); FP6: rows x cols bytes.
+ *              The layout is the same for every axis.
+ *   scales     device out, one byte per block: row axis [rows][cols/B], column
+ *              axis [rows/B][cols], 2D [rows/32][cols/32].
+ *   tensor_scale  device float: written (MX_TS_COMPUTE) or read (MX_TS_GIVEN);
+ *              may be NULL with MX_TS_NONE.
+ *   macro_scales  device out, E4M3 per 1x128 macro block along the axis
+ *              (row / 2D: [rows][cols/128]; column: [rows/128][cols]); needed iff
+ *              cfg->macro_block == 128.
+ *   offsets    device out, bf16 bits per block (same layout as scales); needed
+ *              iff cfg->asymmetric.
+ *   stats      device out, MX_STATS_LEN doubles, or NULL: fidelity of the
+ *              dequantized tensor against x, fused into the same pass.
+ *   workspace  device scratch of sizes.workspace_bytes (needed when stats != NULL
+ *              or cfg->tensor_scale == MX_TS_COMPUTE).
+ * Shapes: cols % block == 0 (row), rows % block == 0 (column), both % 32 (2D),
+ * % 128 along the axis for MBS, cols % 8 == 0 always.  Block non-finite
+ * values give the NaN scale code and zero element codes.
+ */
+int mx_quantize(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t rows, int64_t cols,
+                void *codes, uint8_t *scales, float *tensor_scale, uint8_t *macro_scales,
+                uint16_t *offsets, double *stats, void *workspace, int64_t workspace_bytes,
+                void *stream);
+
+/*
+ * mx_hadamard_quantize -- mx_quantize preceded, in the same pass, by the
+ * block Hadamard rotation y = x H_n / sqrt(n), n = cfg->hadamard in {16, 32},
+ * over groups of n consecutive elements along the block axis (the row
+ * direction for 2D) ([BRIDGING] sec. 2.1-2.3: fused online rotation).
+ * Sylvester ordering, butterflies (a, b) -> (a + b, a - b) in binary32 with
+ * stride 1, 2, 4, ..., then a multiply by binary32(1/sqrt(n)).
+ * Everything (scales, stats, tensor scale) refers to y.  `rotated` (device,
+ * fp32 rows x cols, nullable) receives y.
+ */
+int mx_hadamard_quantize(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t rows,
+                         int64_t cols, void *codes, uint8_t *scales, float *tensor_scale,
+                         uint8_t *macro_scales, uint16_t *offsets, double *stats,
+                         float *rotated, void *workspace, int64_t workspace_bytes, void *stream);
+
+/*
+ * mx_dequantize -- x_hat from codes and scales ([MX-TRAIN] fake quantization).
+ * x_hat = (q * s_b) * s_T (NEAREST rule); q * 2^k (power-of-two rules), times
+ * the macro scale with MBS, plus the offset when asymmetric; each step one
+ * binary32 operation.  NaN scale codes give NaN.  With cfg->hadamard != 0 the
+ * normalised rotation (its own inverse) is applied afterwards, returning to
+ * the input space.  out: device, rows x cols, bf16 (RNE) or fp32 (out_dtype).
+ */
+int mx_dequantize(const mx_config *cfg, const void *codes, const uint8_t *scales,
+                  const float *tensor_scale, const uint8_t *macro_scales,
+                  const uint16_t *offsets, int64_t rows, int64_t cols, void *out,
+                  int32_t out_dtype, void *stream);
+
+/*
+ * mx_qsnr -- fidelity reductions of x_hat against x ([MXFP4-OAS] Sec.3 Eq. (1);
+ * [MX-TRAIN] R-MSE; [FINER] per-block MSE): stats as above, and when
+ * per_block_mse != NULL the mean squared error of every block of the given
+ * block size and axis (layout of `scales`).  x, x_hat: device, bf16 or fp32.
+ * Reduction order is fixed: results are reproducible run to run.
+ */
+int64_t mx_qsnr_workspace_bytes(int64_t rows, int64_t cols);
+int mx_qsnr(const void *x, int32_t x_dtype, const void *x_hat, int32_t x_hat_dtype, int64_t rows,
+            int64_t cols, int32_t block, int32_t axis, double *stats, float *per_block_mse,
+            void *workspace, int64_t workspace_bytes, void *stream);
+
+/*
+ * mx_gemm -- block-scaled FP4 GEMM on the tcgen05 tensor cores,
+ * C[M x N] = A^Q (B^Q)^T with FP32 accumulation ([BRIDGING] sec. 2.3;
+ * [MXFP4-OAS] Fig. 5).  A^Q: M x K E2M1 codes, B^Q: N x K E2M1 codes, both
+ * row-major along K as written by mx_quantize (row axis).  Scales in the
+ * canonical row-axis layout.  MXFP4: block 32, E8M0 (ca/cb rule FLOOR, CEIL
+ * or OAS).  NVFP4: block 16, UE4M3 NEAREST with tensor scales tsA/tsB (device
+ * floats; NULL = 1).  C: device, bf16 or fp32 (c_dtype), row-major M x N.
+ * M % 128 == 0, N % 128 == 0, K % 256 == 0.
+ */
+int mx_gemm(const mx_config *ca, const mx_config *cb, const void *Aq, const uint8_t *Asf,
+            const void *Bq, const uint8_t *Bsf, const float *tsA, const float *tsB, int64_t M,
+            int64_t N, int64_t K, void *C, int32_t c_dtype, void *stream);
+
+/*
+ * mx_gemm_qsnr -- post-operation QSNR ([MXFP4-OAS] Sec.3 Eq. (2)):
+ * 10 log10(||A B^T||_F^2 / ||A B^T - A^Q (B^Q)^T||_F^2) with A [M x K] and
+ * B [N x K] bf16 (device).  Both products are formed tile by tile on the
+ * tensor cores (bf16 with FP32 accumulation, and block-scaled FP4) and the
+ * epilogue reduces the two sums without writing C.  stats: device, 3 doubles
+ * [sum C_ref^2, sum (C_ref - C_q)^2, QSNR dB].  Shapes as mx_gemm.
+ */
+int64_t mx_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int mx_gemm_qsnr(const mx_config *ca, const mx_config *cb, const void *A, const void *B, int64_t M,
+                 int64_t N, int64_t K, const void *Aq, const uint8_t *Asf, const void *Bq,
+                 const uint8_t *Bsf, const float *tsA, const float *tsB, double *stats,
+                 void *workspace, int64_t workspace_bytes, void *stream);
+
+/* Device status word of the bounded in-kernel waits (GEMM pipeline): reads
+ * and clears it (synchronises `stream`).  *status = 0 when no wait gave up. */
+int mx_device_status(void *stream, int32_t *status);
+
+/* Human-readable text of a status code. */
+const char *mx_strerror(int code);
+
+/* Library version string. */
+const char *mx_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MX_H_ */

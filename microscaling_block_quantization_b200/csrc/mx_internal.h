@@ -1,0 +1,79 @@
+// Internal launch parameters shared by the library's translation units.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mx_device.cuh"
+
+namespace mxk {
+
+// Upper bound on the CTAs of a reducing launch: each CTA writes one partial
+// record of kPartialDoubles doubles into the caller's workspace.
+constexpr int kMaxPartials = 4096;
+constexpr int kPartialDoubles = 8;
+// workspace: [0, 256) control words (tensor amax), then the partials
+constexpr int64_t kWsHeader = 256;
+constexpr int64_t kWorkspaceBytes = kWsHeader + (int64_t)kMaxPartials * kPartialDoubles * 8;
+
+struct QParams {
+    const void *x;
+    int64_t rows, cols;
+    void *codes;
+    uint8_t *scales;
+    float *tensor_scale;     // device; read when ts_mode != TS_NONE
+    uint8_t *macro;
+    uint16_t *offsets;
+    float *rotated;          // y output (fp32), or null
+    double *partials;        // per-CTA stats records, or null (no stats)
+    unsigned int *amax_word; // tensor-amax accumulator (AMAX launches)
+    ElemDesc ed;
+    ScaleDesc sd;
+    int block;               // B
+    int lanes_per_block;     // row axis: B / 8
+    int round_mode;
+    int asym;
+    int mbs;                 // 0 / 128
+    int had;                 // 0 / 16 / 32
+    int ts_mode;
+    uint64_t seed;
+};
+
+struct DParams {
+    const void *codes;
+    const uint8_t *scales;
+    const float *tensor_scale;
+    const uint8_t *macro;
+    const uint16_t *offsets;
+    int64_t rows, cols;
+    void *out;
+    int out_fp32;
+    ElemDesc ed;
+    ScaleDesc sd;
+    int block, axis, asym, mbs, had, ts_mode;
+};
+
+struct SParams {
+    const void *x;
+    const void *xh;
+    int x_fp32, xh_fp32;
+    int64_t rows, cols;
+    int block, axis;
+    float *per_block_mse;
+    double *partials;
+};
+
+// per-launch helpers implemented in the .cu files
+int launch_quantize(const QParams &p, int axis, int in_fp32, int fast, cudaStream_t st,
+                    int *grid_out);
+int launch_tensor_amax(const QParams &p, int axis, int in_fp32, cudaStream_t st);
+int launch_finalize_tensor_scale(const QParams &p, cudaStream_t st);
+int launch_dequantize(const DParams &p, cudaStream_t st);
+int launch_qsnr(const SParams &p, cudaStream_t st, int *grid_out);
+int launch_finalize_stats(const double *partials, int nparts, double count, double *stats,
+                          cudaStream_t st);
+int device_sm_count();
+int launch_quantize_col(const QParams &p, int axis, int in_fp32, int fast, cudaStream_t st,
+                        int *grid_out);
+int launch_amax_col(const QParams &p, int in_fp32, cudaStream_t st);
+
+}  // namespace mxk

@@ -1,0 +1,212 @@
+// Device helpers shared by the quantizer kernels: vector loads, lane-group
+// reductions, the binary64 fidelity accumulators, the dequantization rule,
+// the MBS macro-scale code and the row-direction Hadamard butterflies.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <float.h>
+#include <stdint.h>
+
+#include "mx_device.cuh"
+#include "mx_internal.h"
+
+namespace mxk {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kThreads = 256;
+
+// ------------------------------------------------------------------ loads --
+__device__ __forceinline__ void unpack_bf16x2(uint32_t w, float &lo, float &hi)
+{
+    lo = __uint_as_float(w << 16);
+    hi = __uint_as_float(w & 0xffff0000u);
+}
+
+// 8 consecutive elements starting at element index e (e % 8 == 0)
+__device__ __forceinline__ void load8(const __nv_bfloat16 *x, int64_t e, float v[8])
+{
+    uint4 u = __ldg(reinterpret_cast<const uint4 *>(x + e));
+    unpack_bf16x2(u.x, v[0], v[1]);
+    unpack_bf16x2(u.y, v[2], v[3]);
+    unpack_bf16x2(u.z, v[4], v[5]);
+    unpack_bf16x2(u.w, v[6], v[7]);
+}
+__device__ __forceinline__ void load8(const float *x, int64_t e, float v[8])
+{
+    float4 a = __ldg(reinterpret_cast<const float4 *>(x + e));
+    float4 b = __ldg(reinterpret_cast<const float4 *>(x + e) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// CPT consecutive elements of one row (CPT * sizeof(T) in {8, 16} bytes)
+template <int CPT>
+__device__ __forceinline__ void load_row(const __nv_bfloat16 *x, int64_t e, float v[CPT])
+{
+    if constexpr (CPT == 8) {
+        load8(x, e, v);
+    } else {
+        uint2 u = __ldg(reinterpret_cast<const uint2 *>(x + e));
+        unpack_bf16x2(u.x, v[0], v[1]);
+        unpack_bf16x2(u.y, v[2], v[3]);
+    }
+}
+template <int CPT>
+__device__ __forceinline__ void load_row(const float *x, int64_t e, float v[CPT])
+{
+    static_assert(CPT == 4, "fp32 rows are loaded 4 at a time");
+    float4 a = __ldg(reinterpret_cast<const float4 *>(x + e));
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+
+__device__ __forceinline__ void store8f(float *y, int64_t e, const float v[8])
+{
+    reinterpret_cast<float4 *>(y + e)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4 *>(y + e)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+// ------------------------------------------------------ group reductions --
+// Reductions over aligned groups of G lanes (G a power of two, warp-uniform).
+__device__ __forceinline__ float grp_max(float v, int G)
+{
+    for (int o = 1; o < G; o <<= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+    return v;
+}
+__device__ __forceinline__ float grp_min(float v, int G)
+{
+    for (int o = 1; o < G; o <<= 1) v = fminf(v, __shfl_xor_sync(kFull, v, o));
+    return v;
+}
+__device__ __forceinline__ int grp_or(int v, int G)
+{
+    for (int o = 1; o < G; o <<= 1) v |= __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+
+__device__ __forceinline__ int nonfinite(float v) { return !(fabsf(v) <= FLT_MAX); }
+
+// ---------------------------------------------------------------- stats ----
+struct Acc {
+    double x2, e2, e, ftz, nz;
+};
+
+// binary32 sums over a handful of elements, folded into binary64
+template <int N>
+__device__ __forceinline__ void acc_add(Acc &a, const float y[N], const float xh[N])
+{
+    float sx = 0.f, se = 0.f, sb = 0.f;
+    int f = 0, z = 0;
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+        float d = y[j] - xh[j];
+        sx = fmaf(y[j], y[j], sx);
+        se = fmaf(d, d, se);
+        sb -= d;
+        int nzj = (y[j] != 0.0f);
+        z += nzj;
+        f += nzj & (xh[j] == 0.0f);
+    }
+    a.x2 += (double)sx;
+    a.e2 += (double)se;
+    a.e += (double)sb;
+    a.ftz += (double)f;
+    a.nz += (double)z;
+}
+
+__device__ __forceinline__ double warp_sum(double v)
+{
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(kFull, v, o);
+    return v;
+}
+
+// CTA reduction in a fixed order; thread 0 writes the CTA's record.
+static __device__ __noinline__ void write_partials(double *partials, const Acc &a)
+{
+    __shared__ double sh[32][5];
+    double v[5] = {a.x2, a.e2, a.e, a.ftz, a.nz};
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int i = 0; i < 5; ++i) v[i] = warp_sum(v[i]);
+    if (lane == 0)
+#pragma unroll
+        for (int i = 0; i < 5; ++i) sh[w][i] = v[i];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double s[5] = {0, 0, 0, 0, 0};
+        for (int k = 0; k < (int)(blockDim.x >> 5); ++k)
+            for (int i = 0; i < 5; ++i) s[i] += sh[k][i];
+        double *o = partials + (int64_t)blockIdx.x * kPartialDoubles;
+        for (int i = 0; i < 5; ++i) o[i] = s[i];
+        o[5] = o[6] = o[7] = 0.0;
+    }
+}
+
+// x_hat of one element from its grid value q (the dequantization rule).
+__device__ __forceinline__ float deq_value(const QParams &p, float q, const BlockScale &bs,
+                                           float sm, float o, float sT)
+{
+    if (bs.nan) return __uint_as_float(0x7fc00000u);
+    if (p.sd.fmt != S_E8M0 && p.sd.rule == R_NEAREST) return __fmul_rn(__fmul_rn(q, bs.deq), sT);
+    float v = __fmul_rn(q, bs.deq);
+    if (p.mbs) v = __fmul_rn(v, sm);
+    if (p.asym) v = __fadd_rn(v, o);
+    return v;
+}
+
+// Macro-block (MBS) scale code from the macro absmax and a non-finite flag:
+// E4M3 nearest to m / (max_elem / 2^emax), m the mantissa of the absmax.
+__device__ __forceinline__ uint32_t macro_code(const ElemDesc &ed, float amax, int bad)
+{
+    if (bad) return 0x7fu;
+    if (amax == 0.0f) return e4m3_encode_pos(1.0f);
+    int e;
+    float m;
+    frexp_exact(amax, e, m);
+    return e4m3_encode_pos(__fdiv_rn(m, __fdiv_rn(ed.maxv, (float)(1 << ed.emax))));
+}
+
+// ------------------------------------------------------------ rotation -----
+// Butterfly stages of the Sylvester-ordered fast Walsh-Hadamard transform on
+// a row chunk of 8 elements held by consecutive lanes (stride 8 and 16 are
+// across lanes), then the binary32 1/sqrt(n) multiply.
+__device__ __forceinline__ void hadamard_chunk8(float y[8], int n, int lane)
+{
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1)
+#pragma unroll
+        for (int i = 0; i < 8; i += 2 * h)
+#pragma unroll
+            for (int j = i; j < i + h; ++j) {
+                float a = y[j], b = y[j + h];
+                y[j] = __fadd_rn(a, b);
+                y[j + h] = __fsub_rn(a, b);
+            }
+    for (int m = 1; m < n / 8; m <<= 1) {
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float w = __shfl_xor_sync(kFull, y[j], m);
+            y[j] = upper ? __fsub_rn(w, y[j]) : __fadd_rn(y[j], w);
+        }
+    }
+    const float c = hadamard_scale(n);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(y[j], c);
+}
+
+
+template <typename K>
+static int grid_for(K kernel, int64_t work_warps, int threads = kThreads, size_t smem = 0)
+{
+    int occ = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, smem) != cudaSuccess || occ < 1)
+        occ = 1;
+    int64_t g = (int64_t)device_sm_count() * occ;
+    const int64_t need = (work_warps + (threads / 32) - 1) / (threads / 32);
+    if (need < g) g = need;
+    if (g < 1) g = 1;
+    if (g > kMaxPartials) g = kMaxPartials;
+    return (int)g;
+}
+
+}  // namespace mxk

@@ -1,0 +1,104 @@
+"""The C-ABI library loads, exports every entry point include/mx.h declares,
+and rejects invalid arguments on the host (no GPU needed: these calls return
+before any CUDA call)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def mx():
+    from microscaling_block_quantization_b200 import build
+    build.build()
+    import microscaling_block_quantization_b200 as m
+    m.lib()
+    return m
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(mx_[a-z_0-9]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(mx):
+    names = declared_functions()
+    assert {"mx_quantize", "mx_dequantize", "mx_hadamard_quantize", "mx_qsnr",
+            "mx_gemm_qsnr"} <= set(names)
+    L = C.CDLL(mx.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version_and_strerror(mx):
+    assert "sm_100a" in mx.mx_version()
+    assert mx.mx_strerror(0) == "ok"
+    assert "aligned" in mx.mx_strerror(-3)
+
+
+def test_query_sizes_host_only(mx):
+    s = mx.query_sizes(mx.MXFP4, 256, 256)
+    assert s.codes_bytes == 256 * 128 and s.n_scales == 256 * 8 and s.workspace_bytes > 0
+    s = mx.query_sizes(mx.NVFP4, 8192, 4096)
+    assert s.n_scales == 8192 * 256
+    s = mx.query_sizes(mx.Config(elem=mx.E2M3, axis=mx.AXIS_COL), 64, 96)
+    assert s.codes_bytes == 64 * 96 and s.n_scales == 2 * 96
+    s = mx.query_sizes(mx.Config(axis=mx.AXIS_2D, macro_block=128), 64, 256)
+    assert s.n_scales == 2 * 8 and s.n_macro == 64 * 2
+    s = mx.query_sizes(mx.Config(elem=mx.INT4, asymmetric=1, rule=mx.RULE_CEIL), 32, 64)
+    assert s.n_offsets == 64
+
+
+@pytest.mark.parametrize("cfg,rows,cols,rc", [
+    (dict(block=24), 64, 96, -2),                         # unsupported block
+    (dict(axis=2, block=16), 64, 64, -2),                 # 2D is 32 x 32
+    (dict(rule=3), 64, 64, -1),                           # NEAREST needs UE4M3/UE5M3
+    (dict(scale_fmt=1, rule=3, asymmetric=1), 64, 64, -2),
+    (dict(tensor_scale=1), 64, 64, -1),                   # tensor scale with E8M0
+    (dict(macro_block=64), 64, 128, -1),
+    (dict(macro_block=128), 64, 96, -1),                  # cols % 128
+    (dict(block=32), 64, 48, -1),                         # cols % block
+    (dict(rule=2, oas_tau=float("nan")), 64, 64, -1),
+    (dict(elem=9), 64, 64, -1),
+])
+def test_invalid_configs_rejected_on_host(mx, cfg, rows, cols, rc):
+    c = mx.Config(**cfg)
+    got = mx.mx_quantize(c, C.c_void_p(4096), 0, rows, cols, C.c_void_p(4096), C.c_void_p(4096),
+                         C.c_void_p(4096), C.c_void_p(4096), C.c_void_p(4096), None, None, 0, None)
+    assert got == rc
+
+
+def test_alignment_and_workspace_rejected_on_host(mx):
+    c = mx.MXFP4
+    P = C.c_void_p
+    assert mx.mx_quantize(c, P(4100), 0, 64, 64, P(4096), P(4096), None, None, None, None, None, 0,
+                          None) == -3
+    # stats requested without a workspace
+    assert mx.mx_quantize(c, P(4096), 0, 64, 64, P(4096), P(4096), None, None, None, P(4096), None,
+                          0, None) == -5
+    # hadamard config on the plain entry point, and the reverse
+    assert mx.mx_quantize(mx.Config(hadamard=32), P(4096), 0, 64, 64, P(4096), P(4096), None, None,
+                          None, None, None, 0, None) == -1
+    assert mx.mx_hadamard_quantize(c, P(4096), 0, 64, 64, P(4096), P(4096), None, None, None, None,
+                                   None, None, 0, None) == -1
+    # column-axis rotation longer than the block
+    assert mx.mx_hadamard_quantize(mx.Config(axis=1, block=8, hadamard=16), P(4096), 0, 64, 64,
+                                   P(4096), P(4096), None, None, None, None, None, None, 0,
+                                   None) == -2
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    import microscaling_block_quantization_b200 as m
+    monkeypatch.setattr(m, "_lib", None)
+    monkeypatch.setattr(m, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError):
+        m.lib()

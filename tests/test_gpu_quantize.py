@@ -1,0 +1,315 @@
+"""GPU parity: the sm_100a kernels (through the C ABI) against the CPU oracle.
+
+Bit-exact: packed codes, scale codes, macro-scale codes, offsets, the
+per-tensor scale, the rotated tensor and the dequantized values.
+Tolerance (binary64 sums of binary32 terms in a different order): 1e-4
+relative on the squared sums / MSE / R-MSE, 1e-3 dB on QSNR, exact counts.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from microscaling_block_quantization_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+REL = 1e-4
+
+
+@pytest.fixture(scope="module")
+def mx():
+    from microscaling_block_quantization_b200 import build
+    build.build()
+    import microscaling_block_quantization_b200 as m
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return m
+
+
+def ocfg(orc, c):
+    return orc.Cfg(elem=c.elem, scale_fmt=c.scale_fmt, rule=c.rule, oas_tau=c.oas_tau,
+                   block=c.block, axis=c.axis, round_mode=c.round, asymmetric=c.asymmetric,
+                   tensor_scale=c.tensor_scale, macro_block=c.macro_block, hadamard=c.hadamard,
+                   seed=c.seed)
+
+
+def assert_same_f32(a, b, what):
+    a = np.asarray(a, np.float32).ravel()
+    b = np.asarray(b, np.float32).ravel()
+    ab, bb = a.view(np.uint32), b.view(np.uint32)
+    nan = np.isnan(a) & np.isnan(b)
+    bad = (ab != bb) & ~nan
+    assert not bad.any(), f"{what}: {bad.sum()} mismatches, first at {np.argmax(bad)}: {a[bad][:4]} vs {b[bad][:4]}"
+
+
+def assert_stats(g, o, n):
+    g = np.asarray(g, np.float64)
+    for i in (0, 1, 5, 6):
+        if math.isnan(o[i]):
+            assert math.isnan(g[i])
+        else:
+            assert abs(g[i] - o[i]) <= REL * abs(o[i]) + 1e-300, (i, g[i], o[i])
+    if math.isfinite(o[7]):
+        assert abs(g[7] - o[7]) <= 1e-3, (g[7], o[7])
+    else:
+        assert (math.isnan(g[7]) and math.isnan(o[7])) or g[7] == o[7]
+    if math.isfinite(o[1]):
+        assert abs(g[2] - o[2]) <= 1e-6 * math.sqrt(max(n * o[1], 1e-300)) + 1e-300, (g[2], o[2])
+    assert g[3] == o[3] and g[4] == o[4] and g[10] == o[10]
+
+
+def run_case(mx, orc, x_cpu, cfg, check_stats=True, given_ts=None):
+    rows, cols = x_cpu.shape
+    x = x_cpu.cuda()
+    ts_in = None
+    if given_ts is not None:
+        ts_in = torch.tensor([given_ts], dtype=torch.float32, device="cuda")
+    q = mx.quantize(x, cfg, stats=check_stats, tensor_scale=ts_in, rotated=bool(cfg.hadamard))
+    xh = mx.dequantize(q, torch.float32)
+    torch.cuda.synchronize()
+    oc = ocfg(orc, cfg)
+    r = orc.quantize(oc, x_cpu, tensor_scale=given_ts)
+    assert np.array_equal(q.codes.cpu().numpy(), r["packed"].ravel()), "packed codes"
+    assert np.array_equal(q.scales.cpu().numpy(), r["scales"]), "scale codes"
+    if cfg.tensor_scale:
+        assert_same_f32(q.tensor_scale.cpu().numpy(), [r["tensor_scale"]], "tensor scale")
+    if cfg.macro_block:
+        assert np.array_equal(q.macro.cpu().numpy(), r["macro"]), "macro scale codes"
+    if cfg.asymmetric:
+        assert np.array_equal(q.offsets.cpu().numpy().view(np.uint16), r["offsets"]), "offsets"
+    if cfg.hadamard:
+        assert_same_f32(q.rotated.cpu().numpy(), r["y"], "rotated tensor")
+    oxh = orc.dequantize(oc, r["packed"], r["scales"], r["tensor_scale"], r["macro"],
+                         r["offsets"], rows, cols, unrotate=False)
+    if cfg.hadamard:
+        # the library rotates back on dequantize; compare against the oracle's
+        oxu = orc.dequantize(oc, r["packed"], r["scales"], r["tensor_scale"], r["macro"],
+                             r["offsets"], rows, cols, unrotate=True)
+        assert_same_f32(xh.cpu().numpy(), oxu, "dequantized (rotated back)")
+    else:
+        assert_same_f32(xh.cpu().numpy(), oxh, "dequantized")
+    if check_stats:
+        ost, _ = orc.stats(r["y"], oxh)
+        assert_stats(q.stats.cpu().numpy(), ost, rows * cols)
+    return q, r
+
+
+SHAPES = [(256, 256), (40, 544), (96, 1024)]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("block", [8, 16, 32, 64, 128, 256])
+def test_mxfp4_row_blocks(mx, orc, shape, block):
+    rows, cols = shape
+    if cols % block:
+        pytest.skip("shape not divisible by block")
+    x = inputs.laplace_outlier_cols(rows, cols, seed=4, n_outlier_cols=4)
+    run_case(mx, orc, x, mx.Config(block=block))
+
+
+def test_c1_reference_case(mx, orc):
+    """256 x 256 N(0,1) seed 0, MXFP4 floor RTNE: codes, scales, x_hat, MSE, QSNR."""
+    run_case(mx, orc, inputs.small_normal(256, 256, seed=0), mx.MXFP4)
+
+
+@pytest.mark.parametrize("rule,tau", [(1, 7.0), (2, 6.0), (2, 6.5), (2, 7.0), (2, 7.5), (2, 8.0)])
+def test_scale_rules(mx, orc, rule, tau):
+    x = inputs.laplace_outlier_cols(96, 1024, seed=4)
+    run_case(mx, orc, x, mx.Config(rule=rule, oas_tau=tau))
+
+
+@pytest.mark.parametrize("fmt,rule,ts,block", [
+    (1, 3, 1, 16),    # NVFP4: UE4M3 + computed FP32 tensor scale
+    (1, 3, 0, 16),    # UE4M3 without a tensor scale
+    (2, 3, 0, 16),    # UE5M3
+    (2, 3, 1, 8),
+    (1, 3, 0, 8),
+    (1, 0, 0, 16),    # E4M3 as power-of-two scales
+    (2, 1, 0, 32),
+    (1, 2, 0, 16),
+])
+@pytest.mark.parametrize("sigma", [0.002, 0.2])
+def test_ue_scales(mx, orc, fmt, rule, ts, block, sigma):
+    x = inputs.normal(128, 512, sigma=sigma, seed=1)
+    run_case(mx, orc, x, mx.Config(block=block, scale_fmt=fmt, rule=rule, tensor_scale=ts))
+
+
+def test_given_tensor_scale(mx, orc):
+    x = inputs.normal(64, 256, sigma=0.02, seed=2)
+    run_case(mx, orc, x, mx.Config(block=16, scale_fmt=1, rule=3, tensor_scale=2), given_ts=1.5e-5)
+
+
+@pytest.mark.parametrize("elem,rule,asym,rnd", [
+    (1, 1, 0, 0),     # E3M0 with ceil scale
+    (2, 0, 0, 0),     # E2M3
+    (3, 0, 0, 0),     # E3M2
+    (4, 0, 0, 0),     # INT4 symmetric
+    (4, 1, 1, 0),     # INT4 asymmetric min/max
+    (0, 0, 1, 0),     # E2M1 asymmetric
+    (0, 0, 0, 1),     # ceil rounding
+    (0, 0, 0, 2),     # stochastic rounding
+    (2, 0, 0, 2),
+    (4, 1, 1, 2),
+    (1, 1, 0, 1),
+])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_elements_and_rounding(mx, orc, elem, rule, asym, rnd, dtype):
+    x = inputs.gradient_like(64, 512, seed=5, dtype=dtype)
+    run_case(mx, orc, x, mx.Config(elem=elem, rule=rule, asymmetric=asym, round=rnd, seed=12345))
+
+
+@pytest.mark.parametrize("axis,block", [(1, 8), (1, 16), (1, 32), (2, 32)])
+@pytest.mark.parametrize("variant", ["plain", "oas", "mbs", "fp6", "asym", "sr", "nvfp4"])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_column_and_2d(mx, orc, axis, block, variant, dtype):
+    rows, cols = 128, 544 if variant != "mbs" else 640
+    x = inputs.laplace_outlier_cols(rows, cols, seed=4, n_outlier_cols=4, dtype=dtype)
+    kw = dict(axis=axis, block=block)
+    if variant == "oas":
+        kw.update(rule=2, oas_tau=7.0)
+    elif variant == "mbs":
+        kw.update(macro_block=128)
+    elif variant == "fp6":
+        kw.update(elem=2)
+    elif variant == "asym":
+        kw.update(elem=4, asymmetric=1, rule=1)
+    elif variant == "sr":
+        kw.update(round=2, seed=7)
+    elif variant == "nvfp4":
+        kw.update(scale_fmt=1, rule=3, tensor_scale=1)
+    run_case(mx, orc, x, mx.Config(**kw))
+
+
+@pytest.mark.parametrize("axis,block,n", [(0, 32, 32), (0, 16, 16), (0, 32, 16), (0, 16, 32),
+                                          (1, 32, 32), (1, 16, 16), (1, 32, 16), (2, 32, 32),
+                                          (2, 32, 16)])
+@pytest.mark.parametrize("extra", ["plain", "nvfp4", "mbs"])
+def test_hadamard(mx, orc, axis, block, n, extra):
+    x = inputs.laplace_outlier_cols(128, 640, seed=4, n_outlier_cols=4)
+    kw = dict(axis=axis, block=block, hadamard=n)
+    if extra == "nvfp4":
+        kw.update(scale_fmt=1, rule=3, tensor_scale=1, block=16 if axis != 2 else 32)
+        if axis == 1 and n > kw["block"]:
+            pytest.skip("column rotation longer than the block")
+    elif extra == "mbs":
+        kw.update(macro_block=128)
+    run_case(mx, orc, x, mx.Config(**kw))
+
+
+def test_mbs_row(mx, orc):
+    x = inputs.laplace_outlier_cols(128, 1024, seed=4)
+    for block in (8, 16, 32, 64, 128):
+        run_case(mx, orc, x, mx.Config(block=block, macro_block=128))
+        run_case(mx, orc, x, mx.Config(block=block, macro_block=128, rule=2))
+
+
+# ------------------------------------------------------------- edge cases ----
+def test_special_values(mx, orc):
+    """NaN / Inf blocks, all-zero blocks, signed zeros, bf16 extremes and
+    subnormals, every bf16 bit pattern."""
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(2048, 32)
+    x = torch.from_numpy(pats.view(np.int16)).view(torch.bfloat16)
+    for cfg in (dict(), dict(rule=1), dict(rule=2), dict(elem=2), dict(elem=3), dict(elem=1, rule=1),
+                dict(elem=4), dict(round=1), dict(round=2, seed=3)):
+        run_case(mx, orc, x, mx.Config(**cfg), check_stats=False)
+    x16 = torch.from_numpy(pats.reshape(4096, 16).view(np.int16)).view(torch.bfloat16)
+    for cfg in (dict(block=16, scale_fmt=1, rule=3), dict(block=16, scale_fmt=2, rule=3),
+                dict(block=16, scale_fmt=1, rule=0)):
+        run_case(mx, orc, x16, mx.Config(**cfg), check_stats=False)
+
+
+def test_zeros_and_empty(mx, orc):
+    z = torch.zeros(64, 256, dtype=torch.bfloat16)
+    q, _ = run_case(mx, orc, z, mx.MXFP4)
+    st = q.stats.cpu().numpy()
+    assert math.isnan(st[7]) and st[5] == 0
+    e = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    q = mx.quantize(e, mx.MXFP4)
+    st = q.stats.cpu().numpy()
+    assert st[10] == 0 and math.isnan(st[7])
+
+
+def test_fast_path_conversion_rounding(mx):
+    """The E2M1 conversion instruction used by the fast path, swept over
+    [-7.5, 7.5] with the block scale pinned to 1: every code is the nearest
+    grid point (ties to the even code), saturating at 6, sign kept."""
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+    v = np.linspace(-7.5, 7.5, 32 * 2048, dtype=np.float32).reshape(2048, 32)
+    v[:, 0] = 6.0                                   # fixes every block scale to 1
+    q = mx.quantize(torch.from_numpy(v).cuda(), mx.MXFP4, stats=False)
+    codes = q.codes.cpu().numpy()
+    lo, hi = codes & 0xF, codes >> 4
+    c = np.stack([lo, hi], axis=-1).reshape(2048, 32)
+    mag = np.abs(v.astype(np.float64))
+    d = np.abs(mag[..., None] - grid)
+    best = np.argmin(d, axis=-1)
+    ties = (np.sort(d, axis=-1)[..., 0] == np.sort(d, axis=-1)[..., 1])
+    best = np.where(ties & (best % 2 == 1), best + 1, best)
+    best = np.minimum(best, 7)
+    want = best | ((np.signbit(v)).astype(np.int64) << 3)
+    assert np.array_equal(c, want)
+
+
+# ------------------------------------------------------- standalone qsnr ----
+@pytest.mark.parametrize("axis,block", [(0, 32), (0, 8), (0, 256), (1, 16), (1, 32), (2, 32)])
+def test_qsnr_and_per_block_mse(mx, orc, axis, block):
+    x = inputs.laplace_outlier_cols(128, 512, seed=4)
+    q = mx.quantize(x.cuda(), mx.Config(axis=axis, block=block), stats=False)
+    xh = mx.dequantize(q, torch.float32)
+    st, pb = mx.qsnr(x.cuda(), xh, block=block, axis=axis, per_block=True)
+    ost, opb = orc.stats(orc.input_f32(x), xh.cpu().numpy(), block=block, axis=axis)
+    assert_stats(st.cpu().numpy(), ost, x.numel())
+    assert np.allclose(pb.cpu().numpy(), opb, rtol=1e-5, atol=1e-30)
+    xb = mx.dequantize(q, torch.bfloat16)
+    assert torch.equal(xb.cpu(), xh.cpu().to(torch.bfloat16))
+    st2, _ = mx.qsnr(x.cuda(), xb)
+    ost2, _ = orc.stats(orc.input_f32(x), orc.input_f32(xb.cpu()))
+    assert_stats(st2.cpu().numpy(), ost2, x.numel())
+
+
+def test_stats_reproducible(mx):
+    x = inputs.laplace_outlier_cols(512, 1024, seed=4).cuda()
+    a = mx.quantize(x, mx.MXFP4).stats.cpu().numpy()
+    b = mx.quantize(x, mx.MXFP4).stats.cpu().numpy()
+    assert np.array_equal(a, b)
+
+
+# ------------------------------------------------------ full-size configs ----
+@pytest.mark.parametrize("name", ["c3_row", "c3_col", "c3_2d", "c3_mbs", "c3_had", "c3_oas"])
+def test_activation_config_full_size(mx, orc, name):
+    """8192 x 4096 Laplace activations with 16 outlier columns: every output
+    against the oracle at full size, in the launch configuration of the
+    benchmark."""
+    x = _c3()
+    cfg = {"c3_row": mx.MXFP4, "c3_col": mx.Config(axis=1), "c3_2d": mx.Config(axis=2),
+           "c3_mbs": mx.Config(macro_block=128), "c3_had": mx.Config(hadamard=32),
+           "c3_oas": mx.Config(rule=2, oas_tau=7.0)}[name]
+    run_case(mx, orc, x, cfg)
+
+
+_C3 = {}
+
+
+def _c3():
+    if "x" not in _C3:
+        _C3["x"] = inputs.laplace_outlier_cols(8192, 4096, seed=4)
+    return _C3["x"]
+
+
+def test_gradient_config_full_size(mx, orc):
+    """4096 x 14336 fp32 gradients with 1% large entries, stochastic rounding
+    (Philox keyed on the seed and the element index): codes and scales against
+    the oracle at full size; the sampled 256 rows also through dequantize."""
+    x = inputs.gradient_like(4096, 14336, seed=5)
+    cfg = mx.Config(round=2, seed=5)
+    q = mx.quantize(x.cuda(), cfg)
+    full = orc.quantize(ocfg(orc, cfg), x)
+    assert np.array_equal(q.codes.cpu().numpy(), full["packed"].ravel())
+    assert np.array_equal(q.scales.cpu().numpy(), full["scales"])
+    rows = np.random.default_rng(0).choice(4096, 256, replace=False)
+    xh = mx.dequantize(q, torch.float32).cpu().numpy()
+    oxh = orc.dequantize(ocfg(orc, cfg), full["packed"], full["scales"], None, None, None,
+                         4096, 14336)
+    assert_same_f32(xh[rows], oxh[rows], "dequantized sample")
