@@ -197,24 +197,39 @@ def run_ours(args, rank, world, device):
             outs[(key, "src")] = src
 
     def run_call(name, t, cfg, kind):
+        # stream=None: the current stream, i.e. the capture stream inside a graph
         key = (name, t)
         if kind == "q":
-            mx.quantize(T[t], cfg, out=outs[key], stream=stream)
+            mx.quantize(T[t], cfg, out=outs[key])
         else:
-            mx.dequantize(outs[(key, "src")], out=outs[key], stream=stream)
+            mx.dequantize(outs[(key, "src")], out=outs[key])
 
     step_bytes = sum(algo_bytes(cfg, *T[t].shape, kind) for _, t, cfg, kind in plan)
     launches = sum(launches_per_call(cfg, kind) for _, _, cfg, kind in plan)
 
-    # warm-up
-    for _ in range(args.warmup):
+    # eager warm-up (allocates the workspace, caches kernel attributes)
+    for _ in range(max(1, args.warmup)):
         for call in plan:
             run_call(*call)
     torch.cuda.synchronize(device)
 
-    # timed region: events around every call (same stream)
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in plan] for _ in range(args.steps)]
+    # the step, and every launch of it, captured as CUDA graphs: the kernels
+    # run back to back with no host work between them
+    step_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(step_graph):
+        for call in plan:
+            run_call(*call)
+    call_graphs = []
+    for call in plan:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run_call(*call)
+        call_graphs.append(g)
+    for _ in range(args.warmup):
+        step_graph.replay()
+    torch.cuda.synchronize(device)
+
+    # timed region: exactly K steps between CUDA events on the replay stream
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
@@ -222,10 +237,7 @@ def run_ours(args, rank, world, device):
     with ClockSampler(device.index) as clk:
         start.record(stream)
         for s in range(args.steps):
-            for i, call in enumerate(plan):
-                ev[s][i][0].record(stream)
-                run_call(*call)
-                ev[s][i][1].record(stream)
+            step_graph.replay()
         stop.record(stream)
         torch.cuda.synchronize(device)
     elapsed_ms = start.elapsed_time(stop)
@@ -237,13 +249,21 @@ def run_ours(args, rank, world, device):
     ms_per_step = elapsed_ms / args.steps
     value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
 
-    # per-row throughput from the events
+    # per-launch device time: each launch's graph replayed K times between
+    # events (inputs larger than L2, the same launch configuration as the step)
     rows = {}
     for i, (name, t, cfg, kind) in enumerate(plan):
-        d = [ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)]
+        g = call_graphs[i]
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
         r = rows.setdefault(name, {"bytes": 0, "ms": 0.0})
         r["bytes"] += algo_bytes(cfg, *T[t].shape, kind)
-        r["ms"] += statistics.mean(d)
+        r["ms"] += e0.elapsed_time(e1) / args.steps
     for r in rows.values():
         r["GB_per_s"] = round(r["bytes"] / (r["ms"] * 1e-3) / 1e9, 1)
         r["us"] = round(r["ms"] * 1e3, 2)
@@ -332,23 +352,28 @@ def run_gemm(mx, A, W, device, args, world):
     fp4_peak = pk["bf16_tflops"] * 4.0      # nominal dense ratio fp4 : bf16 = 9 : 2.25
     stream = torch.cuda.current_stream(device)
     flop = 2.0 * M_TOK * N_OUT * K_DIM
-    for name, cfg in (("mxfp4", mx.MXFP4), ("nvfp4", mx.NVFP4)):
+    for name, cfg in (("mxfp4", mx.Config(sf_layout=1)),
+                      ("nvfp4", mx.Config(block=16, scale_fmt=1, rule=3, tensor_scale=1, sf_layout=1))):
         qa = mx.quantize(A, cfg, stats=False)
         qw = mx.quantize(W, cfg, stats=False)
         C = torch.empty((M_TOK, N_OUT), dtype=torch.bfloat16, device=device)
         try:
-            mx.gemm(qa, qw, out=C, stream=stream)
+            mx.gemm(qa, qw, out=C)
         except mx.MXError as e:
             out[name] = {"unavailable": str(e)}
             continue
         for _ in range(args.warmup):
-            mx.gemm(qa, qw, out=C, stream=stream)
+            mx.gemm(qa, qw, out=C)
         torch.cuda.synchronize(device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            mx.gemm(qa, qw, out=C)
+        g.replay()
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         steps = max(5, args.steps)
         s.record(stream)
         for _ in range(steps):
-            mx.gemm(qa, qw, out=C, stream=stream)
+            g.replay()
         e.record(stream)
         torch.cuda.synchronize(device)
         ms = s.elapsed_time(e) / steps
@@ -358,9 +383,15 @@ def run_gemm(mx, A, W, device, args, world):
                             "unit": "TFLOP/s", "frac": round(tf / fp4_peak, 4),
                             "peak_source": f"{pk_src} bf16 x 4 (nominal fp4:bf16 dense ratio)"}}
         try:
-            st = mx.gemm_qsnr(A, W, qa, qw, stream=stream)
+            st = mx.gemm_qsnr(A, W, qa, qw)
+            torch.cuda.synchronize(device)
+            s.record(stream)
+            st = mx.gemm_qsnr(A, W, qa, qw)
+            e.record(stream)
             torch.cuda.synchronize(device)
             rec["qsnr_ab_db"] = round(float(st[2].item()), 4)
+            rec["qsnr_ab_ms"] = round(s.elapsed_time(e), 3)
+            rec["device_status"] = mx.mx_device_status()
         except mx.MXError as e:
             rec["qsnr_ab"] = f"unavailable: {e}"
         out[name] = rec

@@ -107,7 +107,11 @@ typedef struct {
     int32_t tensor_scale;  /* MX_TS_* (UE4M3/UE5M3 with MX_RULE_NEAREST only) */
     int32_t macro_block;   /* 0 or 128: MBS macro scale per 1x128 along the axis */
     int32_t hadamard;      /* 0, 16 or 32: block Hadamard rotation (mx_hadamard_quantize) */
-    int32_t reserved;      /* must be 0 */
+    int32_t sf_layout;     /* scales layout: 0 canonical (below); 1 tcgen05 chunks (row axis
+                              only; rows % 128 == 0, (cols / block) % 4 == 0): for row r and
+                              scale j of a row holding S = cols / block scales, byte
+                              ((r/128)*(S/4) + j/4)*512 + (r%32)*16 + ((r/32)%4)*4 + j%4,
+                              the layout mx_gemm copies into tensor memory */
     uint64_t seed;         /* stochastic-rounding key */
 } mx_config;
 
@@ -139,7 +143,8 @@ int mx_query_sizes(const mx_config *cfg, int64_t rows, int64_t cols, mx_sizes *o
  *              in the low nibble of byte (r, j); FP6: rows x cols bytes.
  *              The layout is the same for every axis.
  *   scales     device out, one byte per block: row axis [rows][cols/B], column
- *              axis [rows/B][cols], 2D [rows/32][cols/32].
+ *              axis [rows/B][cols], 2D [rows/32][cols/32] (cfg->sf_layout == 0), or
+ *              the tcgen05 chunk layout (cfg->sf_layout == 1, row axis).
  *   tensor_scale  device float: written (MX_TS_COMPUTE) or read (MX_TS_GIVEN);
  *              may be NULL with MX_TS_NONE.
  *   macro_scales  device out, E4M3 per 1x128 macro block along the axis

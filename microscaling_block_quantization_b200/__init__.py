@@ -44,7 +44,7 @@ class mx_config(C.Structure):
     _fields_ = [("elem", C.c_int32), ("scale_fmt", C.c_int32), ("rule", C.c_int32),
                 ("oas_tau", C.c_float), ("block", C.c_int32), ("axis", C.c_int32),
                 ("round", C.c_int32), ("asymmetric", C.c_int32), ("tensor_scale", C.c_int32),
-                ("macro_block", C.c_int32), ("hadamard", C.c_int32), ("reserved", C.c_int32),
+                ("macro_block", C.c_int32), ("hadamard", C.c_int32), ("sf_layout", C.c_int32),
                 ("seed", C.c_uint64)]
 
 
@@ -68,11 +68,12 @@ class Config:
     macro_block: int = 0
     hadamard: int = 0
     seed: int = 0
+    sf_layout: int = 0
 
     def c(self) -> mx_config:
         return mx_config(self.elem, self.scale_fmt, self.rule, self.oas_tau, self.block,
                          self.axis, self.round, self.asymmetric, self.tensor_scale,
-                         self.macro_block, self.hadamard, 0, self.seed)
+                         self.macro_block, self.hadamard, self.sf_layout, self.seed)
 
 
 MXFP4 = Config()

@@ -67,7 +67,8 @@ int check_config(const mx_config *c, int64_t rows, int64_t cols, bool want_had)
 {
     if (!c) return MX_ERR_INVALID;
     if (rows < 0 || cols < 0) return MX_ERR_INVALID;
-    if (c->reserved != 0) return MX_ERR_INVALID;
+    if (c->sf_layout != 0 && c->sf_layout != 1) return MX_ERR_INVALID;
+    if (c->sf_layout == 1 && c->axis != MX_AXIS_ROW) return MX_ERR_UNSUPPORTED;
     if (c->elem < MX_E2M1 || c->elem > MX_INT4) return MX_ERR_INVALID;
     if (c->scale_fmt < MX_SCALE_E8M0 || c->scale_fmt > MX_SCALE_UE5M3) return MX_ERR_INVALID;
     if (c->rule < MX_RULE_FLOOR || c->rule > MX_RULE_NEAREST) return MX_ERR_INVALID;
@@ -107,6 +108,7 @@ int check_config(const mx_config *c, int64_t rows, int64_t cols, bool want_had)
     if (rows == 0 || cols == 0) return MX_OK;
     if (cols % 8) return MX_ERR_INVALID;
     if (c->axis == MX_AXIS_ROW && cols % B) return MX_ERR_INVALID;
+    if (c->sf_layout == 1 && (rows % 128 || (cols / B) % 4)) return MX_ERR_INVALID;
     if (c->axis == MX_AXIS_COL && rows % B) return MX_ERR_INVALID;
     if (c->axis == MX_AXIS_2D && (rows % 32 || cols % 32)) return MX_ERR_INVALID;
     if (c->macro_block) {
@@ -190,6 +192,7 @@ int quantize_impl(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t 
     p.had = cfg->hadamard;
     p.ts_mode = cfg->tensor_scale;
     p.seed = cfg->seed;
+    p.sf_gemm = cfg->sf_layout;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     p.amax_word = ws ? reinterpret_cast<unsigned int *>(ws) : nullptr;
     double *partials = ws ? reinterpret_cast<double *>(ws + kWsHeader) : nullptr;
@@ -295,6 +298,7 @@ int mx_dequantize(const mx_config *cfg, const void *codes, const uint8_t *scales
     p.mbs = cfg->macro_block;
     p.had = cfg->hadamard;
     p.ts_mode = cfg->tensor_scale;
+    p.sf_gemm = cfg->sf_layout;
     return launch_dequantize(p, static_cast<cudaStream_t>(stream)) ? MX_ERR_CUDA : MX_OK;
 }
 

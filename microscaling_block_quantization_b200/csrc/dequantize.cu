@@ -149,7 +149,13 @@ __global__ void __launch_bounds__(kThreads) k_dequant_chunk(const DParams p)
             } else {
                 const int64_t b = (p.axis == AX_ROW) ? e0 / p.block
                                                      : (row / 32) * (p.cols / 32) + col0 / 32;
-                const uint32_t s = p.scales[b];
+                uint32_t s;
+                if (p.axis == AX_ROW && p.sf_gemm) {
+                    const int64_t S = p.cols / p.block;
+                    s = p.scales[sf_chunk_index(row, col0 / p.block, S)];
+                } else {
+                    s = p.scales[b];
+                }
                 const uint16_t o = p.asym ? p.offsets[b] : 0;
                 const uint32_t m = p.mbs ? p.macro[row * (p.cols / 128) + col0 / 128] : 0u;
 #pragma unroll
@@ -394,9 +400,7 @@ __global__ void __launch_bounds__(kThreads) k_qsnr_blocks_col(const SParams p)
 template <typename K>
 int grid_of(K kernel, int64_t work_warps)
 {
-    int occ = 1;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kThreads, 0) != cudaSuccess || occ < 1)
-        occ = 1;
+    const int occ = cached_occupancy(reinterpret_cast<const void *>(kernel), kThreads, 0);
     int64_t g = (int64_t)device_sm_count() * occ;
     const int64_t need = (work_warps + (kThreads / 32) - 1) / (kThreads / 32);
     if (need < g) g = need;

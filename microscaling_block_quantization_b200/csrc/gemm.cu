@@ -1,24 +1,541 @@
-// Block-scaled FP4 GEMM entry points (tcgen05 kernel in progress).
+// Block-scaled FP4 GEMM on the sm_100a 5th-generation tensor cores, and the
+// post-operation QSNR of "Unveiling the Potential of Quantization with MXFP4"
+// (Sec.3 Eq. (2)); the product is the A B^T of the same page's Fig. 5 (MBS
+// matrix multiply), the Blackwell FP4 GEMM of "Bridging the Gap ...
+// Microscaling FP4 Quantization" (sec. 2.3).
+//
+// One CTA computes a 128 x 128 tile of C = A^Q (B^Q)^T with FP32 accumulation
+// in tensor memory:
+//   warp 0       TMA producer: 2-D tensor copies of the packed E2M1 (or bf16)
+//                tiles with 128-byte swizzle, 1-D bulk copies of the scale
+//                chunks (512-byte 128-row x 4-scale chunks, written in that
+//                layout by the quantizer), one mbarrier per stage;
+//   warp 1       tensor memory owner and MMA issuer: tcgen05.cp of the scale
+//                chunks into tensor memory, tcgen05.mma kind::mxf4 (E8M0,
+//                32-element blocks) / kind::mxf4nvf4 (UE4M3, 16-element
+//                blocks) / kind::f16 (bf16), tcgen05.commit to free stages;
+//   warps 2..5   epilogue: tcgen05.ld of the accumulator lanes of their
+//                quadrant, per-tensor scales, and either the C store or the
+//                QSNR sums against a previously computed C_q.
+// No TMA multicast anywhere; every wait on an mbarrier is bounded and sets a
+// device status word instead of hanging.
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "mx.h"
+#include "mx_internal.h"
+
+namespace mxg {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int kStages = 3;
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 256;
+constexpr int kTileBytes = BM * 128;              // one operand tile: 128 rows x 128 bytes
+constexpr uint64_t kWaitNs = 2000000000ull;       // bound of one mbarrier wait: 2 s
+
+enum { KIND_BF16 = 0, KIND_MXF4 = 1, KIND_NVF4 = 2 };
+enum { EPI_BF16 = 0, EPI_F32 = 1, EPI_QSNR = 2 };
+
+// device status word of the bounded waits (read and cleared by mx_device_status)
+__device__ int g_status;
+
+struct GParams {
+    int M, N, K;
+    const uint8_t *sfa, *sfb;    // scale chunks (FP4 kinds)
+    const float *tsA, *tsB;      // per-tensor scales or null
+    void *C;                     // EPI_BF16 / EPI_F32 output, row-major M x N
+    const float *Cq;             // EPI_QSNR: the quantized product, fp32 M x N
+    double *partials;            // EPI_QSNR: per-CTA [sum C^2, sum (C - Cq)^2]
+};
+
+template <int KIND>
+struct Kind {
+    static constexpr int kChunks = KIND == KIND_MXF4 ? 2 : KIND == KIND_NVF4 ? 4 : 0;  // per stage
+    static constexpr int kSfBytes = kChunks * 512;                                    // per operand
+    static constexpr int kKPerStage = KIND == KIND_BF16 ? 64 : 256;                   // elements
+    static constexpr int kStageBytes = 2 * kTileBytes + 2 * kSfBytes;
+    static constexpr int kSfCols = 2 * kChunks * 4;                                   // TMEM columns
+};
+
+// ------------------------------------------------------------ primitives --
+__device__ __forceinline__ uint32_t saddr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t phase)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(saddr(bar)), "r"(phase) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t now_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait: false (and the status word set) once kWaitNs have passed.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase, int where)
+{
+    if (mbar_try(bar, phase)) return true;
+    const uint64_t t0 = now_ns();
+    while (true) {
+        if (mbar_try(bar, phase)) return true;
+        if (now_ns() - t0 > kWaitNs) break;
+    }
+    atomicCAS(&g_status, 0, where);
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%3, %4}], [%2];"
+                 ::"r"(saddr(dst)), "l"((uint64_t)map), "r"(saddr(bar)), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(saddr(dst)), "l"(src), "r"(bytes), "r"(saddr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(saddr(bar)) : "memory");
+}
+
+// K-major operand tile with 128-byte swizzle: 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr)
+{
+    uint64_t d = (uint64_t)((addr >> 4) & 0x3fffu);
+    d |= (uint64_t)1 << 16;                  // leading byte offset (16 B units; unused by SW128 K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;        // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1 << 46;                  // descriptor version (sm100)
+    d |= (uint64_t)2 << 61;                  // SWIZZLE_128B
+    return d;
+}
+// 32 rows x 16 bytes, unswizzled (a scale chunk): 8-row groups 128 bytes apart.
+__device__ __forceinline__ uint64_t desc_sf(uint32_t addr)
+{
+    uint64_t d = (uint64_t)((addr >> 4) & 0x3fffu);
+    d |= (uint64_t)(128 >> 4) << 16;
+    d |= (uint64_t)(128 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
+}
+
+// Instruction descriptors (M = 128, N = BN, K-major operands, FP32 accumulate).
+template <int KIND>
+__device__ __forceinline__ uint32_t idesc_base()
+{
+    uint32_t d = 0;
+    if (KIND == KIND_BF16) {
+        d |= 1u << 4;      // accumulator F32
+        d |= 1u << 7;      // A bf16
+        d |= 1u << 10;     // B bf16
+    } else {
+        d |= 1u << 7;      // A E2M1
+        d |= 1u << 10;     // B E2M1
+        if (KIND == KIND_MXF4) d |= 1u << 23;   // scales UE8M0 (UE4M3 = 0)
+    }
+    d |= (uint32_t)(BN >> 3) << 17;
+    d |= (uint32_t)(BM >> 4) << 24;
+    return d;
+}
+
+template <int KIND>
+__device__ __forceinline__ void mma(uint32_t dt, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t sfa,
+                                    uint32_t sfb, uint32_t acc)
+{
+    if constexpr (KIND == KIND_BF16) {
+        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+                     ::"r"(dt), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(0), "r"(0), "r"(0), "r"(0));
+        (void)sfa;
+        (void)sfb;
+    } else if constexpr (KIND == KIND_MXF4) {
+        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+                     ::"r"(dt), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
+    } else {
+        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+                     ::"r"(dt), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
+    }
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float v[32])
+{
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32"
+                 " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
+                 " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+                   "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+                   "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+                   "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+                   "=r"(r[31])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---------------------------------------------------------------- kernel --
+template <int KIND, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm(const GParams p, const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB)
+{
+    using KT = Kind<KIND>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *sA = smem;                                   // kStages x 16 KB
+    uint8_t *sB = sA + kStages * kTileBytes;              // kStages x 16 KB
+    uint8_t *sSFA = sB + kStages * kTileBytes;            // kStages x kSfBytes
+    uint8_t *sSFB = sSFA + kStages * KT::kSfBytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sSFB + kStages * KT::kSfBytes);
+    uint64_t *empty = full + kStages;
+    uint64_t *accf = empty + kStages;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(accf + 1);
+    double *red = reinterpret_cast<double *>(tmem_holder + 4);   // 4 warps x 2 sums
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+    const int ktiles = p.K / KT::kKPerStage;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accf, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(saddr(tmem_holder)), "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_holder;
+    const uint32_t tsf = tbase + BN;                      // scale-factor ring after the accumulator
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const int sfrow_chunks = (p.K / (KIND == KIND_MXF4 ? 32 : 16)) / 4;   // chunks per 128 rows
+            for (int kt = 0; kt < ktiles; ++kt) {
+                const int s = kt % kStages;
+                if (kt >= kStages && !mbar_wait(&empty[s], ((kt / kStages) - 1) & 1, 1)) break;
+                mbar_expect_tx(&full[s], KT::kStageBytes);
+                const int kx = KIND == KIND_BF16 ? kt * 64 : kt * 128;    // elements (bf16) / bytes (FP4)
+                tma_load_2d(sA + s * kTileBytes, &tmA, &full[s], kx, m0);
+                tma_load_2d(sB + s * kTileBytes, &tmB, &full[s], kx, n0);
+                if constexpr (KIND != KIND_BF16) {
+                    const size_t ca = ((size_t)(m0 / 128) * sfrow_chunks + (size_t)kt * KT::kChunks) * 512;
+                    const size_t cb = ((size_t)(n0 / 128) * sfrow_chunks + (size_t)kt * KT::kChunks) * 512;
+                    bulk_load(sSFA + s * KT::kSfBytes, p.sfa + ca, KT::kSfBytes, &full[s]);
+                    bulk_load(sSFB + s * KT::kSfBytes, p.sfb + cb, KT::kSfBytes, &full[s]);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc0 = idesc_base<KIND>();
+            bool ok = true;
+            for (int kt = 0; kt < ktiles; ++kt) {
+                const int s = kt % kStages;
+                if (!mbar_wait(&full[s], (kt / kStages) & 1, 2)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t sfa_t = tsf + s * KT::kSfCols;           // this stage's scale columns
+                const uint32_t sfb_t = sfa_t + KT::kChunks * 4;
+                if constexpr (KIND != KIND_BF16) {
+#pragma unroll
+                    for (int c = 0; c < KT::kChunks; ++c) {
+                        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                                     ::"r"(sfa_t + 4 * c), "l"(desc_sf(saddr(sSFA + s * KT::kSfBytes + c * 512))));
+                        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                                     ::"r"(sfb_t + 4 * c), "l"(desc_sf(saddr(sSFB + s * KT::kSfBytes + c * 512))));
+                    }
+                }
+                const uint32_t a0 = saddr(sA + s * kTileBytes), b0 = saddr(sB + s * kTileBytes);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    // each MMA covers 32 bytes of the 128-byte row: K = 64 (FP4) or 16 (bf16)
+                    uint32_t idesc = idesc0, sfa = 0, sfb = 0;
+                    if constexpr (KIND == KIND_MXF4) {
+                        const uint32_t id = (k & 1) * 2;                 // byte of the 4-scale word
+                        idesc |= (id << 29) | (id << 4);
+                        sfa = sfa_t + 4 * (k >> 1);
+                        sfb = sfb_t + 4 * (k >> 1);
+                    } else if constexpr (KIND == KIND_NVF4) {
+                        sfa = sfa_t + 4 * k;
+                        sfb = sfb_t + 4 * k;
+                    }
+                    mma<KIND>(tbase, desc_sw128(a0 + 32 * k), desc_sw128(b0 + 32 * k), idesc, sfa, sfb,
+                              (kt > 0 || k > 0) ? 1u : 0u);
+                }
+                tc_commit(&empty[s]);
+            }
+            if (ok) tc_commit(accf);
+        }
+        __syncwarp();
+    } else {
+        // epilogue: warp w reads accumulator lanes 32 * (w % 4) .. + 31
+        const int q = warp & 3;
+        const int row = m0 + 32 * q + lane;
+        const bool ready = mbar_wait(accf, 0, 3);
+        tc_fence_after();
+        float scale = 1.0f;
+        if (p.tsA) scale = __fmul_rn(scale, *p.tsA);
+        if (p.tsB) scale = __fmul_rn(scale, *p.tsB);
+        double s_ref = 0.0, s_err = 0.0;
+        if (ready) {
+#pragma unroll 1
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                float v[32];
+                tmem_ld32(tbase + ((uint32_t)(32 * q) << 16) + ch * 32, v);
+                const int col = n0 + ch * 32;
+                if constexpr (EPI == EPI_BF16) {
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.C) + (size_t)row * p.N + col;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            w[j] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[i + 2 * j] * scale)) |
+                                   ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[i + 2 * j + 1] * scale)) << 16);
+                        *reinterpret_cast<uint4 *>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                } else if constexpr (EPI == EPI_F32) {
+                    float *dst = static_cast<float *>(p.C) + (size_t)row * p.N + col;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4 *>(dst + i) =
+                            make_float4(v[i] * scale, v[i + 1] * scale, v[i + 2] * scale, v[i + 3] * scale);
+                } else {
+                    const float *cq = p.Cq + (size_t)row * p.N + col;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        const float4 c4 = *reinterpret_cast<const float4 *>(cq + i);
+                        const float cr[4] = {v[i] * scale, v[i + 1] * scale, v[i + 2] * scale, v[i + 3] * scale};
+                        const float cqv[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const double a = (double)cr[j], d = a - (double)cqv[j];
+                            s_ref += a * a;
+                            s_err += d * d;
+                        }
+                    }
+                }
+            }
+        }
+        if constexpr (EPI == EPI_QSNR) {
+            for (int o = 16; o > 0; o >>= 1) {
+                s_ref += __shfl_down_sync(0xffffffffu, s_ref, o);
+                s_err += __shfl_down_sync(0xffffffffu, s_err, o);
+            }
+            if (lane == 0) {
+                red[2 * (warp - 2)] = s_ref;
+                red[2 * (warp - 2) + 1] = s_err;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if constexpr (EPI == EPI_QSNR) {
+        if (threadIdx.x == 0) {
+            double a = 0.0, b = 0.0;
+            for (int w = 0; w < 4; ++w) { a += red[2 * w]; b += red[2 * w + 1]; }
+            double *o = p.partials + 2 * ((size_t)blockIdx.y * gridDim.x + blockIdx.x);
+            o[0] = a;
+            o[1] = b;
+        }
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(kTmemCols));
+    }
+}
+
+// Sum the per-CTA records in a fixed order: [sum C_ref^2, sum err^2, QSNR dB].
+__global__ void k_gemm_qsnr_finalize(const double *partials, int n, double *out)
+{
+    __shared__ double sh[256][2];
+    double a = 0.0, b = 0.0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        a += partials[2 * i];
+        b += partials[2 * i + 1];
+    }
+    sh[threadIdx.x][0] = a;
+    sh[threadIdx.x][1] = b;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+        if ((int)threadIdx.x < w) {
+            sh[threadIdx.x][0] += sh[threadIdx.x + w][0];
+            sh[threadIdx.x][1] += sh[threadIdx.x + w][1];
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const double r = sh[0][0], e = sh[0][1];
+        out[0] = r;
+        out[1] = e;
+        out[2] = (r == 0.0) ? __longlong_as_double(0x7ff8000000000000ll)
+               : (e == 0.0) ? __longlong_as_double(0x7ff0000000000000ll)
+                            : 10.0 * log10(r / e);
+    }
+}
+
+// ------------------------------------------------------------------- host --
+typedef CUresult (*EncodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                CUtensorMapFloatOOBfill);
+
+EncodeTiled encoder()
+{
+    static EncodeTiled fn = nullptr;
+    if (!fn) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<EncodeTiled>(f);
+    }
+    return fn;
+}
+
+// rows x row_bytes operand, box of 128 rows x 128 bytes, 128-byte swizzle
+bool make_map(CUtensorMap *m, const void *base, int rows, int K, bool bf16)
+{
+    EncodeTiled enc = encoder();
+    if (!enc) return false;
+    const cuuint64_t inner = bf16 ? (cuuint64_t)K : (cuuint64_t)K / 2;
+    const cuuint64_t dims[2] = {inner, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {bf16 ? (cuuint64_t)K * 2 : (cuuint64_t)K / 2};
+    const cuuint32_t box[2] = {bf16 ? 64u : 128u, 128u};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+               const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KIND, int EPI>
+int launch(const GParams &p, const void *A, const void *B, cudaStream_t st)
+{
+    CUtensorMap ta, tb;
+    const bool bf16 = KIND == KIND_BF16;
+    if (!make_map(&ta, A, p.M, p.K, bf16) || !make_map(&tb, B, p.N, p.K, bf16)) return MX_ERR_CUDA;
+    using KT = Kind<KIND>;
+    const int smem = 1024 + kStages * KT::kStageBytes + 256;
+    auto k = k_gemm<KIND, EPI>;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return MX_ERR_CUDA;
+        attr = true;
+    }
+    dim3 grid(p.N / BN, p.M / BM);
+    k<<<grid, kThreads, smem, st>>>(p, ta, tb);
+    return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+}
+
+// MXFP4 (E2M1 + E8M0, block 32) or NVFP4 (E2M1 + UE4M3, block 16) operands
+// quantized along K in the tcgen05 scale layout; returns the kind or -1.
+int fp4_kind(const mx_config *a, const mx_config *b)
+{
+    if (!a || !b) return -1;
+    auto same = [](const mx_config *c) {
+        return c->elem == MX_E2M1 && c->axis == MX_AXIS_ROW && c->sf_layout == 1 && !c->asymmetric &&
+               !c->macro_block;
+    };
+    if (!same(a) || !same(b)) return -1;
+    if (a->scale_fmt == MX_SCALE_E8M0 && b->scale_fmt == MX_SCALE_E8M0 && a->block == 32 && b->block == 32)
+        return KIND_MXF4;
+    if (a->scale_fmt == MX_SCALE_UE4M3 && b->scale_fmt == MX_SCALE_UE4M3 && a->rule == MX_RULE_NEAREST &&
+        b->rule == MX_RULE_NEAREST && a->block == 16 && b->block == 16)
+        return KIND_NVF4;
+    return -1;
+}
+
+bool shapes_ok(int64_t M, int64_t N, int64_t K)
+{
+    return M > 0 && N > 0 && K > 0 && M % BM == 0 && N % BN == 0 && K % 256 == 0 && M < (1 << 30) &&
+           N < (1 << 30) && K < (1 << 30);
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+}  // namespace mxg
+
+using namespace mxg;
 
 extern "C" {
 
 int64_t mx_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)
 {
-    (void)M; (void)N; (void)K;
-    return 0;
+    (void)K;
+    if (M <= 0 || N <= 0) return 0;
+    const int64_t tiles = (M / BM) * (N / BN);
+    return 256 + M * N * 4 + tiles * 16;
 }
 
 int mx_gemm(const mx_config *ca, const mx_config *cb, const void *Aq, const uint8_t *Asf,
             const void *Bq, const uint8_t *Bsf, const float *tsA, const float *tsB, int64_t M,
             int64_t N, int64_t K, void *C, int32_t c_dtype, void *stream)
 {
-    (void)ca; (void)cb; (void)Aq; (void)Asf; (void)Bq; (void)Bsf; (void)tsA; (void)tsB;
-    (void)M; (void)N; (void)K; (void)C; (void)c_dtype; (void)stream;
-    return MX_ERR_UNSUPPORTED;
+    const int kind = fp4_kind(ca, cb);
+    if (kind < 0) return MX_ERR_UNSUPPORTED;
+    if (!shapes_ok(M, N, K)) return MX_ERR_INVALID;
+    if (!Aq || !Bq || !Asf || !Bsf || !C) return MX_ERR_INVALID;
+    if (c_dtype != MX_DT_BF16 && c_dtype != MX_DT_FP32) return MX_ERR_INVALID;
+    if (!aligned16(Aq) || !aligned16(Bq) || !aligned16(Asf) || !aligned16(Bsf) || !aligned16(C))
+        return MX_ERR_ALIGN;
+    GParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.sfa = Asf;
+    p.sfb = Bsf;
+    if (kind == KIND_NVF4) {
+        p.tsA = ca->tensor_scale != MX_TS_NONE ? tsA : nullptr;
+        p.tsB = cb->tensor_scale != MX_TS_NONE ? tsB : nullptr;
+    }
+    p.C = C;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (kind == KIND_MXF4)
+        return c_dtype == MX_DT_BF16 ? launch<KIND_MXF4, EPI_BF16>(p, Aq, Bq, st)
+                                     : launch<KIND_MXF4, EPI_F32>(p, Aq, Bq, st);
+    return c_dtype == MX_DT_BF16 ? launch<KIND_NVF4, EPI_BF16>(p, Aq, Bq, st)
+                                 : launch<KIND_NVF4, EPI_F32>(p, Aq, Bq, st);
 }
 
 int mx_gemm_qsnr(const mx_config *ca, const mx_config *cb, const void *A, const void *B, int64_t M,
@@ -26,16 +543,47 @@ int mx_gemm_qsnr(const mx_config *ca, const mx_config *cb, const void *A, const 
                  const uint8_t *Bsf, const float *tsA, const float *tsB, double *stats,
                  void *workspace, int64_t workspace_bytes, void *stream)
 {
-    (void)ca; (void)cb; (void)A; (void)B; (void)M; (void)N; (void)K; (void)Aq; (void)Asf;
-    (void)Bq; (void)Bsf; (void)tsA; (void)tsB; (void)stats; (void)workspace;
-    (void)workspace_bytes; (void)stream;
-    return MX_ERR_UNSUPPORTED;
+    if (fp4_kind(ca, cb) < 0) return MX_ERR_UNSUPPORTED;
+    if (!shapes_ok(M, N, K)) return MX_ERR_INVALID;
+    if (!A || !B || !stats) return MX_ERR_INVALID;
+    if (!workspace || workspace_bytes < mx_gemm_workspace_bytes(M, N, K)) return MX_ERR_WORKSPACE;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(workspace) || ((uintptr_t)stats & 7u))
+        return MX_ERR_ALIGN;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *cq = reinterpret_cast<float *>(ws + 256);
+    double *partials = reinterpret_cast<double *>(ws + 256 + M * N * 4);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // 1) C_q = A^Q (B^Q)^T (block-scaled FP4 MMA), fp32
+    int rc = mx_gemm(ca, cb, Aq, Asf, Bq, Bsf, tsA, tsB, M, N, K, cq, MX_DT_FP32, stream);
+    if (rc != MX_OK) return rc;
+    // 2) C_ref = A B^T (bf16 MMA, FP32 accumulate) with the QSNR sums in the epilogue
+    GParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.Cq = cq;
+    p.partials = partials;
+    rc = launch<KIND_BF16, EPI_QSNR>(p, A, B, st);
+    if (rc != MX_OK) return rc;
+    const int tiles = (int)((M / BM) * (N / BN));
+    k_gemm_qsnr_finalize<<<1, 256, 0, st>>>(partials, tiles, stats);
+    return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
 
 int mx_device_status(void *stream, int32_t *status)
 {
-    (void)stream;
-    if (status) *status = 0;
+    if (!status) return MX_ERR_INVALID;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int v = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return MX_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MX_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return MX_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MX_ERR_CUDA;
+    *status = v;
     return MX_OK;
 }
 

@@ -348,6 +348,14 @@ __device__ __forceinline__ float bf16_round(float v)
     return __fadd_rn(__bfloat162float(__float2bfloat16_rn(v)), 0.0f);
 }
 
+// Byte of scale j of row r in the tcgen05 chunk layout: 512-byte chunks of
+// 128 rows x 4 scales, row r at (r % 32) * 16 + ((r / 32) % 4) * 4 (S scales
+// per row, S % 4 == 0).
+__device__ __forceinline__ int64_t sf_chunk_index(int64_t r, int64_t j, int64_t S)
+{
+    return (((r >> 7) * (S >> 2) + (j >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (j & 3);
+}
+
 // binary32 1/sqrt(n) of the normalised rotation
 __device__ __forceinline__ float hadamard_scale(int n)
 {

@@ -35,6 +35,7 @@ struct QParams {
     int mbs;                 // 0 / 128
     int had;                 // 0 / 16 / 32
     int ts_mode;
+    int sf_gemm;             // scales in the tcgen05 chunk layout (row axis)
     uint64_t seed;
 };
 
@@ -49,7 +50,7 @@ struct DParams {
     int out_fp32;
     ElemDesc ed;
     ScaleDesc sd;
-    int block, axis, asym, mbs, had, ts_mode;
+    int block, axis, asym, mbs, had, ts_mode, sf_gemm;
 };
 
 struct SParams {
@@ -72,6 +73,11 @@ int launch_qsnr(const SParams &p, cudaStream_t st, int *grid_out);
 int launch_finalize_stats(const double *partials, int nparts, double count, double *stats,
                           cudaStream_t st);
 int device_sm_count();
+// Resident CTAs per SM of a kernel at a block size and dynamic shared memory
+// size, queried once per (kernel, threads, smem) and cached (the query and
+// the shared-memory attribute are host work that would otherwise sit between
+// short kernels); raises the kernel's dynamic shared-memory limit as needed.
+int cached_occupancy(const void *kernel, int threads, size_t smem);
 int launch_quantize_col(const QParams &p, int axis, int in_fp32, int fast, cudaStream_t st,
                         int *grid_out);
 int launch_amax_col(const QParams &p, int in_fp32, cudaStream_t st);

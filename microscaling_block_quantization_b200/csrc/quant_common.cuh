@@ -198,9 +198,7 @@ __device__ __forceinline__ void hadamard_chunk8(float y[8], int n, int lane)
 template <typename K>
 static int grid_for(K kernel, int64_t work_warps, int threads = kThreads, size_t smem = 0)
 {
-    int occ = 1;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, smem) != cudaSuccess || occ < 1)
-        occ = 1;
+    const int occ = cached_occupancy(reinterpret_cast<const void *>(kernel), threads, smem);
     int64_t g = (int64_t)device_sm_count() * occ;
     const int64_t need = (work_warps + (threads / 32) - 1) / (threads / 32);
     if (need < g) g = need;

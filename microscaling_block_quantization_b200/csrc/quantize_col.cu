@@ -438,8 +438,6 @@ template <typename K>
 int launch_k(K kernel, const QParams &p, int64_t work_warps, size_t smem, cudaStream_t st,
              int *grid_out)
 {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return -1;
     const int g = grid_for(kernel, work_warps, kColThreads, smem);
     kernel<<<g, kColThreads, smem, st>>>(p);
     if (grid_out) *grid_out = g;

@@ -10,6 +10,8 @@
 // scale); "Bridging the Gap ... Microscaling FP4 Quantization" (sec. 2.2-2.3,
 // rotation fused with quantization); fmread summary of Yang et al. (rounding
 // modes, asymmetric scaling, row / column / 2D blocks).
+#include <mutex>
+
 #include "quant_common.cuh"
 
 namespace mxk {
@@ -107,7 +109,12 @@ __device__ __forceinline__ void row_chunk(const QParams &p, int64_t c, bool ok, 
     }
     if (ok && (lane & (G - 1)) == 0) {
         const int64_t b = c / G;
-        p.scales[b] = (uint8_t)bs.code;
+        if (p.sf_gemm) {
+            const int64_t S = p.cols / p.block;
+            p.scales[sf_chunk_index(b / S, b - (b / S) * S, S)] = (uint8_t)bs.code;
+        } else {
+            p.scales[b] = (uint8_t)bs.code;
+        }
         if (!FAST && p.asym) p.offsets[b] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
     }
     if (stats && ok) {
@@ -219,6 +226,22 @@ __global__ void k_finalize_stats(const double *partials, int nparts, double coun
 }
 
 // ============================================================== launches ===
+int cached_occupancy(const void *kernel, int threads, size_t smem)
+{
+    struct Entry { const void *k; int threads; size_t smem; int occ; };
+    static Entry table[64];
+    static int used = 0;
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+        if (table[i].k == kernel && table[i].threads == threads && table[i].smem == smem) return table[i].occ;
+    if (smem > 48 * 1024) cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int occ = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, smem) != cudaSuccess || occ < 1) occ = 1;
+    if (used < 64) table[used++] = Entry{kernel, threads, smem, occ};
+    return occ;
+}
+
 static int g_sms = 0;
 int device_sm_count()
 {

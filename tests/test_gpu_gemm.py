@@ -1,0 +1,152 @@
+"""GPU parity of the tcgen05 block-scaled FP4 GEMM and of QSNR(AB).
+
+C = A^Q (B^Q)^T is checked against the oracle's dequantized operands
+multiplied in binary64 (the products of E2M1 values and power-of-two or
+UE4M3 scales are exact; the tensor cores accumulate in binary32): normwise
+relative error below 1e-3 and every element within 1e-3 * rms(C).  QSNR(AB)
+(Eq. (2) of the MXFP4 paper's Sec.3) is checked against the oracle's sums,
+1e-3 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+from microscaling_block_quantization_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mx():
+    from microscaling_block_quantization_b200 import build
+    build.build()
+    import microscaling_block_quantization_b200 as m
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return m
+
+
+def chunk_layout(scales: np.ndarray, rows: int, S: int) -> np.ndarray:
+    """Canonical [rows][S] scale bytes -> the 512-byte 128 x 4 chunk layout."""
+    out = np.zeros(rows * S, np.uint8)
+    r = np.arange(rows)[:, None]
+    j = np.arange(S)[None, :]
+    idx = ((r // 128) * (S // 4) + j // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + j % 4
+    out[idx.ravel()] = scales.reshape(rows, S).ravel()
+    return out
+
+
+def configs(mx):
+    return {"mxfp4": mx.Config(sf_layout=1),
+            "nvfp4": mx.Config(block=16, scale_fmt=1, rule=3, tensor_scale=1, sf_layout=1)}
+
+
+def ocfg(orc, name):
+    if name == "mxfp4":
+        return orc.Cfg()
+    return orc.Cfg(block=16, scale_fmt=orc.UE4M3, rule=orc.NEAREST, tensor_scale=orc.TS_COMPUTE)
+
+
+def deq(orc, name, x):
+    r = orc.quantize(ocfg(orc, name), x)
+    return orc.dequantize(ocfg(orc, name), r["packed"], r["scales"], r["tensor_scale"], None, None,
+                          *x.shape), r
+
+
+@pytest.mark.parametrize("name", ["mxfp4", "nvfp4"])
+def test_scale_chunk_layout(mx, orc, name):
+    x = inputs.laplace_outlier_cols(256, 512, seed=6, n_outlier_cols=2)
+    cfg = configs(mx)[name]
+    q = mx.quantize(x.cuda(), cfg)
+    r = orc.quantize(ocfg(orc, name), x)
+    S = 512 // cfg.block
+    assert np.array_equal(q.codes.cpu().numpy(), r["packed"].ravel())
+    assert np.array_equal(q.scales.cpu().numpy(), chunk_layout(r["scales"], 256, S))
+    xh = mx.dequantize(q, torch.float32).cpu().numpy()
+    oxh, _ = deq(orc, name, x)
+    assert np.array_equal(xh.view(np.uint32), oxh.view(np.uint32))
+
+
+def check_gemm(mx, orc, name, M, N, K, out_dtype=torch.float32, seed=0):
+    a = inputs.laplace_outlier_cols(M, K, seed=6 + seed, n_outlier_cols=2)
+    w = inputs.normal(N, K, sigma=0.02, seed=7 + seed)
+    cfg = configs(mx)[name]
+    qa = mx.quantize(a.cuda(), cfg, stats=False)
+    qw = mx.quantize(w.cuda(), cfg, stats=False)
+    c = mx.gemm(qa, qw, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert mx.mx_device_status() == 0
+    ah, _ = deq(orc, name, a)
+    wh, _ = deq(orc, name, w)
+    ref = ah.astype(np.float64) @ wh.astype(np.float64).T
+    got = c.float().cpu().numpy().astype(np.float64)
+    tol = 1e-3 if out_dtype == torch.float32 else 8e-3      # bf16 output rounding
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel < tol, rel
+    rms = np.sqrt(np.mean(ref ** 2))
+    assert np.max(np.abs(got - ref)) <= tol * rms + tol * np.abs(ref).max() * (out_dtype != torch.float32)
+    return rel
+
+
+@pytest.mark.parametrize("name", ["mxfp4", "nvfp4"])
+def test_gemm_single_tile(mx, orc, name):
+    check_gemm(mx, orc, name, 128, 128, 256)
+
+
+@pytest.mark.parametrize("name", ["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("shape", [(256, 384, 1024), (384, 256, 2048), (128, 640, 768)])
+def test_gemm_tiles_and_stage_ring(mx, orc, name, shape):
+    check_gemm(mx, orc, name, *shape)
+
+
+@pytest.mark.parametrize("name", ["mxfp4", "nvfp4"])
+def test_gemm_bf16_output(mx, orc, name):
+    check_gemm(mx, orc, name, 256, 256, 512, out_dtype=torch.bfloat16)
+
+
+def test_gemm_rejects_canonical_scales(mx):
+    a = torch.zeros(128, 256, dtype=torch.bfloat16, device="cuda")
+    q = mx.quantize(a, mx.MXFP4, stats=False)
+    with pytest.raises(mx.MXError) as e:
+        mx.gemm(q, q)
+    assert e.value.code == -2
+
+
+@pytest.mark.parametrize("name", ["mxfp4", "nvfp4"])
+def test_gemm_qsnr_small(mx, orc, name):
+    M, N, K = 256, 256, 512
+    a = inputs.laplace_outlier_cols(M, K, seed=6, n_outlier_cols=2)
+    w = inputs.normal(N, K, sigma=0.02, seed=7)
+    cfg = configs(mx)[name]
+    qa = mx.quantize(a.cuda(), cfg, stats=False)
+    qw = mx.quantize(w.cuda(), cfg, stats=False)
+    st = mx.gemm_qsnr(a.cuda(), w.cuda(), qa, qw).cpu().numpy()
+    ah, _ = deq(orc, name, a)
+    wh, _ = deq(orc, name, w)
+    o = orc.gemm_qsnr(orc.input_f32(a), orc.input_f32(w), ah, wh)
+    assert abs(st[0] - o[0]) <= 1e-3 * o[0]
+    assert abs(st[1] - o[1]) <= 1e-3 * o[1]
+    assert abs(st[2] - o[2]) <= 1e-2
+
+
+@pytest.mark.parametrize("name", ["mxfp4", "nvfp4"])
+def test_gemm_llama_shape_sampled_rows(mx, orc, name):
+    """The 8192 x 4096 by 14336 x 4096 layer in the benchmark's launch
+    configuration: 64 sampled rows of C against the oracle's dequantized
+    operands in binary64."""
+    A, W = inputs.llama_linear()
+    cfg = configs(mx)[name]
+    qa = mx.quantize(A.cuda(), cfg, stats=False)
+    qw = mx.quantize(W.cuda(), cfg, stats=False)
+    c = mx.gemm(qa, qw, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert mx.mx_device_status() == 0
+    rows = np.sort(np.random.default_rng(1).choice(8192, 64, replace=False))
+    wh, _ = deq(orc, name, W)
+    r = orc.quantize(ocfg(orc, name), A)
+    ah = orc.dequantize(ocfg(orc, name), r["packed"], r["scales"], r["tensor_scale"], None, None, 8192, 4096)
+    ref = ah[rows].astype(np.float64) @ wh.astype(np.float64).T
+    got = c[torch.from_numpy(rows).cuda()].cpu().numpy().astype(np.float64)
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel < 1e-3, rel
+    assert np.max(np.abs(got - ref)) <= 1e-3 * np.sqrt(np.mean(ref ** 2))
