@@ -48,6 +48,13 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-gemm", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-case", default=None,
+                    help="run one kernel alone (for ncu captures): quant_mxfp4_row, quant_nvfp4_row, "
+                         "quant_mxfp4_col, quant_mxfp4_2d, quant_had32_row, dequant_mxfp4_row, "
+                         "gemm_mxfp4, gemm_nvfp4")
+    ap.add_argument("--rows", type=int, default=16384)
+    ap.add_argument("--cols", type=int, default=8192)
+    ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
 
 
@@ -472,8 +479,60 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+def kernel_case(args):
+    """One kernel on one synthetic tensor, `reps` times, each timed with CUDA
+    events; the default 16384 x 8192 bf16 input (256 MiB) is larger than L2."""
+    import microscaling_block_quantization_b200 as mx
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(0)
+    case = args.kernel_case
+    res = {"case": case}
+    if case.startswith("gemm"):
+        M, N, K = M_TOK, N_OUT, K_DIM
+        cfg = (mx.Config(sf_layout=1) if case == "gemm_mxfp4" else
+               mx.Config(block=16, scale_fmt=1, rule=3, tensor_scale=1, sf_layout=1))
+        a = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
+        w = (torch.randn(N, K, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        qa, qw = mx.quantize(a, cfg, stats=False), mx.quantize(w, cfg, stats=False)
+        c = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        run = lambda: mx.gemm(qa, qw, out=c)
+        work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
+    else:
+        R, Cc = args.rows, args.cols
+        x = torch.randn(R, Cc, generator=g, device=dev).to(torch.bfloat16)
+        cfg = {"quant_mxfp4_row": mx.MXFP4, "quant_nvfp4_row": mx.NVFP4,
+               "quant_mxfp4_col": mx.Config(axis=1), "quant_mxfp4_2d": mx.Config(axis=2),
+               "quant_had32_row": mx.Config(hadamard=32), "dequant_mxfp4_row": mx.MXFP4}[case]
+        q = mx.quantize(x, cfg)
+        if case.startswith("dequant"):
+            out = torch.empty(R, Cc, dtype=torch.bfloat16, device=dev)
+            run = lambda: mx.dequantize(q, out=out)
+            kind = "d"
+        else:
+            run = lambda: mx.quantize(x, cfg, out=q)
+            kind = "q"
+        work, unit = algo_bytes(cfg, R, Cc, kind) / 1e9, "GB/s"
+        res["algorithmic_bytes"] = algo_bytes(cfg, R, Cc, kind)
+    run()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.reps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        run()
+        e.record()
+        torch.cuda.synchronize()
+        times.append(s.elapsed_time(e))
+    res["us"] = [round(t * 1e3, 2) for t in times]
+    res[unit] = round(work / (min(times) * 1e-3), 1)
+    print(json.dumps(res), flush=True)
+
+
 def main():
     args = parse()
+    if args.kernel_case:
+        kernel_case(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

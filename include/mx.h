@@ -156,8 +156,9 @@ int mx_query_sizes(const mx_config *cfg, int64_t rows, int64_t cols, mx_sizes *o
  *              dequantized tensor against x, fused into the same pass.
  *   workspace  device scratch of sizes.workspace_bytes (needed when stats != NULL
  *              or cfg->tensor_scale == MX_TS_COMPUTE).
- * Shapes: cols % block == 0 (row), rows % block == 0 (column), both % 32 (2D),
- * % 128 along the axis for MBS, cols % 8 == 0 always.  Block non-finite
+ * Shapes: cols % 32 == 0 always (lanes walk rows in 32-element chunks),
+ * rows * cols < 2^40, cols % block == 0 (row), rows % block == 0 (column),
+ * rows % 32 == 0 (2D), % 128 along the axis for MBS.  Block non-finite
  * values give the NaN scale code and zero element codes.
  */
 int mx_quantize(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t rows, int64_t cols,

@@ -106,7 +106,9 @@ int check_config(const mx_config *c, int64_t rows, int64_t cols, bool want_had)
 
     // shapes
     if (rows == 0 || cols == 0) return MX_OK;
-    if (cols % 8) return MX_ERR_INVALID;
+    // kernels walk rows in 32-element chunks (one per lane)
+    if (cols % 32) return MX_ERR_INVALID;
+    if (rows > (INT64_C(1) << 40) / cols) return MX_ERR_INVALID;
     if (c->axis == MX_AXIS_ROW && cols % B) return MX_ERR_INVALID;
     if (c->sf_layout == 1 && (rows % 128 || (cols / B) % 4)) return MX_ERR_INVALID;
     if (c->axis == MX_AXIS_COL && rows % B) return MX_ERR_INVALID;

@@ -41,47 +41,6 @@ __device__ __forceinline__ float deq_one(const DParams &p, uint32_t code, uint32
     return v;
 }
 
-__device__ __forceinline__ void hadamard8(float y[8], int n, int lane)
-{
-#pragma unroll
-    for (int h = 1; h < 8; h <<= 1)
-#pragma unroll
-        for (int i = 0; i < 8; i += 2 * h)
-#pragma unroll
-            for (int j = i; j < i + h; ++j) {
-                float a = y[j], b = y[j + h];
-                y[j] = __fadd_rn(a, b);
-                y[j + h] = __fsub_rn(a, b);
-            }
-    for (int m = 1; m < n / 8; m <<= 1) {
-        const bool upper = (lane & m) != 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float w = __shfl_xor_sync(kFull, y[j], m);
-            y[j] = upper ? __fsub_rn(w, y[j]) : __fadd_rn(y[j], w);
-        }
-    }
-    const float c = hadamard_scale(n);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) y[j] = __fmul_rn(y[j], c);
-}
-
-__device__ __forceinline__ void store8(void *out, bool f32, int64_t e, const float v[8])
-{
-    if (f32) {
-        float *o = static_cast<float *>(out) + e;
-        reinterpret_cast<float4 *>(o)[0] = make_float4(v[0], v[1], v[2], v[3]);
-        reinterpret_cast<float4 *>(o)[1] = make_float4(v[4], v[5], v[6], v[7]);
-    } else {
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            w[i] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i])) |
-                   ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * i + 1])) << 16);
-        *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + e) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
-
 __device__ __forceinline__ void unpack_bf16x2(uint32_t w, float &lo, float &hi)
 {
     lo = __uint_as_float(w << 16);
@@ -105,73 +64,124 @@ __device__ __forceinline__ void load8any(const void *x, bool f32, int64_t e, flo
 }
 
 // ------------------------------------------------------------ dequantize --
-// Thread = 8 consecutive elements of a row (every axis); the rotation, when
-// on, runs along rows (row and 2D layouts).
+// Thread = 32 consecutive elements of a row (every axis): one 16-byte code
+// load (4-bit) or two (FP6), the block scales of those elements, and 64 / 128
+// output bytes; the rotation, when on, runs along rows inside the thread
+// (row and 2D layouts).
+__device__ __forceinline__ void hadamard32(float y[32], int n)
+{
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1) {
+        if (h >= n) break;
+#pragma unroll
+        for (int i = 0; i < 32; i += 2 * h)
+#pragma unroll
+            for (int j = i; j < i + h; ++j) {
+                const float a = y[j], b = y[j + h];
+                y[j] = __fadd_rn(a, b);
+                y[j + h] = __fsub_rn(a, b);
+            }
+    }
+    const float c = hadamard_scale(n);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) y[j] = __fmul_rn(y[j], c);
+}
+
+template <bool FAST>
 __global__ void __launch_bounds__(kThreads) k_dequant_chunk(const DParams p)
 {
     const int lane = threadIdx.x & 31;
-    const int64_t nchunks = p.rows * p.cols / 8;
-    const int64_t ntiles = (nchunks + 31) / 32;
-    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const uint32_t nch = (uint32_t)(p.rows * p.cols / 32);
+    const uint32_t cpr = (uint32_t)(p.cols / 32);                 // chunks per row
+    const uint32_t gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nw = (gridDim.x * blockDim.x) >> 5;
     const float sT = (p.ts_mode != TS_NONE && p.tensor_scale) ? *p.tensor_scale : 1.0f;
-    for (int64_t t = gw; t < ntiles; t += nw) {
-        const int64_t c = t * 32 + lane;
-        const bool ok = c < nchunks;
-        float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const bool nearest = p.sd.fmt != S_E8M0 && p.sd.rule == R_NEAREST;
+    const int B = p.block;
+    const int lb = __ffs(B) - 1;                                   // B is a power of two
+    const uint32_t S = (uint32_t)(p.cols >> lb);                   // row-axis scales per row
+    for (uint32_t c0 = gw * 32; c0 < nch; c0 += nw * 32) {
+        const uint32_t c = c0 + lane;
+        const bool ok = c < nch;
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0.0f;
         if (ok) {
-            const int64_t e0 = c * 8;
-            const int64_t row = e0 / p.cols, col0 = e0 - row * p.cols;
-            uint32_t lo, hi = 0;
+            const uint32_t row = c / cpr;
+            const uint32_t col0 = (c - row * cpr) * 32;
+            uint32_t w[8];
             if (p.ed.code_bits == 4) {
-                lo = reinterpret_cast<const uint32_t *>(p.codes)[c];
+                const uint4 u = reinterpret_cast<const uint4 *>(p.codes)[c];
+                w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
             } else {
-                const uint2 w = reinterpret_cast<const uint2 *>(p.codes)[c];
-                lo = w.x;
-                hi = w.y;
+                const uint4 u0 = reinterpret_cast<const uint4 *>(p.codes)[2 * (size_t)c];
+                const uint4 u1 = reinterpret_cast<const uint4 *>(p.codes)[2 * (size_t)c + 1];
+                w[0] = u0.x; w[1] = u0.y; w[2] = u0.z; w[3] = u0.w;
+                w[4] = u1.x; w[5] = u1.y; w[6] = u1.z; w[7] = u1.w;
             }
-            uint32_t sc[8];
-            uint16_t of[8];
-            uint32_t mc[8];
-            if (p.axis == AX_COL) {
-                const int64_t b0 = (row / p.block) * p.cols + col0;
-                const uint2 s2 = *reinterpret_cast<const uint2 *>(p.scales + b0);
+            if (FAST) {
+                // E2M1, symmetric, power-of-two or NEAREST scales, row or 2D axis, no MBS
 #pragma unroll
-                for (int j = 0; j < 8; ++j) sc[j] = ((j < 4 ? s2.x : s2.y) >> (8 * (j & 3))) & 0xffu;
-                if (p.asym)
+                for (int g = 0; g < 4; ++g) {
+                    const uint32_t col = col0 + 8 * g;
+                    uint32_t sc;
+                    if (p.axis == AX_ROW)
+                        sc = p.sf_gemm ? p.scales[sf_chunk_index(row, col >> lb, S)]
+                                       : p.scales[(size_t)row * S + (col >> lb)];
+                    else
+                        sc = p.scales[(size_t)(row >> 5) * (p.cols >> 5) + (col >> 5)];
+                    const float sb = scale_value(p.sd, sc);
+                    float q[8];
+                    e2m1x8_values(w[g], q);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) of[j] = p.offsets[b0 + j];
-                if (p.mbs) {
-                    const uint2 m2 = *reinterpret_cast<const uint2 *>(p.macro + (row / 128) * p.cols + col0);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) mc[j] = ((j < 4 ? m2.x : m2.y) >> (8 * (j & 3))) & 0xffu;
+                    for (int i = 0; i < 8; ++i)
+                        v[8 * g + i] = nearest ? __fmul_rn(__fmul_rn(q[i], sb), sT) : __fmul_rn(q[i], sb);
                 }
             } else {
-                const int64_t b = (p.axis == AX_ROW) ? e0 / p.block
-                                                     : (row / 32) * (p.cols / 32) + col0 / 32;
-                uint32_t s;
-                if (p.axis == AX_ROW && p.sf_gemm) {
-                    const int64_t S = p.cols / p.block;
-                    s = p.scales[sf_chunk_index(row, col0 / p.block, S)];
-                } else {
-                    s = p.scales[b];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const uint32_t col = col0 + j;
+                    size_t b;
+                    if (p.axis == AX_ROW) b = (size_t)row * S + (col >> lb);
+                    else if (p.axis == AX_COL) b = (size_t)(row >> lb) * p.cols + col;
+                    else b = (size_t)(row >> 5) * (p.cols >> 5) + (col >> 5);
+                    const uint32_t sc = (p.axis == AX_ROW && p.sf_gemm)
+                                            ? p.scales[sf_chunk_index(row, col >> lb, S)]
+                                            : p.scales[b];
+                    const uint32_t code = (p.ed.code_bits == 4) ? (w[j >> 3] >> (4 * (j & 7))) & 0xfu
+                                                                : (w[j >> 2] >> (8 * (j & 3))) & 0x3fu;
+                    float sm = 1.0f;
+                    if (p.mbs) {
+                        const size_t mi = (p.axis == AX_COL) ? (size_t)(row / 128) * p.cols + col
+                                                             : (size_t)row * (p.cols / 128) + col / 128;
+                        sm = e4m3_value(p.macro[mi]);
+                    }
+                    const float o = p.asym ? __uint_as_float((uint32_t)p.offsets[b] << 16) : 0.0f;
+                    v[j] = deq_one(p, code, sc, sT, sm, o);
                 }
-                const uint16_t o = p.asym ? p.offsets[b] : 0;
-                const uint32_t m = p.mbs ? p.macro[row * (p.cols / 128) + col0 / 128] : 0u;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) { sc[j] = s; of[j] = o; mc[j] = m; }
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t code = (p.ed.code_bits == 4) ? (lo >> (4 * j)) & 0xfu
-                                    : ((j < 4 ? lo : hi) >> (8 * (j & 3))) & 0x3fu;
-                const float sm = p.mbs ? e4m3_value(mc[j]) : 1.0f;
-                const float o = p.asym ? __uint_as_float((uint32_t)of[j] << 16) : 0.0f;
-                v[j] = deq_one(p, code, sc[j], sT, sm, o);
             }
         }
-        if (p.had) hadamard8(v, p.had, lane);
-        if (ok) store8(p.out, p.out_fp32, c * 8, v);
+        if (p.had) hadamard32(v, p.had);
+        if (ok) {
+            const int64_t e0 = (int64_t)c * 32;
+            if (p.out_fp32) {
+                float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + e0);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            } else {
+                uint4 *o = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + e0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    uint32_t t[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * i + 2 * k], v[8 * i + 2 * k + 1]);
+                        t[k] = *reinterpret_cast<uint32_t *>(&h);
+                    }
+                    o[i] = make_uint4(t[0], t[1], t[2], t[3]);
+                }
+            }
+        }
     }
 }
 
@@ -417,9 +427,15 @@ int launch_dequantize(const DParams &p, cudaStream_t st)
         const int g = grid_of(k_dequant_colhad, items);
         k_dequant_colhad<<<g, kThreads, 0, st>>>(p);
     } else {
-        const int64_t tiles = (p.rows * p.cols / 8 + 31) / 32;
-        const int g = grid_of(k_dequant_chunk, tiles);
-        k_dequant_chunk<<<g, kThreads, 0, st>>>(p);
+        const int64_t warps = (p.rows * p.cols / 32 + 31) / 32;
+        const bool fast = p.ed.elem == E2M1 && !p.asym && !p.mbs && p.axis != AX_COL;
+        if (fast) {
+            const int g = grid_of(k_dequant_chunk<true>, warps);
+            k_dequant_chunk<true><<<g, kThreads, 0, st>>>(p);
+        } else {
+            const int g = grid_of(k_dequant_chunk<false>, warps);
+            k_dequant_chunk<false><<<g, kThreads, 0, st>>>(p);
+        }
     }
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }

@@ -120,7 +120,7 @@ __device__ __forceinline__ double warp_sum(double v)
 }
 
 // CTA reduction in a fixed order; thread 0 writes the CTA's record.
-static __device__ __noinline__ void write_partials(double *partials, const Acc &a)
+static __device__ __forceinline__ void write_partials(double *partials, const Acc &a)
 {
     __shared__ double sh[32][5];
     double v[5] = {a.x2, a.e2, a.e, a.ftz, a.nz};

@@ -17,142 +17,249 @@
 namespace mxk {
 
 // ================================================================ row axis ==
-// Thread = chunk of 8 consecutive elements of a row; a block of B elements is
-// B/8 consecutive lanes; U chunks per lane in flight.
-template <bool FAST>
-__device__ __forceinline__ void row_chunk(const QParams &p, int64_t c, bool ok, float y[8],
-                                          float sT, Acc &acc, int lane, bool stats)
+// Thread = 32 consecutive elements of a row (four 16-byte loads in flight for
+// bf16, eight for fp32).  A block of B <= 32 elements lies inside the thread
+// (32 / B blocks per thread); a block of B > 32 spans B / 32 consecutive lanes.
+// A 1 x 128 macro block spans 4 lanes; a 16- or 32-point rotation group lies
+// inside the thread.
+
+__device__ __forceinline__ float fmax_nan(float a, float b)
 {
-    const int G = p.lanes_per_block;
-    if (p.had) hadamard_chunk8(y, p.had, lane);
-    if (p.rotated && ok) store8f(p.rotated, c * 8, y);
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
 
-    float xq[8];
-    float sm = 1.0f;
-    if (p.mbs) {
-        float m = 0.0f;
-        int bad = 0;
+__device__ __forceinline__ void load32(const __nv_bfloat16 *x, int64_t e, float v[32])
+{
+    const uint4 *p = reinterpret_cast<const uint4 *>(x + e);
+    uint4 u[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            bad |= nonfinite(y[j]);
-            m = fmaxf(m, fabsf(y[j]));
-        }
-        m = grp_max(m, 16);
-        bad = grp_or(bad, 16);
-        uint32_t code = macro_code(p.ed, m, bad);
-        sm = e4m3_value(code);
-        const float inv = __fdiv_rn(1.0f, sm);
+    for (int i = 0; i < 4; ++i) u[i] = __ldg(p + i);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) xq[j] = __fmul_rn(y[j], inv);
-        if (ok && (lane & 15) == 0) p.macro[c >> 4] = (uint8_t)code;
-    } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) xq[j] = y[j];
+    for (int i = 0; i < 4; ++i) {
+        unpack_bf16x2(u[i].x, v[8 * i + 0], v[8 * i + 1]);
+        unpack_bf16x2(u[i].y, v[8 * i + 2], v[8 * i + 3]);
+        unpack_bf16x2(u[i].z, v[8 * i + 4], v[8 * i + 5]);
+        unpack_bf16x2(u[i].w, v[8 * i + 6], v[8 * i + 7]);
     }
-
-    int bad = 0;
+}
+__device__ __forceinline__ void load32(const float *x, int64_t e, float v[32])
+{
+    const float4 *p = reinterpret_cast<const float4 *>(x + e);
+    float4 u[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) bad |= nonfinite(xq[j]);
-    bad = grp_or(bad, G);
-
-    float o = 0.0f;
-    if (!FAST && p.asym) {
-        float mn = xq[0], mx = xq[0];
+    for (int i = 0; i < 8; ++i) u[i] = __ldg(p + i);
 #pragma unroll
-        for (int j = 1; j < 8; ++j) {
-            mn = fminf(mn, xq[j]);
-            mx = fmaxf(mx, xq[j]);
-        }
-        mn = grp_min(mn, G);
-        mx = grp_max(mx, G);
-        if (!bad) o = p.ed.is_int ? bf16_round(mn) : bf16_round(__fmul_rn(__fadd_rn(mx, mn), 0.5f));
-#pragma unroll
-        for (int j = 0; j < 8; ++j) xq[j] = __fsub_rn(xq[j], o);
-    }
-
-    float alpha = 0.0f;
-    const bool raw_max = !FAST && p.ed.is_int && p.asym;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) alpha = fmaxf(alpha, raw_max ? xq[j] : fabsf(xq[j]));
-    alpha = grp_max(alpha, G);
-    const BlockScale bs = block_scale(p.ed, p.sd, alpha, bad, sT);
-
-    float q[8];
-    if constexpr (FAST) {
-        float v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = __fmul_rn(xq[j], bs.inv);
-        const uint32_t pk = bs.zero ? 0u : cvt_e2m1x8(v);
-        if (ok) reinterpret_cast<uint32_t *>(p.codes)[c] = pk;
-        if (stats) e2m1x8_values(pk, q);
-    } else {
-        uint4 w0 = make_uint4(0, 0, 0, 0), w1 = w0;
-        if (p.round_mode == RD_SR) {
-            w0 = element_words(p.seed, (uint64_t)c * 2);
-            w1 = element_words(p.seed, (uint64_t)c * 2 + 1);
-        }
-        uint32_t lo = 0, hi = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t u = word_of(j < 4 ? w0 : w1, j & 3);
-            uint32_t code = 0;
-            q[j] = 0.0f;
-            if (!bs.zero) code = encode_elem(p.ed, p.round_mode, __fmul_rn(xq[j], bs.inv), u, q[j]);
-            if (p.ed.code_bits == 4) lo |= code << (4 * j);
-            else if (j < 4) lo |= code << (8 * j);
-            else hi |= code << (8 * (j - 4));
-        }
-        if (ok) {
-            if (p.ed.code_bits == 4) reinterpret_cast<uint32_t *>(p.codes)[c] = lo;
-            else reinterpret_cast<uint2 *>(p.codes)[c] = make_uint2(lo, hi);
-        }
-    }
-    if (ok && (lane & (G - 1)) == 0) {
-        const int64_t b = c / G;
-        if (p.sf_gemm) {
-            const int64_t S = p.cols / p.block;
-            p.scales[sf_chunk_index(b / S, b - (b / S) * S, S)] = (uint8_t)bs.code;
-        } else {
-            p.scales[b] = (uint8_t)bs.code;
-        }
-        if (!FAST && p.asym) p.offsets[b] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
-    }
-    if (stats && ok) {
-        float xh[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) xh[j] = deq_value(p, q[j], bs, sm, o, sT);
-        acc_add<8>(acc, y, xh);
+    for (int i = 0; i < 8; ++i) {
+        v[4 * i + 0] = u[i].x; v[4 * i + 1] = u[i].y; v[4 * i + 2] = u[i].z; v[4 * i + 3] = u[i].w;
     }
 }
 
-template <typename InT, bool FAST>
+// in-thread block Hadamard on 32 elements: groups of n (16 or 32)
+__device__ __forceinline__ void hadamard32(float y[32], int n)
+{
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1) {
+        if (h >= n) break;
+#pragma unroll
+        for (int i = 0; i < 32; i += 2 * h)
+#pragma unroll
+            for (int j = i; j < i + h; ++j) {
+                const float a = y[j], b = y[j + h];
+                y[j] = __fadd_rn(a, b);
+                y[j + h] = __fsub_rn(a, b);
+            }
+    }
+    const float c = hadamard_scale(n);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) y[j] = __fmul_rn(y[j], c);
+}
+
+// number of zero-magnitude E2M1 codes among the 8 nibbles of w
+__device__ __forceinline__ int zero_codes8(uint32_t w)
+{
+    const uint32_t m = w & 0x77777777u;
+    const uint32_t t = (m | (m >> 1) | (m >> 2)) & 0x11111111u;
+    return 8 - __popc(t);
+}
+
+template <typename InT, int B, bool FAST>
 __global__ void __launch_bounds__(kThreads) k_quant_row(const QParams p)
 {
-    constexpr int U = 2;
+    constexpr int NB = B <= 32 ? 32 / B : 1;    // blocks per thread
+    constexpr int G = B <= 32 ? 1 : B / 32;     // lanes per block
+    constexpr int L = B <= 32 ? B : 32;         // elements of a block held by the thread
     const InT *x = static_cast<const InT *>(p.x);
     const int lane = threadIdx.x & 31;
-    const int64_t nchunks = p.rows * p.cols / 8;
-    const int64_t per_tile = 32 * U;
-    const int64_t ntiles = (nchunks + per_tile - 1) / per_tile;
-    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const uint32_t nch = (uint32_t)(p.rows * p.cols / 32);
+    const uint32_t gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nw = (gridDim.x * blockDim.x) >> 5;
     const bool stats = p.partials != nullptr;
     const float sT = (p.ts_mode != TS_NONE) ? *p.tensor_scale : 1.0f;
+    const bool nearest = p.sd.fmt != S_E8M0 && p.sd.rule == R_NEAREST;
+    const uint32_t S = (uint32_t)(p.cols / B);  // scales per row
     Acc acc = {0, 0, 0, 0, 0};
-    for (int64_t t = gw; t < ntiles; t += nw) {
-        float v[U][8];
+
+    for (uint32_t c0 = gw * 32; c0 < nch; c0 += nw * 32) {
+        const uint32_t c = c0 + lane;
+        const bool ok = c < nch;
+        const int64_t e0 = (int64_t)c * 32;
+        float y[32];
+        if (ok) load32(x, e0, y);
+        else
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t c = t * per_tile + u * 32 + lane;
-            if (c < nchunks) load8(x, c * 8, v[u]);
-            else
+            for (int j = 0; j < 32; ++j) y[j] = 0.0f;
+
+        if (p.had) hadamard32(y, p.had);
+        if (p.rotated && ok)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
+            for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4 *>(p.rotated + e0 + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+
+        // macro-block scale (MBS) over 4 lanes
+        float sm = 1.0f, invm = 1.0f;
+        if (p.mbs) {
+            float m = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) m = fmax_nan(m, fabsf(y[j]));
+            int bad = !(m <= FLT_MAX);
+            float mm = bad ? 0.0f : m;
+            mm = grp_max(mm, 4);
+            bad = grp_or(bad, 4);
+            const uint32_t code = macro_code(p.ed, mm, bad);
+            sm = e4m3_value(code);
+            invm = __fdiv_rn(1.0f, sm);
+            if (ok && (lane & 3) == 0) p.macro[c >> 2] = (uint8_t)code;
         }
+        auto xq = [&](int j) -> float { return p.mbs ? __fmul_rn(y[j], invm) : y[j]; };
+
+        uint32_t words[FAST ? 4 : 8];   // 4-bit: 4 words of 8 nibbles; FP6: 8 words of 4 bytes
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t c = t * per_tile + u * 32 + lane;
-            row_chunk<FAST>(p, c, c < nchunks, v[u], sT, acc, lane, stats);
+        for (int i = 0; i < (FAST ? 4 : 8); ++i) words[i] = 0;
+        uint32_t scode[NB];
+        uint16_t obits[NB];
+
+#pragma unroll
+        for (int k = 0; k < NB; ++k) {
+            const int j0 = k * L;
+            float a = 0.0f, mn = FLT_MAX, mx = -FLT_MAX;
+#pragma unroll
+            for (int j = j0; j < j0 + L; ++j) {
+                const float v = xq(j);
+                a = fmax_nan(a, fabsf(v));
+                if (!FAST && p.asym) { mn = fminf(mn, v); mx = fmaxf(mx, v); }
+            }
+            int bad = !(a <= FLT_MAX);
+            if (G > 1) {
+                a = grp_max(bad ? 0.0f : a, G);
+                bad = grp_or(bad, G);
+                if (!FAST && p.asym) { mn = grp_min(mn, G); mx = grp_max(mx, G); }
+            }
+            float o = 0.0f;
+            if (!FAST && p.asym) {
+                if (!bad) o = p.ed.is_int ? bf16_round(mn) : bf16_round(__fmul_rn(__fadd_rn(mx, mn), 0.5f));
+                float ra = 0.0f;
+#pragma unroll
+                for (int j = j0; j < j0 + L; ++j) {
+                    const float d = __fsub_rn(xq(j), o);
+                    ra = fmaxf(ra, p.ed.is_int ? d : fabsf(d));
+                }
+                if (G > 1) ra = grp_max(ra, G);
+                a = ra;
+            }
+            const BlockScale bs = block_scale(p.ed, p.sd, bad ? 0.0f : a, bad, sT);
+            scode[k] = bs.code;
+            obits[k] = (!FAST && p.asym) ? __bfloat16_as_ushort(__float2bfloat16_rn(o)) : (uint16_t)0;
+
+            if constexpr (FAST) {
+                // E2M1, RTNE: conversion instruction, 8 elements per word
+                float deqT = bs.nan ? __uint_as_float(0x7fc00000u)
+                           : nearest ? __fmul_rn(bs.deq, sT) : bs.deq;
+                if (p.mbs) deqT = __fmul_rn(deqT, sm);
+                float sx = 0.f, se = 0.f, sb = 0.f;
+                int xz = 0, qz = 0;
+#pragma unroll
+                for (int w = 0; w < L / 8; ++w) {
+                    const int jb = j0 + 8 * w;
+                    float s8[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) s8[i] = __fmul_rn(xq(jb + i), bs.inv);
+                    const uint32_t word = bs.zero ? 0u : cvt_e2m1x8(s8);
+                    words[jb >> 3] = word;
+                    if (stats) {
+                        float q[8];
+                        e2m1x8_values(word, q);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float yv = y[jb + i];
+                            const float d = fmaf(-q[i], deqT, yv);
+                            se = fmaf(d, d, se);
+                            sx = fmaf(yv, yv, sx);
+                            sb -= d;
+                            xz += (yv == 0.0f);
+                        }
+                        qz += zero_codes8(word);
+                    }
+                }
+                if (stats && ok) {
+                    acc.x2 += (double)sx;
+                    acc.e2 += (double)se;
+                    acc.e += (double)sb;
+                    acc.nz += (double)(L - xz);
+                    acc.ftz += bs.nan ? 0.0 : (double)(qz - xz);
+                }
+            } else {
+                uint4 rw = make_uint4(0, 0, 0, 0);
+                float yv[L], xh[L];
+#pragma unroll
+                for (int j = j0; j < j0 + L; ++j) {
+                    if (p.round_mode == RD_SR && (j & 3) == 0)
+                        rw = element_words(p.seed, ((uint64_t)e0 + j) >> 2);
+                    float q = 0.0f;
+                    uint32_t code = 0;
+                    if (!bs.zero) {
+                        float v = xq(j);
+                        if (p.asym) v = __fsub_rn(v, o);
+                        code = encode_elem(p.ed, p.round_mode, __fmul_rn(v, bs.inv), word_of(rw, j & 3), q);
+                    }
+                    if (p.ed.code_bits == 4) words[j >> 3] |= code << (4 * (j & 7));
+                    else words[j >> 2] |= code << (8 * (j & 3));
+                    yv[j - j0] = y[j];
+                    xh[j - j0] = deq_value(p, q, bs, sm, o, sT);
+                }
+                if (stats && ok) acc_add<L>(acc, yv, xh);
+            }
+        }
+
+        if (ok) {
+            // codes: 16 bytes (4-bit) or 32 bytes (FP6) per thread
+            if (FAST || p.ed.code_bits == 4) {
+                reinterpret_cast<uint4 *>(p.codes)[c] = make_uint4(words[0], words[1], words[2], words[3]);
+            } else {
+                uint4 *dst = reinterpret_cast<uint4 *>(p.codes) + 2 * (size_t)c;
+                dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+                dst[1] = make_uint4(words[FAST ? 0 : 4], words[FAST ? 0 : 5], words[FAST ? 0 : 6], words[FAST ? 0 : 7]);
+            }
+            // scales (and offsets): NB per thread, or one per G lanes
+            if (G == 1 || (lane & (G - 1)) == 0) {
+                const uint32_t b0 = (G == 1) ? c * NB : c / G;
+                if (p.sf_gemm) {
+                    const uint32_t r = b0 / S, j = b0 - r * S;
+#pragma unroll
+                    for (int k = 0; k < NB; ++k) p.scales[sf_chunk_index(r, j + k, S)] = (uint8_t)scode[k];
+                } else if (NB == 4) {
+                    *reinterpret_cast<uint32_t *>(p.scales + b0) =
+                        scode[0] | (scode[NB > 1 ? 1 : 0] << 8) | (scode[NB > 2 ? 2 : 0] << 16) | (scode[NB > 3 ? 3 : 0] << 24);
+                } else if (NB == 2) {
+                    *reinterpret_cast<uint16_t *>(p.scales + b0) = (uint16_t)(scode[0] | (scode[NB > 1 ? 1 : 0] << 8));
+                } else {
+                    p.scales[b0] = (uint8_t)scode[0];
+                }
+                if (!FAST && p.asym)
+#pragma unroll
+                    for (int k = 0; k < NB; ++k) p.offsets[b0 + k] = obits[k];
+            }
         }
     }
     if (stats) write_partials(p.partials, acc);
@@ -165,18 +272,20 @@ __global__ void __launch_bounds__(kThreads) k_amax_row(const QParams p)
 {
     const InT *x = static_cast<const InT *>(p.x);
     const int lane = threadIdx.x & 31;
-    const int64_t nchunks = p.rows * p.cols / 8;
-    const int64_t ntiles = (nchunks + 31) / 32;
-    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const uint32_t nch = (uint32_t)(p.rows * p.cols / 32);
+    const uint32_t gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nw = (gridDim.x * blockDim.x) >> 5;
     float m = 0.0f;
-    for (int64_t t = gw; t < ntiles; t += nw) {
-        const int64_t c = t * 32 + lane;
-        float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        if (c < nchunks) load8(x, c * 8, v);
-        if (p.had) hadamard_chunk8(v, p.had, lane);
+    for (uint32_t c0 = gw * 32; c0 < nch; c0 += nw * 32) {
+        const uint32_t c = c0 + lane;
+        float v[32];
+        if (c < nch) load32(x, (int64_t)c * 32, v);
+        else
 #pragma unroll
-        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+        if (p.had) hadamard32(v, p.had);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
     }
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
     if (lane == 0 && m > 0.0f) atomicMax(p.amax_word, __float_as_uint(m));
@@ -253,20 +362,34 @@ int device_sm_count()
     return g_sms;
 }
 
-template <typename InT>
-static int launch_row(const QParams &p, int fast, cudaStream_t st, int *grid_out)
+template <typename InT, int B>
+static int launch_row_b(const QParams &p, int fast, cudaStream_t st, int *grid_out)
 {
-    const int64_t tiles = (p.rows * p.cols / 8 + 63) / 64;
+    const int64_t warps = (p.rows * p.cols / 32 + 31) / 32;
     if (fast) {
-        const int g = grid_for(k_quant_row<InT, true>, tiles);
-        k_quant_row<InT, true><<<g, kThreads, 0, st>>>(p);
+        const int g = grid_for(k_quant_row<InT, B, true>, warps);
+        k_quant_row<InT, B, true><<<g, kThreads, 0, st>>>(p);
         *grid_out = g;
     } else {
-        const int g = grid_for(k_quant_row<InT, false>, tiles);
-        k_quant_row<InT, false><<<g, kThreads, 0, st>>>(p);
+        const int g = grid_for(k_quant_row<InT, B, false>, warps);
+        k_quant_row<InT, B, false><<<g, kThreads, 0, st>>>(p);
         *grid_out = g;
     }
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+template <typename InT>
+static int launch_row(const QParams &p, int fast, cudaStream_t st, int *grid_out)
+{
+    switch (p.block) {
+    case 8: return launch_row_b<InT, 8>(p, fast, st, grid_out);
+    case 16: return launch_row_b<InT, 16>(p, fast, st, grid_out);
+    case 32: return launch_row_b<InT, 32>(p, fast, st, grid_out);
+    case 64: return launch_row_b<InT, 64>(p, fast, st, grid_out);
+    case 128: return launch_row_b<InT, 128>(p, fast, st, grid_out);
+    case 256: return launch_row_b<InT, 256>(p, fast, st, grid_out);
+    default: return -1;
+    }
 }
 
 int launch_quantize(const QParams &p, int axis, int in_fp32, int fast, cudaStream_t st, int *grid_out)
@@ -283,7 +406,7 @@ int launch_tensor_amax(const QParams &p, int axis, int in_fp32, cudaStream_t st)
     if (axis == AX_COL && p.had) {
         if (launch_amax_col(p, in_fp32, st)) return -1;
     } else {
-        const int64_t tiles = (p.rows * p.cols / 8 + 31) / 32;
+        const int64_t tiles = (p.rows * p.cols / 32 + 31) / 32;
         if (in_fp32) {
             const int g = grid_for(k_amax_row<float>, tiles);
             k_amax_row<float><<<g, kThreads, 0, st>>>(p);

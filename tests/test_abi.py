@@ -67,6 +67,7 @@ def test_query_sizes_host_only(mx):
     (dict(macro_block=64), 64, 128, -1),
     (dict(macro_block=128), 64, 96, -1),                  # cols % 128
     (dict(block=32), 64, 48, -1),                         # cols % block
+    (dict(block=16), 64, 16, -1),                         # cols % 32 (lanes walk 32-element chunks)
     (dict(rule=2, oas_tau=float("nan")), 64, 64, -1),
     (dict(elem=9), 64, 64, -1),
 ])
