@@ -167,6 +167,30 @@ int mx_quantize(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t ro
                 void *stream);
 
 /*
+ * mx_quantize_noalloc -- mx_quantize for callers that cannot allocate device
+ * memory: plain C callers holding no device allocator, code running while a
+ * CUDA graph is being captured (cudaMalloc is not allowed there), services
+ * that reserved all of HBM up front.  The pages have no counterpart: this is
+ * an interface convenience, not part of the method.
+ *   Same arguments and results as mx_quantize, without the workspace: the
+ *   scratch lives in a fixed device array inside the library (262,400 bytes,
+ *   the most mx_quantize can need: a 256-byte header and one 64-byte record
+ *   for each of at most 4096 CTAs), held by every GPU that loads the library
+ *   until the process exits.  A configuration needing more scratch is
+ *   rejected with MX_ERR_WORKSPACE.  Nothing is allocated: no cudaMalloc, no
+ *   cudaFree, no allocating library routine.
+ *   The first call on a device resolves the array's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture.  Every call shares the one array and leaves its contents behind
+ *   (the call clears what must start at zero), so calls that overlap on the
+ *   GPU -- on different streams, or from different threads -- race: order them
+ *   on one stream.  Rotation (mx_hadamard_quantize) is not covered.
+ */
+int mx_quantize_noalloc(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t rows,
+                        int64_t cols, void *codes, uint8_t *scales, float *tensor_scale,
+                        uint8_t *macro_scales, uint16_t *offsets, double *stats, void *stream);
+
+/*
  * mx_hadamard_quantize -- mx_quantize preceded, in the same pass, by the
  * block Hadamard rotation y = x H_n / sqrt(n), n = cfg->hadamard in {16, 32},
  * over groups of n consecutive elements along the block axis (the row

@@ -102,6 +102,7 @@ def lib() -> C.CDLL:
         L.mx_query_sizes.argtypes = [cfgp, i64, i64, C.POINTER(mx_sizes)]
         L.mx_quantize.argtypes = [cfgp, P, i32, i64, i64, P, P, P, P, P, P, P, i64, P]
         L.mx_hadamard_quantize.argtypes = [cfgp, P, i32, i64, i64, P, P, P, P, P, P, P, P, i64, P]
+        L.mx_quantize_noalloc.argtypes = [cfgp, P, i32, i64, i64, P, P, P, P, P, P, P]
         L.mx_dequantize.argtypes = [cfgp, P, P, P, P, P, i64, i64, P, i32, P]
         L.mx_qsnr_workspace_bytes.argtypes = [i64, i64]
         L.mx_qsnr_workspace_bytes.restype = i64
@@ -114,7 +115,7 @@ def lib() -> C.CDLL:
         L.mx_strerror.argtypes = [C.c_int]
         L.mx_strerror.restype = C.c_char_p
         L.mx_version.restype = C.c_char_p
-        for f in ("mx_query_sizes", "mx_quantize", "mx_hadamard_quantize", "mx_dequantize",
+        for f in ("mx_query_sizes", "mx_quantize", "mx_quantize_noalloc", "mx_hadamard_quantize", "mx_dequantize",
                   "mx_qsnr", "mx_gemm", "mx_gemm_qsnr", "mx_device_status"):
             getattr(L, f).restype = C.c_int
         _lib = L
@@ -173,6 +174,16 @@ def mx_quantize(cfg: Config, x, x_dtype, rows, cols, codes, scales, tensor_scale
     c = cfg.c()
     return lib().mx_quantize(C.byref(c), x, x_dtype, rows, cols, codes, scales, tensor_scale,
                              macro, offsets, stats, workspace, workspace_bytes, stream)
+
+
+def mx_quantize_noalloc(cfg: Config, x, x_dtype, rows, cols, codes, scales, tensor_scale, macro,
+                        offsets, stats, stream) -> int:
+    """mx_quantize without a workspace argument, for callers that cannot
+    allocate device memory; its scratch is a fixed array inside the library
+    shared by all calls (order the calls on one stream)."""
+    c = cfg.c()
+    return lib().mx_quantize_noalloc(C.byref(c), x, x_dtype, rows, cols, codes, scales,
+                                     tensor_scale, macro, offsets, stats, stream)
 
 
 def mx_hadamard_quantize(cfg: Config, x, x_dtype, rows, cols, codes, scales, tensor_scale, macro,
