@@ -55,6 +55,7 @@ def parse():
     ap.add_argument("--rows", type=int, default=16384)
     ap.add_argument("--cols", type=int, default=8192)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--no-stats", action="store_true", help="kernel cases: quantize without the fused stats")
     return ap.parse_args()
 
 
@@ -287,6 +288,8 @@ def run_ours(args, rank, world, device):
                 "algorithmic_bytes_per_launch": {"A": algo_bytes(mx.MXFP4, M_TOK, K_DIM, "q"),
                                                  "W": algo_bytes(mx.MXFP4, N_OUT, K_DIM, "q")}}
 
+    extra = run_extra_rows(mx, A, device, args)
+
     # end to end through the public API with host buffers
     e2e = run_e2e(mx, A_cpu, W_cpu, plan, outs, device, args, step_bytes, world)
 
@@ -297,7 +300,43 @@ def run_ours(args, rank, world, device):
     gemm = None if args.no_gemm else run_gemm(mx, A, W, device, args, world)
     return dict(value=value, ms_per_step=ms_per_step, step_bytes=step_bytes, launches=launches,
                 rows=rows, roofline=roofline, e2e=e2e, fidelity=fid, gemm=gemm,
-                clocks=clk.summary())
+                clocks=clk.summary(), extra=extra)
+
+
+def run_extra_rows(mx, A, device, args):
+    """The other rows of the path, outside the headline step: column and 2D
+    blocks on the activation tensor, and on a gradient-like fp32 4096 x 14336
+    tensor stochastic rounding, FP6, asymmetric INT4 and E3M0 with the ceil
+    scale.  Each launch is captured as a graph and replayed K times."""
+    from microscaling_block_quantization_b200 import inputs
+    G = inputs.gradient_like(4096, 14336, seed=5).to(device)
+    cases = [("mxfp4_col_A", A, mx.Config(axis=1)), ("mxfp4_2d_A", A, mx.Config(axis=2)),
+             ("e2m1_sr_grad_fp32", G, mx.Config(round=mx.ROUND_STOCHASTIC, seed=5)),
+             ("e2m3_grad_fp32", G, mx.Config(elem=mx.E2M3)),
+             ("int4_asym_grad_fp32", G, mx.Config(elem=mx.INT4, asymmetric=1, rule=mx.RULE_CEIL)),
+             ("e3m0_ceil_grad_fp32", G, mx.Config(elem=mx.E3M0, rule=mx.RULE_CEIL))]
+    out = {}
+    stream = torch.cuda.current_stream(device)
+    for name, x, cfg in cases:
+        q = mx.alloc_outputs(cfg, *x.shape, device, stats=True)
+        mx.quantize(x, cfg, out=q)
+        torch.cuda.synchronize(device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            mx.quantize(x, cfg, out=q)
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        ms = e0.elapsed_time(e1) / args.steps
+        nb = algo_bytes(cfg, *x.shape, "q", in_bytes=x.element_size())
+        out[name] = {"GB_per_s": round(nb / (ms * 1e-3) / 1e9, 1), "us": round(ms * 1e3, 2),
+                     "qsnr_db": round(float(q.stats[7].item()), 4), "bias": float(q.stats[8].item())}
+    del G
+    return out
 
 
 def run_e2e(mx, A_cpu, W_cpu, plan, outs, device, args, step_bytes, world):
@@ -486,7 +525,7 @@ def kernel_case(args):
     dev = torch.device("cuda", 0)
     g = torch.Generator(device=dev).manual_seed(0)
     case = args.kernel_case
-    res = {"case": case}
+    res = {"case": case, "stats": not args.no_stats}
     if case.startswith("gemm"):
         M, N, K = M_TOK, N_OUT, K_DIM
         cfg = (mx.Config(sf_layout=1) if case == "gemm_mxfp4" else
@@ -503,7 +542,7 @@ def kernel_case(args):
         cfg = {"quant_mxfp4_row": mx.MXFP4, "quant_nvfp4_row": mx.NVFP4,
                "quant_mxfp4_col": mx.Config(axis=1), "quant_mxfp4_2d": mx.Config(axis=2),
                "quant_had32_row": mx.Config(hadamard=32), "dequant_mxfp4_row": mx.MXFP4}[case]
-        q = mx.quantize(x, cfg)
+        q = mx.quantize(x, cfg, stats=not args.no_stats)
         if case.startswith("dequant"):
             out = torch.empty(R, Cc, dtype=torch.bfloat16, device=dev)
             run = lambda: mx.dequantize(q, out=out)
@@ -582,6 +621,7 @@ def main():
         "clocks": r["clocks"],
         "rows": r["rows"],
         "gemm": r["gemm"],
+        "extra_rows": r["extra"],
         "fidelity": r["fidelity"],
     }
     print(json.dumps(line), flush=True)

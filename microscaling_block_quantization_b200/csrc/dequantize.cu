@@ -131,11 +131,17 @@ __global__ void __launch_bounds__(kThreads) k_dequant_chunk(const DParams p)
                     else
                         sc = p.scales[(size_t)(row >> 5) * (p.cols >> 5) + (col >> 5)];
                     const float sb = scale_value(p.sd, sc);
+                    const float2 sb2 = make_float2(sb, sb), sT2 = make_float2(sT, sT);
                     float q[8];
                     e2m1x8_values(w[g], q);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        v[8 * g + i] = nearest ? __fmul_rn(__fmul_rn(q[i], sb), sT) : __fmul_rn(q[i], sb);
+                    for (int i = 0; i < 8; i += 2) {
+                        // (q * s_b) [* s_T], each product one binary32 rounding per lane
+                        float2 t = __fmul2_rn(make_float2(q[i], q[i + 1]), sb2);
+                        if (nearest) t = __fmul2_rn(t, sT2);
+                        v[8 * g + i] = t.x;
+                        v[8 * g + i + 1] = t.y;
+                    }
                 }
             } else {
 #pragma unroll

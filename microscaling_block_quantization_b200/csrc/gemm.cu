@@ -382,6 +382,201 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Persistent 128 x 256 variant for the FP4 kinds: one CTA per SM walks its
+// share of the output tiles; 4 stages of A (16 KB) + B (32 KB) + scales in
+// shared memory; the accumulator (256 TMEM columns) is released as soon as the
+// eight epilogue warps have moved it into registers, so the stores of tile i
+// overlap the MMAs of tile i + 1, and the producer keeps loading across tiles.
+constexpr int BNP = 256;
+constexpr int kStagesP = 4;
+constexpr int kThreadsP = 320;                 // producer, MMA, 8 epilogue warps
+constexpr int kTmemColsP = 512;
+
+template <int KIND>
+struct KindP {
+    static constexpr int kChunks = KIND == KIND_MXF4 ? 2 : 4;       // 4-scale chunks per stage (K = 256)
+    static constexpr int kSfaBytes = kChunks * 512;                  // 128 rows of A
+    static constexpr int kSfbBytes = 2 * kChunks * 512;              // 256 rows of B
+    static constexpr int kABytes = BM * 128, kBBytes = BNP * 128;
+    static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+    static constexpr int kSfCols = kChunks * 4 + 2 * kChunks * 4;    // TMEM columns per stage
+};
+
+template <int KIND>
+__device__ __forceinline__ uint32_t idesc_p()
+{
+    uint32_t d = (1u << 7) | (1u << 10);          // A, B E2M1
+    if (KIND == KIND_MXF4) d |= 1u << 23;        // UE8M0 scales
+    d |= (uint32_t)(BNP >> 3) << 17;
+    d |= (uint32_t)(BM >> 4) << 24;
+    return d;
+}
+
+template <int KIND, int EPI>
+__global__ void __launch_bounds__(kThreadsP, 1)
+    k_gemm_p(const GParams p, const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB)
+{
+    using KT = KindP<KIND>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *sA = smem;
+    uint8_t *sB = sA + kStagesP * KT::kABytes;
+    uint8_t *sSFA = sB + kStagesP * KT::kBBytes;
+    uint8_t *sSFB = sSFA + kStagesP * KT::kSfaBytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sSFB + kStagesP * KT::kSfbBytes);
+    uint64_t *empty = full + kStagesP;
+    uint64_t *accf = empty + kStagesP;            // accumulator full (MMA -> epilogue)
+    uint64_t *acce = accf + 1;                    // accumulator free (epilogue -> MMA)
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acce + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntn = p.N / BNP, ntm = p.M / BM;
+    const int ntiles = ntn * ntm;
+    const int ktiles = p.K / 256;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStagesP; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accf, 1);
+        mbar_init(acce, 8);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(saddr(tmem_holder)), "r"(kTmemColsP));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_holder;
+    const uint32_t tsf = tbase + BNP;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const int sf_chunks_row = (p.K / (KIND == KIND_MXF4 ? 32 : 16)) / 4;
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                const int m0 = (tile / ntn) * BM, n0 = (tile % ntn) * BNP;
+                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                    const int s = it % kStagesP;
+                    if (it >= (uint32_t)kStagesP && !mbar_wait(&empty[s], ((it / kStagesP) - 1) & 1, 11)) { ok = false; break; }
+                    mbar_expect_tx(&full[s], KT::kStageBytes);
+                    tma_load_2d(sA + s * KT::kABytes, &tmA, &full[s], kt * 128, m0);
+                    tma_load_2d(sB + s * KT::kBBytes, &tmB, &full[s], kt * 128, n0);
+                    const size_t ca = ((size_t)(m0 / 128) * sf_chunks_row + (size_t)kt * KT::kChunks) * 512;
+                    const size_t cb0 = ((size_t)(n0 / 128) * sf_chunks_row + (size_t)kt * KT::kChunks) * 512;
+                    const size_t cb1 = ((size_t)(n0 / 128 + 1) * sf_chunks_row + (size_t)kt * KT::kChunks) * 512;
+                    bulk_load(sSFA + s * KT::kSfaBytes, p.sfa + ca, KT::kSfaBytes, &full[s]);
+                    bulk_load(sSFB + s * KT::kSfbBytes, p.sfb + cb0, KT::kChunks * 512, &full[s]);
+                    bulk_load(sSFB + s * KT::kSfbBytes + KT::kChunks * 512, p.sfb + cb1, KT::kChunks * 512, &full[s]);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc0 = idesc_p<KIND>();
+            uint32_t it = 0, tcount = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tcount) {
+                // wait until the epilogue has drained the previous tile's accumulator
+                if (tcount > 0 && !mbar_wait(acce, (tcount - 1) & 1, 12)) { ok = false; break; }
+                tc_fence_after();
+                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                    const int s = it % kStagesP;
+                    if (!mbar_wait(&full[s], (it / kStagesP) & 1, 13)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sfa_t = tsf + s * KT::kSfCols;
+                    const uint32_t sfb_t = sfa_t + KT::kChunks * 4;
+#pragma unroll
+                    for (int c = 0; c < KT::kChunks; ++c) {
+                        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                                     ::"r"(sfa_t + 4 * c), "l"(desc_sf(saddr(sSFA + s * KT::kSfaBytes + c * 512))));
+                        // B rows 0..127 -> columns 8c..8c+3, rows 128..255 -> 8c+4..8c+7
+                        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                                     ::"r"(sfb_t + 8 * c), "l"(desc_sf(saddr(sSFB + s * KT::kSfbBytes + c * 512))));
+                        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                                     ::"r"(sfb_t + 8 * c + 4),
+                                       "l"(desc_sf(saddr(sSFB + s * KT::kSfbBytes + KT::kChunks * 512 + c * 512))));
+                    }
+                    const uint32_t a0 = saddr(sA + s * KT::kABytes), b0 = saddr(sB + s * KT::kBBytes);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        uint32_t idesc = idesc0, sfa, sfb;
+                        if constexpr (KIND == KIND_MXF4) {
+                            const uint32_t id = (k & 1) * 2;
+                            idesc |= (id << 29) | (id << 4);
+                            sfa = sfa_t + 4 * (k >> 1);
+                            sfb = sfb_t + 8 * (k >> 1);
+                        } else {
+                            sfa = sfa_t + 4 * k;
+                            sfb = sfb_t + 8 * k;
+                        }
+                        mma<KIND>(tbase, desc_sw128(a0 + 32 * k), desc_sw128(b0 + 32 * k), idesc, sfa, sfb,
+                                  (kt > 0 || k > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&empty[s]);
+                }
+                if (ok) tc_commit(accf);
+            }
+        }
+        __syncwarp();
+    } else {
+        // eight epilogue warps: quadrant q = warp % 4 (TMEM lanes), column half h
+        const int q = warp & 3, h = (warp - 2) >> 2;
+        float scale = 1.0f;
+        if (p.tsA) scale = __fmul_rn(scale, *p.tsA);
+        if (p.tsB) scale = __fmul_rn(scale, *p.tsB);
+        uint32_t tcount = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tcount) {
+            const int m0 = (tile / ntn) * BM, n0 = (tile % ntn) * BNP;
+            if (!mbar_wait(accf, tcount & 1, 14)) break;
+            tc_fence_after();
+            float v[128];
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch)
+                tmem_ld32(tbase + ((uint32_t)(32 * q) << 16) + h * 128 + ch * 32, v + 32 * ch);
+            // the accumulator is in registers: hand it back to the MMA warp
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(acce)) : "memory");
+            const int row = m0 + 32 * q + lane;
+            const int col = n0 + h * 128;
+            if constexpr (EPI == EPI_BF16) {
+                __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.C) + (size_t)row * p.N + col;
+#pragma unroll
+                for (int i = 0; i < 128; i += 8) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        __nv_bfloat162 t2 = __floats2bfloat162_rn(v[i + 2 * j] * scale, v[i + 2 * j + 1] * scale);
+                        w[j] = *reinterpret_cast<uint32_t *>(&t2);
+                    }
+                    *reinterpret_cast<uint4 *>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            } else {
+                float *dst = static_cast<float *>(p.C) + (size_t)row * p.N + col;
+#pragma unroll
+                for (int i = 0; i < 128; i += 4)
+                    *reinterpret_cast<float4 *>(dst + i) =
+                        make_float4(v[i] * scale, v[i + 1] * scale, v[i + 2] * scale, v[i + 3] * scale);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(kTmemColsP));
+    }
+}
+
 // Sum the per-CTA records in a fixed order: [sum C_ref^2, sum err^2, QSNR dB].
 __global__ void k_gemm_qsnr_finalize(const double *partials, int n, double *out)
 {
@@ -432,14 +627,14 @@ EncodeTiled encoder()
 }
 
 // rows x row_bytes operand, box of 128 rows x 128 bytes, 128-byte swizzle
-bool make_map(CUtensorMap *m, const void *base, int rows, int K, bool bf16)
+bool make_map(CUtensorMap *m, const void *base, int rows, int K, bool bf16, unsigned box_rows = 128)
 {
     EncodeTiled enc = encoder();
     if (!enc) return false;
     const cuuint64_t inner = bf16 ? (cuuint64_t)K : (cuuint64_t)K / 2;
     const cuuint64_t dims[2] = {inner, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {bf16 ? (cuuint64_t)K * 2 : (cuuint64_t)K / 2};
-    const cuuint32_t box[2] = {bf16 ? 64u : 128u, 128u};
+    const cuuint32_t box[2] = {bf16 ? 64u : 128u, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
                const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -464,6 +659,28 @@ int launch(const GParams &p, const void *A, const void *B, cudaStream_t st)
     }
     dim3 grid(p.N / BN, p.M / BM);
     k<<<grid, kThreads, smem, st>>>(p, ta, tb);
+    return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+}
+
+
+template <int KIND, int EPI>
+int launch_p(const GParams &p, const void *A, const void *B, cudaStream_t st)
+{
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, A, p.M, p.K, false, 128) || !make_map(&tb, B, p.N, p.K, false, 256)) return MX_ERR_CUDA;
+    using KT = KindP<KIND>;
+    const int smem = 1024 + kStagesP * KT::kStageBytes + 256;
+    auto k = k_gemm_p<KIND, EPI>;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return MX_ERR_CUDA;
+        attr = true;
+    }
+    const int tiles = (p.M / BM) * (p.N / BNP);
+    int grid = mxk::device_sm_count();
+    if (grid > tiles) grid = tiles;
+    k<<<grid, kThreadsP, smem, st>>>(p, ta, tb);
     return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
 
@@ -531,6 +748,13 @@ int mx_gemm(const mx_config *ca, const mx_config *cb, const void *Aq, const uint
     }
     p.C = C;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (N % BNP == 0) {
+        if (kind == KIND_MXF4)
+            return c_dtype == MX_DT_BF16 ? launch_p<KIND_MXF4, EPI_BF16>(p, Aq, Bq, st)
+                                         : launch_p<KIND_MXF4, EPI_F32>(p, Aq, Bq, st);
+        return c_dtype == MX_DT_BF16 ? launch_p<KIND_NVF4, EPI_BF16>(p, Aq, Bq, st)
+                                     : launch_p<KIND_NVF4, EPI_F32>(p, Aq, Bq, st);
+    }
     if (kind == KIND_MXF4)
         return c_dtype == MX_DT_BF16 ? launch<KIND_MXF4, EPI_BF16>(p, Aq, Bq, st)
                                      : launch<KIND_MXF4, EPI_F32>(p, Aq, Bq, st);

@@ -81,5 +81,8 @@ int cached_occupancy(const void *kernel, int threads, size_t smem);
 int launch_quantize_col(const QParams &p, int axis, int in_fp32, int fast, cudaStream_t st,
                         int *grid_out);
 int launch_amax_col(const QParams &p, int in_fp32, cudaStream_t st);
+// E2M1 round-to-nearest-even, symmetric, row axis, no macro scale, rotation
+// or rotated output: the TMA-fed persistent quantizer.
+int launch_quantize_fast(const QParams &p, int in_fp32, cudaStream_t st, int *grid_out);
 
 }  // namespace mxk

@@ -394,6 +394,9 @@ static int launch_row(const QParams &p, int fast, cudaStream_t st, int *grid_out
 
 int launch_quantize(const QParams &p, int axis, int in_fp32, int fast, cudaStream_t st, int *grid_out)
 {
+    if (axis == AX_ROW && fast && !p.rotated &&
+        ((!p.mbs && !p.had) || p.block == 16 || p.block == 32))
+        return launch_quantize_fast(p, in_fp32, st, grid_out);
     if (axis == AX_ROW)
         return in_fp32 ? launch_row<float>(p, fast, st, grid_out)
                        : launch_row<__nv_bfloat16>(p, fast, st, grid_out);

@@ -90,11 +90,13 @@ def check_gemm(mx, orc, name, M, N, K, out_dtype=torch.float32, seed=0):
 
 @pytest.mark.parametrize("name", ["mxfp4", "nvfp4"])
 def test_gemm_single_tile(mx, orc, name):
-    check_gemm(mx, orc, name, 128, 128, 256)
+    check_gemm(mx, orc, name, 128, 128, 256)        # 128 x 128 tile kernel
+    check_gemm(mx, orc, name, 128, 256, 256)        # persistent 128 x 256 kernel
 
 
 @pytest.mark.parametrize("name", ["mxfp4", "nvfp4"])
-@pytest.mark.parametrize("shape", [(256, 384, 1024), (384, 256, 2048), (128, 640, 768)])
+@pytest.mark.parametrize("shape", [(256, 384, 1024), (384, 256, 2048), (128, 640, 768),
+                                   (384, 512, 1280), (2048, 2560, 512)])
 def test_gemm_tiles_and_stage_ring(mx, orc, name, shape):
     check_gemm(mx, orc, name, *shape)
 
