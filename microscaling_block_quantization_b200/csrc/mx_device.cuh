@@ -233,6 +233,17 @@ __device__ __forceinline__ uint32_t ue_encode_rtne(const ScaleDesc &s, float x)
     return (uint32_t)code;
 }
 
+// UE4M3 nearest-even code of x through the sm_100a E4M3 conversion (round to
+// nearest even, saturating at 448); x <= 0 -> 0, NaN -> 0x7F.
+__device__ __forceinline__ uint32_t ue4m3_encode_hw(float x)
+{
+    if (x != x) return 0x7fu;
+    if (!(x > 0.0f)) return 0u;
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+    return (uint32_t)(r & 0xffu);
+}
+
 // Code of 2^k in the unsigned minifloat (k within [kmin, kmax]).
 __device__ __forceinline__ uint32_t ue_encode_pow2(const ScaleDesc &s, int k)
 {
@@ -281,7 +292,7 @@ __device__ __forceinline__ BlockScale block_scale(const ElemDesc &d, const Scale
     if (nonfinite) { r.code = (uint32_t)s.ue_nan_code; r.zero = 1; r.nan = 1; return r; }
     if (s.rule == R_NEAREST) {
         float sb_real = __fdiv_rn(__fdiv_rn(alpha, d.maxv), sT);
-        r.code = ue_encode_rtne(s, sb_real);
+        r.code = (s.fmt == S_UE4M3) ? ue4m3_encode_hw(sb_real) : ue_encode_rtne(s, sb_real);
         float sb = ue_value(s, r.code);
         r.deq = sb;
         if (sb != sb) { r.zero = 1; r.nan = 1; return r; }

@@ -14,6 +14,13 @@ namespace mxk {
 namespace {
 
 constexpr int kColWarps = 4;
+
+__device__ __forceinline__ float fmax_nan(float a, float b)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
 constexpr int kColThreads = kColWarps * 32;
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
@@ -228,6 +235,126 @@ __global__ void __launch_bounds__(kColThreads) k_quant_col(const QParams p)
 #pragma unroll
                     for (int j = 0; j < CPT; j += 4)
                         *reinterpret_cast<float4 *>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                }
+            }
+
+            // E2M1 round-to-nearest-even without macro scale or offset: one
+            // statistic pass (NaN-propagating abs max) and one encode pass with
+            // packed binary32 pairs
+            if constexpr (FAST) {
+                if (!p.mbs) {
+                    constexpr int NSF = (AXIS == AX_COL) ? CPT : 1;
+                    float a[NSF], mabs[NSF];
+#pragma unroll
+                    for (int s2 = 0; s2 < NSF; ++s2) { a[s2] = 0.0f; mabs[s2] = FLT_MAX; }
+                    for (int r = 0; r < RB; ++r) {
+                        float v[CPT];
+                        t.get(r, v);
+#pragma unroll
+                        for (int j = 0; j < CPT; ++j) {
+                            const int s2 = (AXIS == AX_COL) ? j : 0;
+                            a[s2] = fmax_nan(a[s2], fabsf(v[j]));
+                            mabs[s2] = fminf(mabs[s2], fabsf(v[j]));
+                        }
+                    }
+                    BlockScale bsf[NSF];
+#pragma unroll
+                    for (int s2 = 0; s2 < NSF; ++s2) {
+                        int bad = !(a[s2] <= FLT_MAX);
+                        float aa = bad ? 0.0f : a[s2];
+                        if (AXIS == AX_2D) {
+                            aa = grp_max(aa, G2);
+                            bad = grp_or(bad, G2);
+                            mabs[s2] = grp_min(mabs[s2], G2);
+                        }
+                        bsf[s2] = block_scale(p.ed, p.sd, aa, bad, sT);
+                    }
+                    if (ok) {
+                        if (AXIS == AX_COL) {
+                            uint8_t *dst = p.scales + (r0 / RB) * p.cols + c0;
+                            uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+                            for (int j = 0; j < CPT; ++j) {
+                                if (j < 4) w0 |= bsf[(AXIS == AX_COL) ? j : 0].code << (8 * j);
+                                else w1 |= bsf[(AXIS == AX_COL) ? j : 0].code << (8 * (j - 4));
+                            }
+                            if constexpr (CPT == 8) *reinterpret_cast<uint2 *>(dst) = make_uint2(w0, w1);
+                            else *reinterpret_cast<uint32_t *>(dst) = w0;
+                        } else if ((lane & (G2 - 1)) == 0) {
+                            p.scales[(r0 / 32) * (p.cols / 32) + c0 / 32] = (uint8_t)bsf[0].code;
+                        }
+                    }
+                    const bool nearest = p.sd.fmt != S_E8M0 && p.sd.rule == R_NEAREST;
+                    float deqT[NSF];
+#pragma unroll
+                    for (int s2 = 0; s2 < NSF; ++s2)
+                        deqT[s2] = bsf[s2].nan ? __uint_as_float(0x7fc00000u)
+                                 : nearest ? __fmul_rn(bsf[s2].deq, sT) : bsf[s2].deq;
+                    float2 sx2 = make_float2(0.f, 0.f), se2 = sx2, sb2 = sx2;
+                    int qzc[NSF];
+#pragma unroll
+                    for (int s2 = 0; s2 < NSF; ++s2) qzc[s2] = 0;
+                    for (int r = 0; r < RB; ++r) {
+                        const int64_t e0 = (r0 + r) * p.cols + c0;
+                        float v[CPT];
+                        t.get(r, v);
+                        float s8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+                        for (int j = 0; j < CPT; j += 2) {
+                            const int sa = (AXIS == AX_COL) ? j : 0, sb_ = (AXIS == AX_COL) ? j + 1 : 0;
+                            const float2 pr = __fmul2_rn(make_float2(v[j], v[j + 1]),
+                                                         make_float2(bsf[sa].inv, bsf[sb_].inv));
+                            s8[j] = bsf[sa].zero ? 0.0f : pr.x;
+                            s8[j + 1] = bsf[sb_].zero ? 0.0f : pr.y;
+                        }
+                        uint32_t lo = cvt_e2m1x8(s8);
+                        if (CPT == 4) lo &= 0xffffu;
+                        if (ok) {
+                            uint8_t *dst = static_cast<uint8_t *>(p.codes) + e0 / 2;
+                            if constexpr (CPT == 8) *reinterpret_cast<uint32_t *>(dst) = lo;
+                            else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)lo;
+                        }
+                        if (stats && ok) {
+                            float q[8];
+                            e2m1x8_values(lo, q);
+#pragma unroll
+                            for (int j = 0; j < CPT; j += 2) {
+                                const int sa = (AXIS == AX_COL) ? j : 0, sb_ = (AXIS == AX_COL) ? j + 1 : 0;
+                                const float2 yv = make_float2(v[j], v[j + 1]);
+                                const float2 d = __ffma2_rn(make_float2(q[j], q[j + 1]),
+                                                            make_float2(-deqT[sa], -deqT[sb_]), yv);
+                                se2 = __ffma2_rn(d, d, se2);
+                                sx2 = __ffma2_rn(yv, yv, sx2);
+                                sb2 = __fadd2_rn(sb2, d);
+                            }
+#pragma unroll
+                            for (int j = 0; j < CPT; ++j) {
+                                const int s2 = (AXIS == AX_COL) ? j : 0;
+                                qzc[s2] += ((lo >> (4 * j)) & 7u) == 0u;
+                            }
+                        }
+                    }
+                    if (stats && ok) {
+                        acc.x2 += (double)(sx2.x + sx2.y);
+                        acc.e2 += (double)(se2.x + se2.y);
+                        acc.e += -(double)(sb2.x + sb2.y);
+#pragma unroll
+                        for (int s2 = 0; s2 < NSF; ++s2) {
+                            int xz = 0;
+                            if (mabs[s2] == 0.0f)
+                                for (int r = 0; r < RB; ++r) {
+                                    float v[CPT];
+                                    t.get(r, v);
+#pragma unroll
+                                    for (int j = 0; j < CPT; ++j)
+                                        if ((AXIS == AX_COL) ? j == s2 : true) xz += (v[j] == 0.0f);
+                                }
+                            const int n_lane = (AXIS == AX_COL) ? RB : RB * CPT;
+                            acc.nz += (double)(n_lane - xz);
+                            if (!bsf[s2].nan) acc.ftz += (double)(qzc[s2] - xz);
+                        }
+                    }
+                    continue;
                 }
             }
 

@@ -121,7 +121,7 @@ __device__ __forceinline__ void hadamard32(float y[32], int n)
 // HAD: block rotation before quantization; MBS: 1 x 128 macro scale over the
 // 4 lanes of a macro block (consecutive chunks of a tile are consecutive lanes).
 template <typename InT, int B, bool STATS, bool HAD, bool MBS>
-__global__ void __launch_bounds__(kFastThreads) k_quant_fast(const QParams p, const __grid_constant__ CUtensorMap tm)
+__global__ void __launch_bounds__(kFastThreads, (HAD || MBS) ? 2 : 3) k_quant_fast(const QParams p, const __grid_constant__ CUtensorMap tm)
 {
     using FC = FastCfg<InT>;
     constexpr int NB = B <= 32 ? 32 / B : 1;
