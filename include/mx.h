@@ -10,6 +10,11 @@
  * Ownership: the caller owns every buffer.  The library allocates no device
  * memory; scratch space ("workspace") is passed in by the caller, sized by
  * mx_query_sizes() / mx_qsnr_workspace_bytes() / mx_gemm_workspace_bytes().
+ * The first 256 bytes of a workspace are the library's control words (the
+ * tensor-amax accumulator and a launch ticket): zero them once, before the
+ * first call that uses the workspace (cudaMemset); every call leaves them
+ * zero, so a workspace stays usable as long as calls sharing it are ordered
+ * on one stream.
  * Buffers must stay alive until the stream reaches the end of the call.
  *
  * Sources (the pages this library follows):
@@ -155,9 +160,13 @@ int mx_query_sizes(const mx_config *cfg, int64_t rows, int64_t cols, mx_sizes *o
  *   stats      device out, MX_STATS_LEN doubles, or NULL: fidelity of the
  *              dequantized tensor against x, fused into the same pass.
  *   workspace  device scratch of sizes.workspace_bytes (needed when stats != NULL
- *              or cfg->tensor_scale == MX_TS_COMPUTE).
+ *              or cfg->tensor_scale == MX_TS_COMPUTE), control words zeroed
+ *              before first use (see Ownership above).  The last CTA of the
+ *              quantizer launch sums the statistics and clears the control
+ *              words: one launch per call (two with a computed tensor scale:
+ *              the amax pre-pass, then the quantizer).
  * Shapes: cols % 32 == 0 always (lanes walk rows in 32-element chunks),
- * rows * cols < 2^40, cols % block == 0 (row), rows % block == 0 (column),
+ * rows * cols < 2^36, cols % block == 0 (row), rows % block == 0 (column),
  * rows % 32 == 0 (2D), % 128 along the axis for MBS.  Block non-finite
  * values give the NaN scale code and zero element codes.
  */
@@ -181,8 +190,8 @@ int mx_quantize(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t ro
  *   cudaFree, no allocating library routine.
  *   The first call on a device resolves the array's device address (once per
  *   device, with that device current); make that first call before any stream
- *   capture.  Every call shares the one array and leaves its contents behind
- *   (the call clears what must start at zero), so calls that overlap on the
+ *   capture.  Every call shares the one array (zero at load; every call
+ *   leaves its control words zero), so calls that overlap on the
  *   GPU -- on different streams, or from different threads -- race: order them
  *   on one stream.  Rotation (mx_hadamard_quantize) is not covered.
  */
@@ -258,8 +267,12 @@ int mx_gemm_qsnr(const mx_config *ca, const mx_config *cb, const void *A, const 
                  const uint8_t *Bsf, const float *tsA, const float *tsB, double *stats,
                  void *workspace, int64_t workspace_bytes, void *stream);
 
-/* Device status word of the bounded in-kernel waits (GEMM pipeline): reads
- * and clears it (synchronises `stream`).  *status = 0 when no wait gave up. */
+/* Status words of the bounded in-kernel waits: reads and clears them
+ * (synchronises `stream`).  *status = 0 when no wait gave up, else the code of
+ * the first wait that did: 1-3 and 11-14 the GEMM pipelines, 21-22 the E2M1
+ * nearest-even quantizer's TMA ring, 31-32 the other element types' ring.  A
+ * kernel whose wait gave up has left its loop early, so its outputs are
+ * incomplete; the library has no counterpart on the pages. */
 int mx_device_status(void *stream, int32_t *status);
 
 /* Human-readable text of a status code. */

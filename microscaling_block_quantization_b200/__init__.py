@@ -244,7 +244,9 @@ class Quantized:
 
 
 class Workspace:
-    """Caller-owned scratch buffer, reused across calls."""
+    """Caller-owned scratch buffer, reused across calls.  Allocated zeroed: its
+    first 256 bytes are the library's control words, which must be zero before
+    the first call and which every call leaves zero."""
 
     def __init__(self, device=None):
         self.device = device
@@ -252,7 +254,7 @@ class Workspace:
 
     def get(self, nbytes: int, device) -> torch.Tensor:
         if self.buf is None or self.buf.numel() < nbytes or self.buf.device != device:
-            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+            self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
         return self.buf
 
 

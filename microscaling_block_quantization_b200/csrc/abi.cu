@@ -108,7 +108,8 @@ int check_config(const mx_config *c, int64_t rows, int64_t cols, bool want_had)
     if (rows == 0 || cols == 0) return MX_OK;
     // kernels walk rows in 32-element chunks (one per lane)
     if (cols % 32) return MX_ERR_INVALID;
-    if (rows > (INT64_C(1) << 40) / cols) return MX_ERR_INVALID;
+    // fewer than 2^31 chunks: 32-bit chunk indices and TMA coordinates
+    if (rows > ((INT64_C(1) << 36) - 1) / cols) return MX_ERR_INVALID;
     if (c->axis == MX_AXIS_ROW && cols % B) return MX_ERR_INVALID;
     if (c->sf_layout == 1 && (rows % 128 || (cols / B) % 4)) return MX_ERR_INVALID;
     if (c->axis == MX_AXIS_COL && rows % B) return MX_ERR_INVALID;
@@ -200,15 +201,16 @@ int quantize_impl(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t 
     double *partials = ws ? reinterpret_cast<double *>(ws + kWsHeader) : nullptr;
     const int in_fp32 = x_dtype == MX_DT_FP32;
 
-    if (cfg->tensor_scale == MX_TS_COMPUTE) {
-        if (launch_tensor_amax(p, cfg->axis, in_fp32, st)) return MX_ERR_CUDA;
-        if (launch_finalize_tensor_scale(p, st)) return MX_ERR_CUDA;
-    }
+    // the tensor-amax pre-pass; the quantizer derives s_T from its word
+    if (cfg->tensor_scale == MX_TS_COMPUTE && launch_tensor_amax(p, cfg->axis, in_fp32, st))
+        return MX_ERR_CUDA;
     p.partials = stats ? partials : nullptr;
+    p.stats = stats;
+    p.count = (double)n;
+    p.ticket = need_ws ? reinterpret_cast<unsigned int *>(ws + kWsTicket) : nullptr;
     const int fast = cfg->elem == MX_E2M1 && cfg->round == MX_ROUND_RTNE && !cfg->asymmetric;
     int grid = 0;
     if (launch_quantize(p, cfg->axis, in_fp32, fast, st, &grid)) return MX_ERR_CUDA;
-    if (stats && launch_finalize_stats(partials, grid, (double)n, stats, st)) return MX_ERR_CUDA;
     return MX_OK;
 }
 

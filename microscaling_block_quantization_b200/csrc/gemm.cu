@@ -807,7 +807,9 @@ int mx_device_status(void *stream, int32_t *status)
     if (cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
         return MX_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return MX_ERR_CUDA;
-    *status = v;
+    int vf = 0, vg = 0;
+    if (mxk::take_status_fast(st, &vf) || mxk::take_status_gen(st, &vg)) return MX_ERR_CUDA;
+    *status = v ? v : vf ? vf : vg;
     return MX_OK;
 }
 

@@ -189,6 +189,49 @@ __device__ __forceinline__ void e2m1x8_values(uint32_t packed, float out[8])
     }
 }
 
+// Eight E2M1 nibbles -> their grid values without the conversion
+// instruction: the magnitude bits moved to bits 22..24 form the binary32
+// denormal m * 2^-127, so one exact multiply by 2^126 gives the grid value
+// (0, 0.5, 1, 1.5, 2, 3, 4, 6); the nibble's sign bit becomes bit 31.
+__device__ __forceinline__ void e2m1x8_values_alu(uint32_t packed, float out[8])
+{
+#pragma unroll
+    for (int j = 0; j < 8; j += 2) {
+        const uint32_t t0 = packed >> (4 * j), t1 = packed >> (4 * j + 4);
+        const float2 d = make_float2(bits2f(((t0 & 7u) << 22) | ((t0 & 8u) << 28)),
+                                     bits2f(((t1 & 7u) << 22) | ((t1 & 8u) << 28)));
+        const float2 v = __fmul2_rn(d, make_float2(0x1p126f, 0x1p126f));
+        out[j] = v.x;
+        out[j + 1] = v.y;
+    }
+}
+
+// Eight E2M1 nibbles -> four f16x2 words of their grid values (exact).
+__device__ __forceinline__ void e2m1x8_halves(uint32_t packed, uint32_t h[4])
+{
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(packed));
+}
+
+// (s0 - q0, s1 - q1) in binary32, q the two halves of an f16x2 word: one
+// mixed-precision multiply-add per lane (q * -1 + s, a single rounding).
+__device__ __forceinline__ float2 sub_f16x2_from(float s0, float s1, uint32_t qh)
+{
+    float d0, d1;
+    asm("{\n\t.reg .f16 q0, q1, m1;\n\t"
+        "mov.b32 {q0, q1}, %2;\n\t"
+        "mov.b16 m1, 0xBC00;\n\t"
+        "fma.rn.f32.f16 %0, q0, m1, %3;\n\t"
+        "fma.rn.f32.f16 %1, q1, m1, %4;\n\t}"
+        : "=f"(d0), "=f"(d1) : "r"(qh), "f"(s0), "f"(s1));
+    return make_float2(d0, d1);
+}
+
 // E2M1 code -> value (sign-magnitude nibble)
 __device__ __forceinline__ float e2m1_value(uint32_t code)
 {
@@ -309,6 +352,76 @@ __device__ __forceinline__ BlockScale block_scale(const ElemDesc &d, const Scale
     r.inv = exp2i(-k);
     r.deq = exp2i(k);
     return r;
+}
+
+// Correctly rounded a / b from y = RN(1/b) (b and y normal): q0 = RN(a y)
+// is within 2 ulp of a/b; one residual correction, r = a - b q evaluated by
+// the fused multiply-add, brings it within 1 ulp, and a second one is
+// Markstein's theorem (Markstein, IBM J. Res. Develop. 34(1), 1990): with y
+// within half an ulp of 1/b and q within one ulp of a/b, RN(q + (a - b q) y)
+// is RN(a/b).  Quotients outside the normal range take the IEEE division.
+__device__ __forceinline__ float div_by_recip(float a, float b, float y)
+{
+    const float q0 = __fmul_rn(a, y);
+    if (!(q0 >= 0x1p-124f && q0 <= 0x1p124f)) return __fdiv_rn(a, b);
+    const float q1 = __fmaf_rn(__fmaf_rn(-q0, b, a), y, q0);
+    return __fmaf_rn(__fmaf_rn(-q1, b, a), y, q1);
+}
+
+// Per-launch constants of the nearest (UE4M3 / UE5M3) block scale.
+struct NearScale {
+    float maxv, r_max;      // largest element magnitude and RN(1 / maxv)
+    float sT, r_T;          // tensor scale and RN(1 / sT); r_T = 0: IEEE division
+    const float *inv_tab;   // per scale code: RN(1 / RN(s_b sT)); +inf = zero block
+};
+
+// Same result as block_scale() with a nearest rule: the two quotients of
+// s_b = RTNE((alpha / max) / s_T) through div_by_recip, and the element
+// multiplier from the launch's table of reciprocals.
+__device__ __forceinline__ BlockScale near_block_scale(const ScaleDesc &s, const NearScale &ns, float alpha,
+                                                       int nonfinite)
+{
+    BlockScale r;
+    r.zero = 0; r.nan = 0; r.inv = 0.0f; r.deq = 0.0f;
+    if (nonfinite) { r.code = (uint32_t)s.ue_nan_code; r.zero = 1; r.nan = 1; return r; }
+    const float q1 = div_by_recip(alpha, ns.maxv, ns.r_max);
+    const float sb_real = ns.sT == 1.0f ? q1
+                        : ns.r_T != 0.0f ? div_by_recip(q1, ns.sT, ns.r_T) : __fdiv_rn(q1, ns.sT);
+    r.code = (s.fmt == S_UE4M3) ? ue4m3_encode_hw(sb_real) : ue_encode_rtne(s, sb_real);
+    const float sb = ue_value(s, r.code);
+    r.deq = sb;
+    if (sb != sb) { r.zero = 1; r.nan = 1; return r; }
+    r.inv = ns.inv_tab[r.code];
+    r.zero = !(r.inv < __uint_as_float(0x7f800000u));
+    return r;
+}
+
+// E8M0 scale of a block without branches: k = e - emax (+1 when the
+// significand times 2^emax exceeds thr: the ceil rule with thr = max element,
+// OAS with thr = tau, floor with thr = +inf), clamped to [-127, 127]; a zero
+// or subnormal alpha lands on k = -127, the code of the zero block.
+// thr_m = thr / 2^emax.
+__device__ __forceinline__ BlockScale e8m0_block_scale(float alpha, int nonfinite, int emax, float thr_m)
+{
+    const uint32_t b = __float_as_uint(alpha);
+    const int ef = (int)(b >> 23);
+    const float m = __uint_as_float((b & 0x7fffffu) | 0x3f800000u);
+    int k = ef - 127 - emax + (m > thr_m ? 1 : 0);
+    k = ef == 0 ? -127 : min(max(k, -127), 127);
+    BlockScale r;
+    r.code = nonfinite ? 0xffu : (uint32_t)(k + 127);
+    r.zero = nonfinite || alpha == 0.0f;
+    r.nan = nonfinite;
+    r.inv = __uint_as_float(k <= 126 ? (uint32_t)(127 - k) << 23 : 0x00400000u);
+    r.deq = __uint_as_float(k >= -126 ? (uint32_t)(k + 127) << 23 : 0x00400000u);
+    return r;
+}
+
+// thr_m of e8m0_block_scale for a launch
+__device__ __forceinline__ float e8m0_threshold(const ElemDesc &d, const ScaleDesc &s)
+{
+    const float thr = s.rule == R_CEIL ? d.maxv : s.rule == R_OAS ? s.tau : __uint_as_float(0x7f800000u);
+    return __fmul_rn(thr, __uint_as_float((uint32_t)(127 - d.emax) << 23));
 }
 
 // E4M3 (positive) for the MBS macro scale: nearest-even code of x in

@@ -11,8 +11,11 @@ namespace mxk {
 // record of kPartialDoubles doubles into the caller's workspace.
 constexpr int kMaxPartials = 4096;
 constexpr int kPartialDoubles = 8;
-// workspace: [0, 256) control words (tensor amax), then the partials
+// workspace: [0, 256) control words, then the partials.  Control words: the
+// tensor-amax accumulator at byte 0, the launch ticket at byte 64.  Both are
+// zero before a launch and the launch's last CTA leaves them zero.
 constexpr int64_t kWsHeader = 256;
+constexpr int64_t kWsTicket = 64;
 constexpr int64_t kWorkspaceBytes = kWsHeader + (int64_t)kMaxPartials * kPartialDoubles * 8;
 
 struct QParams {
@@ -26,6 +29,9 @@ struct QParams {
     float *rotated;          // y output (fp32), or null
     double *partials;        // per-CTA stats records, or null (no stats)
     unsigned int *amax_word; // tensor-amax accumulator (AMAX launches)
+    unsigned int *ticket;    // CTAs finished (stats or a computed tensor scale), or null
+    double *stats;           // MX_STATS_LEN doubles, written by the last CTA
+    double count;            // elements
     ElemDesc ed;
     ScaleDesc sd;
     int block;               // B
@@ -67,7 +73,6 @@ struct SParams {
 int launch_quantize(const QParams &p, int axis, int in_fp32, int fast, cudaStream_t st,
                     int *grid_out);
 int launch_tensor_amax(const QParams &p, int axis, int in_fp32, cudaStream_t st);
-int launch_finalize_tensor_scale(const QParams &p, cudaStream_t st);
 int launch_dequantize(const DParams &p, cudaStream_t st);
 int launch_qsnr(const SParams &p, cudaStream_t st, int *grid_out);
 int launch_finalize_stats(const double *partials, int nparts, double count, double *stats,
@@ -84,5 +89,12 @@ int launch_amax_col(const QParams &p, int in_fp32, cudaStream_t st);
 // E2M1 round-to-nearest-even, symmetric, row axis, no macro scale, rotation
 // or rotated output: the TMA-fed persistent quantizer.
 int launch_quantize_fast(const QParams &p, int in_fp32, cudaStream_t st, int *grid_out);
+// Other element types / rounding modes / offsets, row axis, blocks of 32, no
+// macro scale, rotation or rotated output: the TMA-fed persistent quantizer.
+int launch_quantize_gen(const QParams &p, int in_fp32, cudaStream_t st, int *grid_out);
+// Read and clear the status words of the two persistent quantizers'
+// bounded waits (synchronise st); 0 when no wait gave up.
+int take_status_fast(cudaStream_t st, int *v);
+int take_status_gen(cudaStream_t st, int *v);
 
 }  // namespace mxk

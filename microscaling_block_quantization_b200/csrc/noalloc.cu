@@ -55,9 +55,9 @@ extern "C" int mx_quantize_noalloc(const mx_config *cfg, const void *x, int32_t 
     void *scratch = nullptr;
     rc = scratch_for_current_device(&scratch);
     if (rc != MX_OK) return rc;
-    // The scratch needs no clearing: the tensor-amax word is zeroed on the
-    // stream by mx_quantize before use, and every statistics record it reads
-    // is written earlier in the same call.
+    // The scratch needs no clearing: its control words are zero at load and
+    // every call leaves them zero, and every statistics record a call reads is
+    // written earlier in the same call.
     return mx_quantize(cfg, x, x_dtype, rows, cols, codes, scales, tensor_scale, macro_scales, offsets,
                        stats, scratch, kScratchBytes, stream);
 }

@@ -15,6 +15,28 @@ namespace mxk {
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kThreads = 256;
 
+// maximum that propagates NaN (the non-finite block test reads it)
+__device__ __forceinline__ float fmax_nan(float a, float b)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+// three-operand maximum / minimum (sm_100)
+__device__ __forceinline__ float fmax3_nan(float a, float b, float c)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c)
+{
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // ------------------------------------------------------------------ loads --
 __device__ __forceinline__ void unpack_bf16x2(uint32_t w, float &lo, float &hi)
 {
@@ -138,6 +160,71 @@ static __device__ __forceinline__ void write_partials(double *partials, const Ac
         double *o = partials + (int64_t)blockIdx.x * kPartialDoubles;
         for (int i = 0; i < 5; ++i) o[i] = s[i];
         o[5] = o[6] = o[7] = 0.0;
+    }
+}
+
+// Tensor scale of a launch: given, or s_T = amax / (max_elem * scale_max)
+// from the tensor-amax word of the pre-pass (amax = 0 -> 1); CTA 0 stores it.
+__device__ __forceinline__ float launch_tensor_scale(const QParams &p)
+{
+    if (p.ts_mode == TS_NONE) return 1.0f;
+    if (p.ts_mode == TS_GIVEN) return *p.tensor_scale;
+    const float amax = __uint_as_float(__ldcg(p.amax_word));
+    const float ts = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, __fmul_rn(p.ed.maxv, p.sd.ue_maxv));
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.tensor_scale = ts;
+    return ts;
+}
+
+// The derived statistics of the summed records: MSE, R-MSE, QSNR Eq. (1),
+// bias and the flush-to-zero share.
+__device__ __forceinline__ void store_stats(double *stats, const double s[5], double count)
+{
+    const double x2 = s[0], e2 = s[1], e = s[2], ftz = s[3], nz = s[4];
+    stats[0] = x2;
+    stats[1] = e2;
+    stats[2] = e;
+    stats[3] = ftz;
+    stats[4] = nz;
+    const double mse = count > 0 ? e2 / count : 0.0;
+    stats[5] = mse;
+    stats[6] = sqrt(mse);
+    stats[7] = (x2 == 0.0) ? __longlong_as_double(0x7ff8000000000000ll)
+             : (e2 == 0.0) ? __longlong_as_double(0x7ff0000000000000ll)
+                           : 10.0 * log10(x2 / e2);
+    stats[8] = count > 0 ? e / count : 0.0;
+    stats[9] = nz > 0 ? ftz / nz : 0.0;
+    stats[10] = count;
+    for (int k = 11; k < 16; ++k) stats[k] = 0.0;
+}
+
+// Epilogue of a quantizer launch (every thread of the CTA calls it): this
+// CTA's record of the fidelity sums; then the last CTA to finish sums all
+// records in a fixed order into the statistics, and clears the tensor-amax
+// word and the ticket.
+__device__ __forceinline__ void finish_launch(const QParams &p, const Acc &a)
+{
+    if (p.partials) write_partials(p.partials, a);
+    if (!p.ticket) return;
+    __shared__ unsigned s_last;
+    if (threadIdx.x == 0) {
+        __threadfence();
+        s_last = atomicAdd(p.ticket, 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (!s_last || threadIdx.x >= 32) return;
+    __threadfence();
+    if (p.partials) {
+        double s[5] = {0, 0, 0, 0, 0};
+        for (unsigned i = threadIdx.x; i < gridDim.x; i += 32)
+#pragma unroll
+            for (int k = 0; k < 5; ++k) s[k] += __ldcg(p.partials + (size_t)i * kPartialDoubles + k);
+#pragma unroll
+        for (int k = 0; k < 5; ++k) s[k] = warp_sum(s[k]);
+        if (threadIdx.x == 0) store_stats(p.stats, s, p.count);
+    }
+    if (threadIdx.x == 0) {
+        if (p.ts_mode == TS_COMPUTE) *p.amax_word = 0u;
+        *p.ticket = 0u;
     }
 }
 

@@ -15,12 +15,6 @@ namespace {
 
 constexpr int kColWarps = 4;
 
-__device__ __forceinline__ float fmax_nan(float a, float b)
-{
-    float r;
-    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
-    return r;
-}
 constexpr int kColThreads = kColWarps * 32;
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
@@ -173,7 +167,7 @@ __global__ void __launch_bounds__(kColThreads) k_quant_col(const QParams p)
     const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const bool stats = p.partials != nullptr;
-    const float sT = (p.ts_mode != TS_NONE) ? *p.tensor_scale : 1.0f;
+    const float sT = launch_tensor_scale(p);
     constexpr int G2 = 32 / CPT;            // lanes of a 2D tile row
     constexpr int MG = 128 / CPT;           // lanes of a 1 x 128 macro block (2D)
     constexpr int NS = (AXIS == AX_COL) ? CPT : 1;   // blocks held by a lane
@@ -316,7 +310,7 @@ __global__ void __launch_bounds__(kColThreads) k_quant_col(const QParams p)
                         }
                         if (stats && ok) {
                             float q[8];
-                            e2m1x8_values(lo, q);
+                            e2m1x8_values_alu(lo, q);
 #pragma unroll
                             for (int j = 0; j < CPT; j += 2) {
                                 const int sa = (AXIS == AX_COL) ? j : 0, sb_ = (AXIS == AX_COL) ? j + 1 : 0;
@@ -528,7 +522,7 @@ __global__ void __launch_bounds__(kColThreads) k_quant_col(const QParams p)
             }
         }
     }
-    if (stats) write_partials(p.partials, acc);
+    finish_launch(p, acc);
 }
 
 // Tensor absmax with the rotation along columns (column axis with rotation)

@@ -23,12 +23,6 @@ namespace mxk {
 // A 1 x 128 macro block spans 4 lanes; a 16- or 32-point rotation group lies
 // inside the thread.
 
-__device__ __forceinline__ float fmax_nan(float a, float b)
-{
-    float r;
-    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
-    return r;
-}
 
 __device__ __forceinline__ void load32(const __nv_bfloat16 *x, int64_t e, float v[32])
 {
@@ -96,7 +90,7 @@ __global__ void __launch_bounds__(kThreads) k_quant_row(const QParams p)
     const uint32_t gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const uint32_t nw = (gridDim.x * blockDim.x) >> 5;
     const bool stats = p.partials != nullptr;
-    const float sT = (p.ts_mode != TS_NONE) ? *p.tensor_scale : 1.0f;
+    const float sT = launch_tensor_scale(p);
     const bool nearest = p.sd.fmt != S_E8M0 && p.sd.rule == R_NEAREST;
     const uint32_t S = (uint32_t)(p.cols / B);  // scales per row
     Acc acc = {0, 0, 0, 0, 0};
@@ -262,7 +256,7 @@ __global__ void __launch_bounds__(kThreads) k_quant_row(const QParams p)
             }
         }
     }
-    if (stats) write_partials(p.partials, acc);
+    finish_launch(p, acc);
 }
 
 // Tensor absmax of y (NaN skipped) for the per-tensor scale, row chunks
@@ -291,14 +285,6 @@ __global__ void __launch_bounds__(kThreads) k_amax_row(const QParams p)
     if (lane == 0 && m > 0.0f) atomicMax(p.amax_word, __float_as_uint(m));
 }
 
-// s_T = amax_T / (max_elem * max_scale); amax_T = 0 gives 1
-__global__ void k_finalize_tensor_scale(const unsigned int *amax_word, float maxv, float smax,
-                                        float *ts)
-{
-    const float amax = __uint_as_float(*amax_word);
-    *ts = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, __fmul_rn(maxv, smax));
-}
-
 // Sum the per-CTA records in a fixed order and derive MSE, R-MSE, QSNR (Eq. (1)),
 // bias and the flush-to-zero share.
 __global__ void k_finalize_stats(const double *partials, int nparts, double count, double *stats)
@@ -315,22 +301,8 @@ __global__ void k_finalize_stats(const double *partials, int nparts, double coun
         __syncthreads();
     }
     if (threadIdx.x == 0) {
-        double x2 = sh[0][0], e2 = sh[0][1], e = sh[0][2], ftz = sh[0][3], nz = sh[0][4];
-        stats[0] = x2;
-        stats[1] = e2;
-        stats[2] = e;
-        stats[3] = ftz;
-        stats[4] = nz;
-        const double mse = count > 0 ? e2 / count : 0.0;
-        stats[5] = mse;
-        stats[6] = sqrt(mse);
-        stats[7] = (x2 == 0.0) ? __longlong_as_double(0x7ff8000000000000ll)
-                 : (e2 == 0.0) ? __longlong_as_double(0x7ff0000000000000ll)
-                               : 10.0 * log10(x2 / e2);
-        stats[8] = count > 0 ? e / count : 0.0;
-        stats[9] = nz > 0 ? ftz / nz : 0.0;
-        stats[10] = count;
-        for (int k = 11; k < 16; ++k) stats[k] = 0.0;
+        const double t[5] = {sh[0][0], sh[0][1], sh[0][2], sh[0][3], sh[0][4]};
+        store_stats(stats, t, count);
     }
 }
 
@@ -397,6 +369,8 @@ int launch_quantize(const QParams &p, int axis, int in_fp32, int fast, cudaStrea
     if (axis == AX_ROW && fast && !p.rotated &&
         ((!p.mbs && !p.had) || p.block == 16 || p.block == 32))
         return launch_quantize_fast(p, in_fp32, st, grid_out);
+    if (axis == AX_ROW && !fast && !p.rotated && !p.mbs && !p.had && p.block == 32)
+        return launch_quantize_gen(p, in_fp32, st, grid_out);
     if (axis == AX_ROW)
         return in_fp32 ? launch_row<float>(p, fast, st, grid_out)
                        : launch_row<__nv_bfloat16>(p, fast, st, grid_out);
@@ -405,7 +379,6 @@ int launch_quantize(const QParams &p, int axis, int in_fp32, int fast, cudaStrea
 
 int launch_tensor_amax(const QParams &p, int axis, int in_fp32, cudaStream_t st)
 {
-    if (cudaMemsetAsync(p.amax_word, 0, sizeof(unsigned int), st) != cudaSuccess) return -1;
     if (axis == AX_COL && p.had) {
         if (launch_amax_col(p, in_fp32, st)) return -1;
     } else {
@@ -418,12 +391,6 @@ int launch_tensor_amax(const QParams &p, int axis, int in_fp32, cudaStream_t st)
             k_amax_row<__nv_bfloat16><<<g, kThreads, 0, st>>>(p);
         }
     }
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
-}
-
-int launch_finalize_tensor_scale(const QParams &p, cudaStream_t st)
-{
-    k_finalize_tensor_scale<<<1, 1, 0, st>>>(p.amax_word, p.ed.maxv, p.sd.ue_maxv, p.tensor_scale);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

@@ -136,6 +136,40 @@ def test_ue_scales(mx, orc, fmt, rule, ts, block, sigma):
     run_case(mx, orc, x, mx.Config(block=block, scale_fmt=fmt, rule=rule, tensor_scale=ts))
 
 
+def _ue_values(fmt):
+    """Finite values of the unsigned scale format, ascending (codes 0..max)."""
+    bias, top = (7, 0x7E) if fmt == 1 else (15, 0xFE)
+    c = np.arange(top + 1)
+    e, m = c >> 3, c & 7
+    return np.where(e == 0, m * 2.0 ** (1 - bias - 3), (1 + m / 8.0) * 2.0 ** (e - bias))
+
+
+@pytest.mark.parametrize("fmt", [1, 2])
+@pytest.mark.parametrize("ts", [None, 1.0, 0.3712, 1.7e-3, 2.5e4])
+def test_nearest_scale_rounding_boundaries(mx, orc, fmt, ts):
+    """Nearest block scales s_b = RTNE((alpha / 6) / s_T) with the block amax
+    placed within a few ulps of every rounding boundary of the scale format
+    (the midpoints between consecutive codes): the two binary32 quotients must
+    be correctly rounded for the codes to match."""
+    v = _ue_values(fmt)
+    mids = (v[:-1] + v[1:]) / 2.0
+    sT = 1.0 if ts is None else float(np.float32(ts))
+    k = np.arange(-6, 7)
+    target = (mids[:, None] * (1.0 + k[None, :] * 2.0 ** -23)).ravel()
+    alpha = (target * 6.0 * sT).astype(np.float32)
+    j = np.arange(-2, 3, dtype=np.int64)
+    alpha = (alpha.view(np.int32)[:, None].astype(np.int64) + j[None, :]).astype(np.int32).view(np.float32).ravel()
+    alpha = alpha[np.isfinite(alpha) & (alpha > 0) & (alpha < 3.0e38)]
+    nb = (len(alpha) + 15) // 16 * 16
+    alpha = np.resize(alpha, nb)
+    rng = np.random.default_rng(3)
+    blk = (rng.uniform(-1, 1, (nb, 16)) * alpha[:, None] * 0.9).astype(np.float32)
+    blk[:, 0] = alpha
+    x = torch.from_numpy(blk.reshape(-1, 256))
+    cfg = mx.Config(block=16, scale_fmt=fmt, rule=3, tensor_scale=0 if ts is None else 2)
+    run_case(mx, orc, x, cfg, given_ts=None if ts is None else sT)
+
+
 def test_given_tensor_scale(mx, orc):
     x = inputs.normal(64, 256, sigma=0.02, seed=2)
     run_case(mx, orc, x, mx.Config(block=16, scale_fmt=1, rule=3, tensor_scale=2), given_ts=1.5e-5)
@@ -158,6 +192,47 @@ def test_given_tensor_scale(mx, orc):
 def test_elements_and_rounding(mx, orc, elem, rule, asym, rnd, dtype):
     x = inputs.gradient_like(64, 512, seed=5, dtype=dtype)
     run_case(mx, orc, x, mx.Config(elem=elem, rule=rule, asymmetric=asym, round=rnd, seed=12345))
+
+
+@pytest.mark.parametrize("elem", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("rnd", [0, 1, 2])
+@pytest.mark.parametrize("asym", [0, 1])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_general_quantizer_matrix(mx, orc, elem, rnd, asym, dtype):
+    """Every element type x rounding mode x offset on a ragged row count
+    (72 x 544 = 1224 chunks of 32: four full tiles of 256 and a partial one),
+    with zero, NaN and Inf blocks and signed zeros planted."""
+    x = inputs.gradient_like(72, 544, seed=5, dtype=torch.float32)
+    x[3, 32:64] = 0.0
+    x[5, 64:96] = -0.0
+    x[7, 100] = float("nan")
+    x[9, 200] = float("inf")
+    x[11, 0:32] = torch.linspace(-1e-3, 1e-3, 32)
+    x = x.to(dtype)
+    cfg = mx.Config(elem=elem, round=rnd, asymmetric=asym, rule=1 if (elem == 4 and asym) else 0,
+                    seed=0x1234_5678_9ABC)
+    run_case(mx, orc, x, cfg)
+
+
+@pytest.mark.parametrize("elem", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("rnd", [0, 1, 2])
+def test_general_grid_sweep(mx, orc, elem, rnd):
+    """Scaled values swept densely across each grid (multiples of 2^-7, so every
+    grid point and every midpoint is hit exactly) with the block scale pinned to
+    one: element 0 of each block is 2^emax and the others stay below
+    2^(emax+1)."""
+    emax = {0: 2, 1: 4, 2: 2, 3: 4, 4: 2}[elem]
+    maxv = {0: 6.0, 1: 16.0, 2: 7.5, 3: 28.0, 4: 7.0}[elem]
+    lim = min(maxv * 1.06, 2.0 ** (emax + 1) - 2.0 ** -7)
+    v = np.arange(-lim, lim, 2.0 ** -7, dtype=np.float64).astype(np.float32)
+    n = (len(v) + 30) // 31 * 31
+    v = np.resize(v, n).reshape(-1, 31)
+    rows = (v.shape[0] + 7) // 8 * 8
+    blk = np.zeros((rows, 32), np.float32)
+    blk[:, 0] = 2.0 ** emax
+    blk[:v.shape[0], 1:] = v
+    x = torch.from_numpy(blk.reshape(-1, 256))
+    run_case(mx, orc, x, mx.Config(elem=elem, round=rnd, seed=99))
 
 
 @pytest.mark.parametrize("axis,block", [(1, 8), (1, 16), (1, 32), (2, 32)])
@@ -229,6 +304,22 @@ def test_zeros_and_empty(mx, orc):
     q = mx.quantize(e, mx.MXFP4)
     st = q.stats.cpu().numpy()
     assert st[10] == 0 and math.isnan(st[7])
+
+
+def test_workspace_control_words_left_zero(mx):
+    """The quantizer's last CTA sums the statistics and clears the workspace's
+    control words (tensor-amax accumulator, launch ticket): after calls with a
+    computed tensor scale and statistics the first 256 bytes are zero again,
+    and repeated calls give identical statistics."""
+    x = inputs.normal(512, 1024, sigma=0.02, seed=2).cuda()
+    runs = []
+    for cfg in (mx.NVFP4, mx.MXFP4, mx.NVFP4, mx.Config(elem=mx.E2M3), mx.Config(axis=1)):
+        q = mx.quantize(x, cfg, stats=True)
+        torch.cuda.synchronize()
+        ws = mx._default_ws[str(x.device)].buf
+        assert int(ws[:256].count_nonzero()) == 0
+        runs.append(q.stats.cpu().numpy().copy())
+    assert np.array_equal(runs[0], runs[2])
 
 
 def test_fast_path_conversion_rounding(mx):
