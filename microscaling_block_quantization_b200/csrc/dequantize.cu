@@ -191,6 +191,135 @@ __global__ void __launch_bounds__(kThreads) k_dequant_chunk(const DParams p)
     }
 }
 
+// ---------------------------------------------------- E2M1, 8 per lane --
+// Exact unsigned division by a runtime divisor d >= 2 through a multiply-high
+// (Granlund and Montgomery, PLDI 1994, Fig. 4.1): t = umulhi(n, m),
+// q = (t + ((n - t) >> s1)) >> s2 for every 32-bit n.
+struct FastDiv {
+    uint32_t m;
+    int s1, s2;
+};
+
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv &f)
+{
+    const uint32_t t = __umulhi(n, f.m);
+    return (t + ((n - t) >> f.s1)) >> f.s2;
+}
+
+// E8M0 / unsigned-minifloat block-scale value without branches on the code
+__device__ __forceinline__ float scale_value_fast(const ScaleDesc &sd, uint32_t code)
+{
+    if (sd.fmt == S_E8M0)
+        return __uint_as_float(code == 0xffu ? 0x7fc00000u : code ? code << 23 : 0x00400000u);
+    return ue_value(sd, code);
+}
+
+// E2M1, symmetric, no macro scale or rotation, every axis and scale layout.
+// Thread = 8 consecutive elements of a row (an octet: one 32-bit code word
+// in, 16 bytes of bf16 or 32 of fp32 out), so consecutive lanes read and
+// write consecutive addresses; four octets in flight per thread.
+template <int AXIS, bool OUT32>
+__global__ void __launch_bounds__(kThreads) k_dequant_oct(const DParams p, const FastDiv opr_div, uint32_t noct)
+{
+    constexpr int U = 4;
+    const uint32_t T = gridDim.x * blockDim.x;
+    const float sT = (p.ts_mode != TS_NONE && p.tensor_scale) ? *p.tensor_scale : 1.0f;
+    const bool nearest = p.sd.fmt != S_E8M0 && p.sd.rule == R_NEAREST;
+    const int lb = __ffs(p.block) - 1;
+    const uint32_t cols = (uint32_t)p.cols, opr = cols >> 3;
+    const uint32_t S = cols >> lb;
+    const uint32_t *codes = static_cast<const uint32_t *>(p.codes);
+    for (uint32_t o0 = blockIdx.x * blockDim.x + threadIdx.x; o0 < noct; o0 += U * T) {
+        uint32_t w[U], sc[U][AXIS == AX_COL ? 2 : 1];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t o = o0 + u * T;
+            w[u] = 0;
+            sc[u][0] = 0;
+            if (AXIS == AX_COL) sc[u][AXIS == AX_COL ? 1 : 0] = 0;
+            if (o < noct) {
+                w[u] = __ldg(codes + o);
+                if (AXIS == AX_ROW && !p.sf_gemm) {
+                    sc[u][0] = __ldg(p.scales + (o >> (lb - 3)));
+                } else {
+                    const uint32_t row = fast_div(o, opr_div), col = (o - row * opr) << 3;
+                    if (AXIS == AX_ROW) {
+                        sc[u][0] = __ldg(p.scales + sf_chunk_index(row, col >> lb, S));
+                    } else if (AXIS == AX_2D) {
+                        sc[u][0] = __ldg(p.scales + (size_t)(row >> 5) * (cols >> 5) + (col >> 5));
+                    } else {
+                        const uint2 b = __ldg(reinterpret_cast<const uint2 *>(p.scales + (size_t)(row >> lb) * cols + col));
+                        sc[u][0] = b.x;
+                        sc[u][AXIS == AX_COL ? 1 : 0] = b.y;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t o = o0 + u * T;
+            if (o >= noct) break;
+            float q[8];
+            e2m1x8_values(w[u], q);
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+                float s0, s1;
+                if (AXIS == AX_COL) {
+                    const uint32_t word = sc[u][i >> 2];
+                    s0 = scale_value_fast(p.sd, (word >> (8 * (i & 3))) & 0xffu);
+                    s1 = scale_value_fast(p.sd, (word >> (8 * ((i + 1) & 3))) & 0xffu);
+                } else {
+                    s0 = s1 = scale_value_fast(p.sd, sc[u][0]);
+                }
+                float2 t = __fmul2_rn(make_float2(q[i], q[i + 1]), make_float2(s0, s1));
+                if (nearest) t = __fmul2_rn(t, make_float2(sT, sT));
+                v[i] = t.x;
+                v[i + 1] = t.y;
+            }
+            if (OUT32) {
+                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (size_t)o * 8);
+                dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+                dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+            } else {
+                uint32_t t[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+                    t[k] = *reinterpret_cast<uint32_t *>(&h);
+                }
+                reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out))[o] = make_uint4(t[0], t[1], t[2], t[3]);
+            }
+        }
+    }
+}
+
+FastDiv make_fast_div(uint32_t d)
+{
+    int l = 0;
+    while ((1ull << l) < d) ++l;
+    FastDiv f;
+    f.m = (uint32_t)((((1ull << l) - d) << 32) / d + 1);
+    f.s1 = l < 1 ? l : 1;
+    f.s2 = l > 1 ? l - 1 : 0;
+    return f;
+}
+
+template <int AXIS>
+int launch_dequant_oct(const DParams &p, cudaStream_t st)
+{
+    const uint64_t noct = (uint64_t)(p.rows * p.cols / 8);
+    const FastDiv f = make_fast_div((uint32_t)(p.cols / 8));
+    if (p.out_fp32) {
+        const int g = grid_of(k_dequant_oct<AXIS, true>, (int64_t)(noct / 4 + 255) / 256 * 8);
+        k_dequant_oct<AXIS, true><<<g, kThreads, 0, st>>>(p, f, (uint32_t)noct);
+    } else {
+        const int g = grid_of(k_dequant_oct<AXIS, false>, (int64_t)(noct / 4 + 255) / 256 * 8);
+        k_dequant_oct<AXIS, false><<<g, kThreads, 0, st>>>(p, f, (uint32_t)noct);
+    }
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
 // Column axis with the rotation along columns: thread = 4 columns x `block`
 // rows, rotated back in registers.
 __global__ void __launch_bounds__(kThreads) k_dequant_colhad(const DParams p)
@@ -432,6 +561,10 @@ int launch_dequantize(const DParams &p, cudaStream_t st)
         const int64_t items = (p.rows / p.block) * ((p.cols / 4 + 31) / 32);
         const int g = grid_of(k_dequant_colhad, items);
         k_dequant_colhad<<<g, kThreads, 0, st>>>(p);
+    } else if (p.ed.elem == E2M1 && !p.asym && !p.mbs && !p.had && p.rows * p.cols / 8 < (INT64_C(1) << 32)) {
+        if (p.axis == AX_ROW) return launch_dequant_oct<AX_ROW>(p, st);
+        if (p.axis == AX_COL) return launch_dequant_oct<AX_COL>(p, st);
+        return launch_dequant_oct<AX_2D>(p, st);
     } else {
         const int64_t warps = (p.rows * p.cols / 32 + 31) / 32;
         const bool fast = p.ed.elem == E2M1 && !p.asym && !p.mbs && p.axis != AX_COL;

@@ -37,6 +37,49 @@ __device__ __forceinline__ float fmin3(float a, float b, float c)
     return r;
 }
 
+// number of zero-magnitude E2M1 codes among the 8 nibbles of w: a nibble's
+// magnitude m (0..7) plus 7 sets bit 3 exactly when m != 0, with no carry out
+__device__ __forceinline__ int e2m1_zero_codes8(uint32_t w)
+{
+    return 8 - __popc(((w & 0x77777777u) + 0x77777777u) & 0x88888888u);
+}
+
+// max |v| (NaN-propagating) and min |v| of L = 8, 16 or 32 values: L / 8
+// independent chains of three-operand ops, then a short combine (the chains
+// overlap in the pipeline instead of one dependent chain of L / 2 ops)
+template <int L>
+__device__ __forceinline__ float absmax_nan(const float *v)
+{
+    float c[L / 8];
+#pragma unroll
+    for (int i = 0; i < L / 8; ++i) {
+        const float *w = v + 8 * i;
+        float a = fmax3_nan(fabsf(w[0]), fabsf(w[1]), fabsf(w[2]));
+        a = fmax3_nan(a, fabsf(w[3]), fabsf(w[4]));
+        a = fmax3_nan(a, fabsf(w[5]), fabsf(w[6]));
+        c[i] = fmax_nan(a, fabsf(w[7]));
+    }
+    if constexpr (L == 8) return c[0];
+    else if constexpr (L == 16) return fmax_nan(c[0], c[L == 16 ? 1 : 0]);
+    else return fmax_nan(fmax3_nan(c[0], c[L / 8 > 1 ? 1 : 0], c[L / 8 > 2 ? 2 : 0]), c[L / 8 > 3 ? 3 : 0]);
+}
+template <int L>
+__device__ __forceinline__ float absmin(const float *v)
+{
+    float c[L / 8];
+#pragma unroll
+    for (int i = 0; i < L / 8; ++i) {
+        const float *w = v + 8 * i;
+        float a = fmin3(fabsf(w[0]), fabsf(w[1]), fabsf(w[2]));
+        a = fmin3(a, fabsf(w[3]), fabsf(w[4]));
+        a = fmin3(a, fabsf(w[5]), fabsf(w[6]));
+        c[i] = fminf(a, fabsf(w[7]));
+    }
+    if constexpr (L == 8) return c[0];
+    else if constexpr (L == 16) return fminf(c[0], c[L == 16 ? 1 : 0]);
+    else return fminf(fmin3(c[0], c[L / 8 > 1 ? 1 : 0], c[L / 8 > 2 ? 2 : 0]), c[L / 8 > 3 ? 3 : 0]);
+}
+
 // ------------------------------------------------------------------ loads --
 __device__ __forceinline__ void unpack_bf16x2(uint32_t w, float &lo, float &hi)
 {

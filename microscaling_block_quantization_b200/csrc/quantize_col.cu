@@ -241,14 +241,45 @@ __global__ void __launch_bounds__(kColThreads) k_quant_col(const QParams p)
                     float a[NSF], mabs[NSF];
 #pragma unroll
                     for (int s2 = 0; s2 < NSF; ++s2) { a[s2] = 0.0f; mabs[s2] = FLT_MAX; }
-                    for (int r = 0; r < RB; ++r) {
-                        float v[CPT];
-                        t.get(r, v);
+                    if constexpr (CPT == 8) {
+                        // bf16 pairs straight from the tile: |x| by masking the
+                        // sign bits, NaN-propagating max and min per column pair
+                        __nv_bfloat162 am[4], mn[4];
 #pragma unroll
-                        for (int j = 0; j < CPT; ++j) {
-                            const int s2 = (AXIS == AX_COL) ? j : 0;
-                            a[s2] = fmax_nan(a[s2], fabsf(v[j]));
-                            mabs[s2] = fminf(mabs[s2], fabsf(v[j]));
+                        for (int i = 0; i < 4; ++i) {
+                            am[i] = __float2bfloat162_rn(0.0f);
+                            mn[i] = __float2bfloat162_rn(__uint_as_float(0x7f800000u));
+                        }
+                        for (int r = 0; r < RB; ++r) {
+                            const uint4 u = t.base[r * 32];
+                            const uint32_t wv[4] = {u.x & 0x7fff7fffu, u.y & 0x7fff7fffu, u.z & 0x7fff7fffu,
+                                                    u.w & 0x7fff7fffu};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&wv[i]);
+                                am[i] = __hmax2_nan(am[i], b);
+                                mn[i] = __hmin2(mn[i], b);
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float2 fa = __bfloat1622float2(am[i]), fm = __bfloat1622float2(mn[i]);
+                            const int s0 = (AXIS == AX_COL) ? 2 * i : 0, s1 = (AXIS == AX_COL) ? 2 * i + 1 : 0;
+                            a[s0] = fmax_nan(a[s0], fa.x);
+                            a[s1] = fmax_nan(a[s1], fa.y);
+                            mabs[s0] = fminf(mabs[s0], fm.x);
+                            mabs[s1] = fminf(mabs[s1], fm.y);
+                        }
+                    } else {
+                        for (int r = 0; r < RB; ++r) {
+                            float v[CPT];
+                            t.get(r, v);
+#pragma unroll
+                            for (int j = 0; j < CPT; ++j) {
+                                const int s2 = (AXIS == AX_COL) ? j : 0;
+                                a[s2] = fmax_nan(a[s2], fabsf(v[j]));
+                                mabs[s2] = fminf(mabs[s2], fabsf(v[j]));
+                            }
                         }
                     }
                     BlockScale bsf[NSF];
@@ -285,9 +316,7 @@ __global__ void __launch_bounds__(kColThreads) k_quant_col(const QParams p)
                         deqT[s2] = bsf[s2].nan ? __uint_as_float(0x7fc00000u)
                                  : nearest ? __fmul_rn(bsf[s2].deq, sT) : bsf[s2].deq;
                     float2 sx2 = make_float2(0.f, 0.f), se2 = sx2, sb2 = sx2;
-                    int qzc[NSF];
-#pragma unroll
-                    for (int s2 = 0; s2 < NSF; ++s2) qzc[s2] = 0;
+                    int qz = 0;                      // zero-magnitude codes of the lane
                     for (int r = 0; r < RB; ++r) {
                         const int64_t e0 = (r0 + r) * p.cols + c0;
                         float v[CPT];
@@ -321,17 +350,16 @@ __global__ void __launch_bounds__(kColThreads) k_quant_col(const QParams p)
                                 sx2 = __ffma2_rn(yv, yv, sx2);
                                 sb2 = __fadd2_rn(sb2, d);
                             }
-#pragma unroll
-                            for (int j = 0; j < CPT; ++j) {
-                                const int s2 = (AXIS == AX_COL) ? j : 0;
-                                qzc[s2] += ((lo >> (4 * j)) & 7u) == 0u;
-                            }
+                            qz += e2m1_zero_codes8(lo) - (8 - CPT);
                         }
                     }
                     if (stats && ok) {
                         acc.x2 += (double)(sx2.x + sx2.y);
                         acc.e2 += (double)(se2.x + se2.y);
                         acc.e += -(double)(sb2.x + sb2.y);
+                        // flushed = zero codes - exact zeros, NaN blocks (all codes
+                        // zero) left out
+                        int ftz = qz;
 #pragma unroll
                         for (int s2 = 0; s2 < NSF; ++s2) {
                             int xz = 0;
@@ -345,8 +373,9 @@ __global__ void __launch_bounds__(kColThreads) k_quant_col(const QParams p)
                                 }
                             const int n_lane = (AXIS == AX_COL) ? RB : RB * CPT;
                             acc.nz += (double)(n_lane - xz);
-                            if (!bsf[s2].nan) acc.ftz += (double)(qzc[s2] - xz);
+                            ftz -= bsf[s2].nan ? n_lane : xz;
                         }
+                        acc.ftz += (double)ftz;
                     }
                     continue;
                 }

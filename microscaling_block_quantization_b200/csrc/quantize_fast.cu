@@ -72,7 +72,7 @@ __device__ __forceinline__ void hadamard_groups(float y[32])
 // quantization; MBS: 1 x 128 macro scale over the
 // 4 lanes of a macro block (consecutive chunks of a tile are consecutive lanes).
 template <typename InT, int B, bool STATS, int HADN, bool MBS, bool NEAR>
-__global__ void __launch_bounds__(kFastThreads, (HADN || MBS) ? 2 : 3) k_quant_fast(const QParams p, const __grid_constant__ CUtensorMap tm)
+__global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) k_quant_fast(const QParams p, const __grid_constant__ CUtensorMap tm)
 {
     constexpr int NB = B <= 32 ? 32 / B : 1;
     constexpr int G = B <= 32 ? 1 : B / 32;
@@ -143,17 +143,13 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS) ? 2 : 3) k_quant_f
             uint32_t scode[NB];
             // packed two-lane binary32 arithmetic (each lane rounded as a scalar op)
             float2 sx2 = make_float2(0.f, 0.f), se2 = sx2, sb2 = sx2;
+            float2 sx2v[2] = {sx2, sx2};            // sum of y^2, power-of-two scale path
             int nzc = 0, ftzc = 0;
 #pragma unroll
             for (int k = 0; k < NB; ++k) {
                 const int j0 = k * L;
-                float a = 0.0f, mabs = FLT_MAX;
-#pragma unroll
-                for (int j = j0; j < j0 + L; j += 2) {
-                    a = fmax3_nan(a, fabsf(y[j]), fabsf(y[j + 1]));
-                    if (STATS) mabs = fmin3(mabs, fabsf(MBS ? ys[MBS ? j : 0] : y[j]),
-                                            fabsf(MBS ? ys[MBS ? j + 1 : 0] : y[j + 1]));
-                }
+                float a = absmax_nan<L>(y + j0), mabs = 1.0f;
+                if (STATS) mabs = absmin<L>((MBS ? ys : y) + (MBS ? j0 : j0));
                 int bad = !(a <= FLT_MAX);
                 if (G > 1) {
                     a = grp_max(bad ? 0.0f : a, G);
@@ -169,7 +165,7 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS) ? 2 : 3) k_quant_f
                 const float2 nq2 = make_float2(-deqT, -deqT);
                 // power-of-two scale: y = X s exactly, so y - x_hat = X (s - q)
                 // and the block's sums are taken on the scaled values
-                float2 re2 = make_float2(0.f, 0.f), rb2 = re2;
+                float2 re2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)}, rb2[2] = {re2[0], re2[0]};
                 int qz = 0;
 #pragma unroll
                 for (int w = 0; w < L / 8; ++w) {
@@ -190,10 +186,11 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS) ? 2 : 3) k_quant_f
 #pragma unroll
                             for (int e = 0; e < 8; e += 2) {
                                 const float2 d = sub_f16x2_from(s8[e], s8[e + 1], h[e >> 1]);   // s - q
-                                re2 = __ffma2_rn(d, d, re2);
-                                rb2 = __fadd2_rn(rb2, d);
+                                const int u = (e >> 1) & 1;          // two accumulator chains
+                                re2[u] = __ffma2_rn(d, d, re2[u]);
+                                rb2[u] = __fadd2_rn(rb2[u], d);
                                 const float2 yv = make_float2(y[jb + e], y[jb + e + 1]);
-                                sx2 = __ffma2_rn(yv, yv, sx2);
+                                sx2v[u] = __ffma2_rn(yv, yv, sx2v[u]);
                             }
                         } else {
                             float q[8];
@@ -214,8 +211,8 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS) ? 2 : 3) k_quant_f
                 if (STATS) {
                     if (exact && ok) {
                         const double X = bs.nan ? (double)__uint_as_float(0x7fc00000u) : (double)bs.deq;
-                        acc.e2 += (double)(re2.x + re2.y) * X * X;
-                        acc.e -= (double)(rb2.x + rb2.y) * X;
+                        acc.e2 += (double)((re2[0].x + re2[1].x) + (re2[0].y + re2[1].y)) * X * X;
+                        acc.e -= (double)((rb2[0].x + rb2[1].x) + (rb2[0].y + rb2[1].y)) * X;
                     }
                     int xz = 0;
                     if (mabs == 0.0f)                      // rare: count exact zeros
@@ -225,6 +222,7 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS) ? 2 : 3) k_quant_f
                     if (!bs.nan) ftzc += qz - xz;
                 }
             }
+            sx2 = __fadd2_rn(sx2, __fadd2_rn(sx2v[0], sx2v[1]));
             const float sx = sx2.x + sx2.y, se = se2.x + se2.y, sb = -(sb2.x + sb2.y);
             if (ok) {
                 reinterpret_cast<uint4 *>(p.codes)[c] = make_uint4(words[0], words[1], words[2], words[3]);
