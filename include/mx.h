@@ -244,10 +244,11 @@ int mx_qsnr(const void *x, int32_t x_dtype, const void *x_hat, int32_t x_hat_dty
  * C[M x N] = A^Q (B^Q)^T with FP32 accumulation ([BRIDGING] sec. 2.3;
  * [MXFP4-OAS] Fig. 5).  A^Q: M x K E2M1 codes, B^Q: N x K E2M1 codes, both
  * row-major along K as written by mx_quantize (row axis).  Scales in the
- * canonical row-axis layout.  MXFP4: block 32, E8M0 (ca/cb rule FLOOR, CEIL
- * or OAS).  NVFP4: block 16, UE4M3 NEAREST with tensor scales tsA/tsB (device
- * floats; NULL = 1).  C: device, bf16 or fp32 (c_dtype), row-major M x N.
- * M % 128 == 0, N % 128 == 0, K % 256 == 0.
+ * tcgen05 chunk layout (ca/cb->sf_layout = 1, as mx_quantize wrote them).
+ * MXFP4: block 32, E8M0 (ca/cb rule FLOOR, CEIL or OAS).  NVFP4: block 16,
+ * UE4M3 NEAREST with tensor scales tsA/tsB (device floats; used when
+ * ca/cb->tensor_scale != MX_TS_NONE, else 1).  C: device, bf16 or fp32
+ * (c_dtype), row-major M x N.  M % 128 == 0, N % 128 == 0, K % 256 == 0.
  */
 int mx_gemm(const mx_config *ca, const mx_config *cb, const void *Aq, const uint8_t *Asf,
             const void *Bq, const uint8_t *Bsf, const float *tsA, const float *tsB, int64_t M,
@@ -266,6 +267,33 @@ int mx_gemm_qsnr(const mx_config *ca, const mx_config *cb, const void *A, const 
                  int64_t N, int64_t K, const void *Aq, const uint8_t *Asf, const void *Bq,
                  const uint8_t *Bsf, const float *tsA, const float *tsB, double *stats,
                  void *workspace, int64_t workspace_bytes, void *stream);
+
+/*
+ * mx_mbs_gemm_scales -- an MBS operand ([MXFP4-OAS] Sec.4 Macro Block
+ * Scaling: E2M1 codes, E8M0 scale X per 1 x 32 block, E4M3 macro scale S_M per
+ * 1 x 128, x_hat = q X S_M) as an operand of mx_gemm's NVFP4 kind.  The pages
+ * give MBS's GEMM (Fig. 5) but no data path for it; this is one: S_M X is an
+ * E4M3 significand times a power of two, so with a per-tensor power of two
+ * s_T = 2^t it is exactly a UE4M3 value when it falls in UE4M3's normal range.
+ *   cfg          the MBS configuration the operand was quantized with (E2M1,
+ *                E8M0, block 32, macro_block 128, row axis, canonical scales).
+ *   scales       device, rows x cols/32 E8M0 codes (canonical).
+ *   macro_scales device, rows x cols/128 E4M3 codes.
+ *   sf16         device out, rows x cols/16 UE4M3 codes in the tcgen05 chunk
+ *                layout: code(S_M X / s_T) for both 16-element halves of every
+ *                32-block (round to nearest even; NaN scale -> 0x7F; zero
+ *                block -> 0).
+ *   tensor_scale device out, one float: s_T, with t chosen so that the largest
+ *                folded value is below 2^8; values more than 13 binades below
+ *                it are rounded into UE4M3's subnormals (inexact).
+ *   workspace    control words as for mx_quantize (the first 256 bytes).
+ * Then mx_gemm / mx_gemm_qsnr with an NVFP4 configuration (block 16, UE4M3,
+ * NEAREST, sf_layout 1, tensor_scale MX_TS_GIVEN) on the same codes, sf16
+ * and tensor_scale.  rows % 128 == 0, cols % 128 == 0.  Two launches.
+ */
+int mx_mbs_gemm_scales(const mx_config *cfg, const uint8_t *scales, const uint8_t *macro_scales,
+                       int64_t rows, int64_t cols, uint8_t *sf16, float *tensor_scale,
+                       void *workspace, int64_t workspace_bytes, void *stream);
 
 /* Status words of the bounded in-kernel waits: reads and clears them
  * (synchronises `stream`).  *status = 0 when no wait gave up, else the code of

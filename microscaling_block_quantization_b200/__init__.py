@@ -111,12 +111,13 @@ def lib() -> C.CDLL:
         L.mx_gemm_workspace_bytes.restype = i64
         L.mx_gemm.argtypes = [cfgp, cfgp, P, P, P, P, P, P, i64, i64, i64, P, i32, P]
         L.mx_gemm_qsnr.argtypes = [cfgp, cfgp, P, P, i64, i64, i64, P, P, P, P, P, P, P, P, i64, P]
+        L.mx_mbs_gemm_scales.argtypes = [cfgp, P, P, i64, i64, P, P, P, i64, P]
         L.mx_device_status.argtypes = [P, C.POINTER(i32)]
         L.mx_strerror.argtypes = [C.c_int]
         L.mx_strerror.restype = C.c_char_p
         L.mx_version.restype = C.c_char_p
         for f in ("mx_query_sizes", "mx_quantize", "mx_quantize_noalloc", "mx_hadamard_quantize", "mx_dequantize",
-                  "mx_qsnr", "mx_gemm", "mx_gemm_qsnr", "mx_device_status"):
+                  "mx_qsnr", "mx_gemm", "mx_gemm_qsnr", "mx_mbs_gemm_scales", "mx_device_status"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -219,6 +220,13 @@ def mx_gemm_qsnr(ca: Config, cb: Config, A, B, M, N, K, Aq, Asf, Bq, Bsf, tsA, t
     a, b = ca.c(), cb.c()
     return lib().mx_gemm_qsnr(C.byref(a), C.byref(b), A, B, M, N, K, Aq, Asf, Bq, Bsf, tsA, tsB,
                               stats, workspace, workspace_bytes, stream)
+
+
+def mx_mbs_gemm_scales(cfg: Config, scales, macro, rows, cols, sf16, tensor_scale, workspace,
+                       workspace_bytes, stream) -> int:
+    c = cfg.c()
+    return lib().mx_mbs_gemm_scales(C.byref(c), scales, macro, rows, cols, sf16, tensor_scale, workspace,
+                                    workspace_bytes, stream)
 
 
 def mx_device_status(stream=None) -> int:
@@ -355,6 +363,24 @@ def gemm(qa: Quantized, qb: Quantized, out_dtype: torch.dtype = torch.bfloat16,
                  _stream(stream))
     _check("mx_gemm", rc)
     return out
+
+
+def mbs_gemm_operand(q: Quantized, stream=None) -> Quantized:
+    """An MBS-quantized tensor (block 32, E8M0, macro_block 128, canonical
+    scales) as an operand of the NVFP4 GEMM kind (``mx_mbs_gemm_scales``):
+    same codes, UE4M3 16-element scales S_M X / s_T in the tcgen05 chunk
+    layout and the power-of-two tensor scale s_T."""
+    if not q.cfg.macro_block or q.macro is None:
+        raise ValueError("not an MBS-quantized tensor")
+    dev = q.codes.device
+    sf16 = torch.empty(max(q.rows * q.cols // 16, 16), dtype=torch.uint8, device=dev)
+    ts = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = _ws(256, dev)
+    rc = mx_mbs_gemm_scales(q.cfg, _p(q.scales), _p(q.macro), q.rows, q.cols, _p(sf16), _p(ts), _p(ws),
+                            ws.numel(), _stream(stream))
+    _check("mx_mbs_gemm_scales", rc)
+    cfg = Config(block=16, scale_fmt=SCALE_UE4M3, rule=RULE_NEAREST, tensor_scale=TS_GIVEN, sf_layout=1)
+    return Quantized(cfg, q.rows, q.cols, q.codes, sf16[: q.rows * q.cols // 16], ts, None, None, None)
 
 
 def gemm_qsnr(A: torch.Tensor, B: torch.Tensor, qa: Quantized, qb: Quantized,

@@ -285,6 +285,48 @@ __global__ void __launch_bounds__(kThreads) k_amax_row(const QParams p)
     if (lane == 0 && m > 0.0f) atomicMax(p.amax_word, __float_as_uint(m));
 }
 
+// Tensor absmax without rotation (any block axis): consecutive lanes read
+// consecutive 16-byte vectors, four in flight per thread, NaN skipped.  The
+// tensor is walked from its end towards its start, so that the quantizer's
+// forward walk that follows first meets the lines this pass touched last
+// (still in L2 when the tensor is not much larger than L2).
+template <typename InT>
+__global__ void __launch_bounds__(kThreads) k_amax_vec(const QParams p)
+{
+    constexpr int U = 4;
+    const uint4 *x = static_cast<const uint4 *>(p.x);
+    const uint64_t nv = (uint64_t)(p.rows * p.cols) * sizeof(InT) / 16;
+    const uint64_t T = (uint64_t)gridDim.x * blockDim.x;
+    float m = 0.0f;
+    __nv_bfloat162 m2 = __float2bfloat162_rn(0.0f);
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv; i += U * T) {
+        uint4 u[U];
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            const uint64_t j = i + k * T;
+            u[k] = j < nv ? __ldg(x + (nv - 1 - j)) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int k = 0; k < U; ++k) {
+            if constexpr (sizeof(InT) == 2) {
+                const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e])));
+            } else {
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(__uint_as_float(u[k].x)), fabsf(__uint_as_float(u[k].y))),
+                                   fmaxf(fabsf(__uint_as_float(u[k].z)), fabsf(__uint_as_float(u[k].w)))));
+            }
+        }
+    }
+    if constexpr (sizeof(InT) == 2) {
+        const float2 f = __bfloat1622float2(m2);
+        m = fmaxf(f.x, f.y);
+    }
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+    if ((threadIdx.x & 31) == 0 && m > 0.0f) atomicMax(p.amax_word, __float_as_uint(m));
+}
+
 // Sum the per-CTA records in a fixed order and derive MSE, R-MSE, QSNR (Eq. (1)),
 // bias and the flush-to-zero share.
 __global__ void k_finalize_stats(const double *partials, int nparts, double count, double *stats)
@@ -381,6 +423,15 @@ int launch_tensor_amax(const QParams &p, int axis, int in_fp32, cudaStream_t st)
 {
     if (axis == AX_COL && p.had) {
         if (launch_amax_col(p, in_fp32, st)) return -1;
+    } else if (!p.had) {
+        const int64_t warps = (p.rows * p.cols / 8 / 4 + 31) / 32;
+        if (in_fp32) {
+            const int g = grid_for(k_amax_vec<float>, warps);
+            k_amax_vec<float><<<g, kThreads, 0, st>>>(p);
+        } else {
+            const int g = grid_for(k_amax_vec<__nv_bfloat16>, warps);
+            k_amax_vec<__nv_bfloat16><<<g, kThreads, 0, st>>>(p);
+        }
     } else {
         const int64_t tiles = (p.rows * p.cols / 32 + 31) / 32;
         if (in_fp32) {

@@ -152,3 +152,61 @@ def test_gemm_llama_shape_sampled_rows(mx, orc, name):
     rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     assert rel < 1e-3, rel
     assert np.max(np.abs(got - ref)) <= 1e-3 * np.sqrt(np.mean(ref ** 2))
+
+
+def mbs_cfgs(mx, orc):
+    return mx.Config(macro_block=128), orc.Cfg(macro_block=128)
+
+
+def mbs_expected_sf16(orc, r, rows, cols):
+    """The folded UE4M3 16-element scales and the tensor scale, from the
+    oracle's E8M0 block scales and E4M3 macro scales: S_M X / 2^t, t the
+    largest folded exponent minus 7."""
+    sc = r["scales"].reshape(rows, cols // 32).astype(np.int64)
+    mc = np.repeat(r["macro"].reshape(rows, cols // 128), 4, axis=1)
+    sm = np.array([orc.scale_decode(orc.UE4M3, int(c) & 0x7F) for c in range(128)], np.float64)[mc & 0x7F]
+    val = sm * np.exp2(sc - 127.0)
+    live = (sc != 0) & (sc != 255) & ((mc & 0x7F) != 0x7F)
+    emax = int(np.max(np.floor(np.log2(val[live]))))
+    t = emax - 7
+    folded = val / 2.0 ** t
+    codes = np.zeros_like(sc, dtype=np.uint8)
+    for idx in zip(*np.nonzero(live)):
+        codes[idx] = orc.scale_encode_nearest(orc.UE4M3, float(np.float32(folded[idx])))
+    codes[(sc == 255) | ((mc & 0x7F) == 0x7F)] = 0x7F
+    return np.repeat(codes, 2, axis=1), 2.0 ** t
+
+
+@pytest.mark.parametrize("shape", [(256, 256, 512), (384, 512, 1280)])
+def test_mbs_gemm_operands(mx, orc, shape):
+    """Macro Block Scaling operands through the NVFP4 GEMM kind: the folded
+    scales are S_M X / s_T bit for bit, and C equals the product of the MBS
+    dequantized operands (exact products, FP32 accumulation)."""
+    M, N, K = shape
+    a = inputs.laplace_outlier_cols(M, K, seed=6, n_outlier_cols=2)
+    w = inputs.normal(N, K, sigma=0.02, seed=7)
+    cfg, ocf = mbs_cfgs(mx, orc)
+    qa = mx.quantize(a.cuda(), cfg, stats=False)
+    qw = mx.quantize(w.cuda(), cfg, stats=False)
+    fa, fw = mx.mbs_gemm_operand(qa), mx.mbs_gemm_operand(qw)
+    c = mx.gemm(fa, fw, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert mx.mx_device_status() == 0
+    ra, rw = orc.quantize(ocf, a), orc.quantize(ocf, w)
+    for f, r, rows in ((fa, ra, M), (fw, rw, N)):
+        exp, ts = mbs_expected_sf16(orc, r, rows, K)
+        assert np.array_equal(f.scales.cpu().numpy(), chunk_layout(exp, rows, K // 16))
+        assert float(f.tensor_scale.item()) == ts
+    ah = orc.dequantize(ocf, ra["packed"], ra["scales"], ra["tensor_scale"], ra["macro"], None, M, K)
+    wh = orc.dequantize(ocf, rw["packed"], rw["scales"], rw["tensor_scale"], rw["macro"], None, N, K)
+    ref = ah.astype(np.float64) @ wh.astype(np.float64).T
+    got = c.cpu().numpy().astype(np.float64)
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < 1e-3
+    assert np.max(np.abs(got - ref)) <= 1e-3 * np.sqrt(np.mean(ref ** 2))
+
+
+def test_mbs_gemm_scales_rejects_other_configs(mx):
+    x = torch.zeros(128, 256, dtype=torch.bfloat16, device="cuda")
+    q = mx.quantize(x, mx.MXFP4, stats=False)
+    with pytest.raises(ValueError):
+        mx.mbs_gemm_operand(q)
