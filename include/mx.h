@@ -249,6 +249,7 @@ int mx_qsnr(const void *x, int32_t x_dtype, const void *x_hat, int32_t x_hat_dty
  * UE4M3 NEAREST with tensor scales tsA/tsB (device floats; used when
  * ca/cb->tensor_scale != MX_TS_NONE, else 1).  C: device, bf16 or fp32
  * (c_dtype), row-major M x N.  M % 128 == 0, N % 128 == 0, K % 256 == 0.
+ * Tiles: 128 x 256 per SM (persistent) when N % 256 == 0, else 128 x 128.
  */
 int mx_gemm(const mx_config *ca, const mx_config *cb, const void *Aq, const uint8_t *Asf,
             const void *Bq, const uint8_t *Bsf, const float *tsA, const float *tsB, int64_t M,
@@ -297,8 +298,9 @@ int mx_mbs_gemm_scales(const mx_config *cfg, const uint8_t *scales, const uint8_
 
 /* Status words of the bounded in-kernel waits: reads and clears them
  * (synchronises `stream`).  *status = 0 when no wait gave up, else the code of
- * the first wait that did: 1-3 and 11-14 the GEMM pipelines, 21-22 the E2M1
- * nearest-even quantizer's TMA ring, 31-32 the other element types' ring.  A
+ * the first wait that did: 1-3 and 11-14 the GEMM pipelines (128 x 128 and
+ * persistent 128 x 256 tiles), 21-22 the E2M1 nearest-even quantizer's TMA
+ * ring, 31-32 the other element types' ring.  A
  * kernel whose wait gave up has left its loop early, so its outputs are
  * incomplete; the library has no counterpart on the pages. */
 int mx_device_status(void *stream, int32_t *status);

@@ -372,27 +372,27 @@ __device__ __forceinline__ float div_by_recip(float a, float b, float y)
 struct NearScale {
     float maxv, r_max;      // largest element magnitude and RN(1 / maxv)
     float sT, r_T;          // tensor scale and RN(1 / sT); r_T = 0: IEEE division
-    const float *inv_tab;   // per scale code: RN(1 / RN(s_b sT)); +inf = zero block
+    const float2 *tab;      // per scale code: {RN(s_b sT), RN(1 / RN(s_b sT))}; NaN code: {NaN, 0}
 };
 
-// Same result as block_scale() with a nearest rule: the two quotients of
-// s_b = RTNE((alpha / max) / s_T) through div_by_recip, and the element
-// multiplier from the launch's table of reciprocals.
+// Same codes as block_scale() with a nearest rule: the two quotients of
+// s_b = RTNE((alpha / max) / s_T) through div_by_recip; the dequantization
+// factor s_b s_T (in deq) and the element multiplier from the launch's table.
+// A zero block: s_b = 0 (1/0 = +inf).
 __device__ __forceinline__ BlockScale near_block_scale(const ScaleDesc &s, const NearScale &ns, float alpha,
                                                        int nonfinite)
 {
     BlockScale r;
-    r.zero = 0; r.nan = 0; r.inv = 0.0f; r.deq = 0.0f;
-    if (nonfinite) { r.code = (uint32_t)s.ue_nan_code; r.zero = 1; r.nan = 1; return r; }
     const float q1 = div_by_recip(alpha, ns.maxv, ns.r_max);
     const float sb_real = ns.sT == 1.0f ? q1
                         : ns.r_T != 0.0f ? div_by_recip(q1, ns.sT, ns.r_T) : __fdiv_rn(q1, ns.sT);
-    r.code = (s.fmt == S_UE4M3) ? ue4m3_encode_hw(sb_real) : ue_encode_rtne(s, sb_real);
-    const float sb = ue_value(s, r.code);
-    r.deq = sb;
-    if (sb != sb) { r.zero = 1; r.nan = 1; return r; }
-    r.inv = ns.inv_tab[r.code];
-    r.zero = !(r.inv < __uint_as_float(0x7f800000u));
+    r.code = nonfinite ? (uint32_t)s.ue_nan_code
+                       : (s.fmt == S_UE4M3) ? ue4m3_encode_hw(sb_real) : ue_encode_rtne(s, sb_real);
+    const float2 t = ns.tab[r.code];
+    r.deq = t.x;
+    r.inv = t.y;
+    r.nan = r.code >= (uint32_t)s.ue_nan_code;
+    r.zero = r.nan || !(t.y < __uint_as_float(0x7f800000u));
     return r;
 }
 

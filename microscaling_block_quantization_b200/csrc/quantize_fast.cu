@@ -46,7 +46,7 @@ __device__ __forceinline__ void butterfly_stage2(float y[32])
         }
 }
 
-template <int N>
+template <int N, bool SCALE = true>
 __device__ __forceinline__ void hadamard_groups(float y[32])
 {
 #pragma unroll
@@ -59,6 +59,7 @@ __device__ __forceinline__ void hadamard_groups(float y[32])
     butterfly_stage2<4>(y);
     butterfly_stage2<8>(y);
     if constexpr (N == 32) butterfly_stage2<16>(y);
+    if constexpr (!SCALE) return;
     const float c = hadamard_scale(N);
     const float2 c2 = make_float2(c, c);
 #pragma unroll
@@ -84,18 +85,21 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) 
     const uint32_t ntiles = (nch + kConsumers - 1) / kConsumers;
     if (threadIdx.x == 0) ring.init();
     const float sT = launch_tensor_scale(p);
-    // nearest scales: the element multiplier of each scale code, once per CTA
-    __shared__ float inv_tab[NEAR ? 256 : 1];
+    // nearest scales: s_b s_T and its reciprocal for every scale code, once per CTA
+    __shared__ float2 near_tab[NEAR ? 256 : 1];
     if constexpr (NEAR)
-        for (int c = threadIdx.x; c < 256; c += blockDim.x)
-            inv_tab[c] = c < p.sd.ue_nan_code ? __fdiv_rn(1.0f, __fmul_rn(ue_value(p.sd, (uint32_t)c), sT)) : 0.0f;
+        for (int c = threadIdx.x; c < 256; c += blockDim.x) {
+            const float d = __fmul_rn(ue_value(p.sd, (uint32_t)c), sT);
+            near_tab[c] = c < p.sd.ue_nan_code ? make_float2(d, __fdiv_rn(1.0f, d))
+                                               : make_float2(__uint_as_float(0x7fc00000u), 0.0f);
+        }
     __syncthreads();
     NearScale ns;
     ns.maxv = p.ed.maxv;
     ns.r_max = __fdiv_rn(1.0f, p.ed.maxv);
     ns.sT = sT;
     ns.r_T = (sT >= 0x1p-125f && sT <= 0x1p125f) ? __fdiv_rn(1.0f, sT) : 0.0f;
-    ns.inv_tab = inv_tab;
+    ns.tab = near_tab;
 
     Acc acc = {0, 0, 0, 0, 0};
     if (warp == kConsumers / 32) {
@@ -103,8 +107,10 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) 
         if (lane == 0) ring.produce(&tm, ntiles, kWaitEmpty);
         __syncwarp();
     } else {
-        constexpr bool nearest = NEAR;              // UE4M3 / UE5M3 nearest scales
-        constexpr bool exact = !NEAR && !MBS;       // scales are powers of two
+        // rotation with power-of-two scales: the normaliser c = 1/sqrt(n) moves
+        // into the scale, s = y_H * (c * 2^-k) = (y_H * c) * 2^-k exactly
+        constexpr bool FOLD = HADN != 0 && !MBS && !NEAR;
+        const float hc = HADN ? hadamard_scale(HADN) : 1.0f;
         const bool e8m0 = !NEAR && p.sd.fmt == S_E8M0;
         const float thr_m = e8m0_threshold(p.ed, p.sd);
         const uint32_t S = (uint32_t)(p.cols / B);
@@ -112,17 +118,14 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) 
         uint32_t i = 0;
         for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
             if (!ring.acquire(i, kWaitFull)) break;
-            float ys[MBS ? 32 : 1];         // pre-macro-scale values (statistics reference)
             float y[32];
             ring_read_chunk(ring.stage(i % RingCfg<InT>::kStages), t, static_cast<const InT *>(nullptr), y);
             ring.release(i);                  // the chunk is in registers: hand the slot back
-            if constexpr (HADN != 0) hadamard_groups<HADN>(y);
+            if constexpr (HADN != 0) hadamard_groups<HADN, !FOLD>(y);
             // macro-block scale: y' = y * (1 / S_M), x_hat = (q X) S_M
             float sm = 1.0f;
             if constexpr (MBS) {
-                float m = 0.0f;
-#pragma unroll
-                for (int j = 0; j < 32; j += 2) m = fmax3_nan(m, fabsf(y[j]), fabsf(y[j + 1]));
+                const float m = absmax_nan<32>(y);
                 int mbad = !(m <= FLT_MAX);
                 float mm = grp_max(mbad ? 0.0f : m, 4);
                 mbad = grp_or(mbad, 4);
@@ -130,11 +133,12 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) 
                 sm = e4m3_value(mcode);
                 const float invm = __fdiv_rn(1.0f, sm);
                 if ((t & 3) == 0 && tile * kConsumers + t < nch) p.macro[(tile * kConsumers + t) >> 2] = (uint8_t)mcode;
-                // keep y for the statistics: scale a copy below
+                const float2 invm2 = make_float2(invm, invm);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) ys[j] = y[j];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) y[j] = __fmul_rn(y[j], invm);
+                for (int j = 0; j < 32; j += 2) {
+                    const float2 v = __fmul2_rn(make_float2(y[j], y[j + 1]), invm2);
+                    y[j] = v.x; y[j + 1] = v.y;
+                }
             }
 
             const uint32_t c = tile * kConsumers + t;
@@ -142,29 +146,47 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) 
             uint32_t words[4];
             uint32_t scode[NB];
             // packed two-lane binary32 arithmetic (each lane rounded as a scalar op)
-            float2 sx2 = make_float2(0.f, 0.f), se2 = sx2, sb2 = sx2;
-            float2 sx2v[2] = {sx2, sx2};            // sum of y^2, power-of-two scale path
             int nzc = 0, ftzc = 0;
 #pragma unroll
             for (int k = 0; k < NB; ++k) {
                 const int j0 = k * L;
                 float a = absmax_nan<L>(y + j0), mabs = 1.0f;
-                if (STATS) mabs = absmin<L>((MBS ? ys : y) + (MBS ? j0 : j0));
+                if (STATS) mabs = absmin<L>(y + j0);
                 int bad = !(a <= FLT_MAX);
                 if (G > 1) {
                     a = grp_max(bad ? 0.0f : a, G);
                     bad = grp_or(bad, G);
                 }
+                if (FOLD) a = __fmul_rn(a, hc);            // max |y_H c| = RN(max |y_H| c)
                 const BlockScale bs = NEAR ? near_block_scale(p.sd, ns, bad ? 0.0f : a, bad)
                                     : e8m0 ? e8m0_block_scale(bad ? 0.0f : a, bad, p.ed.emax, thr_m)
                                            : block_scale(p.ed, p.sd, bad ? 0.0f : a, bad, sT);
                 scode[k] = bs.code;
-                float deqT = bs.nan ? __uint_as_float(0x7fc00000u) : nearest ? __fmul_rn(bs.deq, sT) : bs.deq;
+                float deqT = bs.nan ? __uint_as_float(0x7fc00000u) : bs.deq;     // nearest: s_b s_T
                 if (MBS) deqT = __fmul_rn(deqT, sm);       // X * S_M is exact (power of two times E4M3)
-                const float2 inv2 = make_float2(bs.inv, bs.inv);
-                const float2 nq2 = make_float2(-deqT, -deqT);
-                // power-of-two scale: y = X s exactly, so y - x_hat = X (s - q)
-                // and the block's sums are taken on the scaled values
+                float inv = bs.inv;
+                // folded rotation: inv = c 2^-k, exact unless subnormal; then
+                // (rare) normalise the block's values first
+                float sxm = MBS ? sm : FOLD ? hc : 1.0f;  // reference values = sxm * y
+                if (FOLD) {
+                    if (inv >= 0x1p-123f || bs.zero) {
+                        inv = __fmul_rn(inv, hc);
+                    } else {
+#pragma unroll
+                        for (int j = j0; j < j0 + L; ++j) y[j] = __fmul_rn(y[j], hc);
+                        sxm = 1.0f;
+                    }
+                }
+                // a flushed block (x_hat = 0, not NaN): residuals are the
+                // reference values themselves, s = sxm * y with factor 1
+                if (bs.zero && !bs.nan) {
+                    inv = sxm;
+                    deqT = 1.0f;
+                }
+                const float2 inv2 = make_float2(inv, inv);
+                float2 sx2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                // residuals on the scaled values: y - x_hat = deqT (s - q), exact
+                // for power-of-two scales, within an ulp of y otherwise
                 float2 re2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)}, rb2[2] = {re2[0], re2[0]};
                 int qz = 0;
 #pragma unroll
@@ -180,50 +202,36 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) 
                     const uint32_t word = bs.zero ? 0u : cvt_e2m1x8(s8);
                     words[jb >> 3] = word;
                     if (STATS) {
-                        if constexpr (exact) {
-                            uint32_t h[4];
-                            e2m1x8_halves(word, h);
+                        uint32_t h[4];
+                        e2m1x8_halves(word, h);
 #pragma unroll
-                            for (int e = 0; e < 8; e += 2) {
-                                const float2 d = sub_f16x2_from(s8[e], s8[e + 1], h[e >> 1]);   // s - q
-                                const int u = (e >> 1) & 1;          // two accumulator chains
-                                re2[u] = __ffma2_rn(d, d, re2[u]);
-                                rb2[u] = __fadd2_rn(rb2[u], d);
-                                const float2 yv = make_float2(y[jb + e], y[jb + e + 1]);
-                                sx2v[u] = __ffma2_rn(yv, yv, sx2v[u]);
-                            }
-                        } else {
-                            float q[8];
-                            e2m1x8_values(word, q);
-#pragma unroll
-                            for (int e = 0; e < 8; e += 2) {
-                                const float2 yv = MBS ? make_float2(ys[MBS ? jb + e : 0], ys[MBS ? jb + e + 1 : 0])
-                                                      : make_float2(y[jb + e], y[jb + e + 1]);
-                                const float2 d = __ffma2_rn(make_float2(q[e], q[e + 1]), nq2, yv);   // y - q deq
-                                se2 = __ffma2_rn(d, d, se2);
-                                sx2 = __ffma2_rn(yv, yv, sx2);
-                                sb2 = __fadd2_rn(sb2, d);
-                            }
+                        for (int e = 0; e < 8; e += 2) {
+                            const float2 d = sub_f16x2_from(s8[e], s8[e + 1], h[e >> 1]);   // s - q
+                            const int u = (e >> 1) & 1;          // two accumulator chains
+                            re2[u] = __ffma2_rn(d, d, re2[u]);
+                            rb2[u] = __fadd2_rn(rb2[u], d);
+                            const float2 yv = make_float2(y[jb + e], y[jb + e + 1]);
+                            sx2[u] = __ffma2_rn(yv, yv, sx2[u]);
                         }
                         qz += zero_codes8(word);
                     }
                 }
                 if (STATS) {
-                    if (exact && ok) {
-                        const double X = bs.nan ? (double)__uint_as_float(0x7fc00000u) : (double)bs.deq;
+                    if (ok) {
+                        // y - x_hat = deqT (s - q); a NaN block makes the sums NaN
+                        const double X = (double)deqT, R = (double)sxm;
                         acc.e2 += (double)((re2[0].x + re2[1].x) + (re2[0].y + re2[1].y)) * X * X;
                         acc.e -= (double)((rb2[0].x + rb2[1].x) + (rb2[0].y + rb2[1].y)) * X;
+                        acc.x2 += (double)((sx2[0].x + sx2[1].x) + (sx2[0].y + sx2[1].y)) * R * R;
                     }
                     int xz = 0;
                     if (mabs == 0.0f)                      // rare: count exact zeros
 #pragma unroll
-                        for (int j = j0; j < j0 + L; ++j) xz += ((MBS ? ys[MBS ? j : 0] : y[j]) == 0.0f);
+                        for (int j = j0; j < j0 + L; ++j) xz += (y[j] == 0.0f);
                     nzc += L - xz;
                     if (!bs.nan) ftzc += qz - xz;
                 }
             }
-            sx2 = __fadd2_rn(sx2, __fadd2_rn(sx2v[0], sx2v[1]));
-            const float sx = sx2.x + sx2.y, se = se2.x + se2.y, sb = -(sb2.x + sb2.y);
             if (ok) {
                 reinterpret_cast<uint4 *>(p.codes)[c] = make_uint4(words[0], words[1], words[2], words[3]);
                 if (G == 1 || (lane & (G - 1)) == 0) {
@@ -243,9 +251,6 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) 
                     }
                 }
                 if (STATS) {
-                    acc.x2 += (double)sx;
-                    acc.e2 += (double)se;
-                    acc.e += (double)sb;
                     acc.nz += (double)nzc;
                     acc.ftz += (double)ftzc;
                 }
