@@ -401,17 +401,17 @@ def run_e2e(mx, A_cpu, W_cpu, plan, outs, device, args, step_bytes, world):
 
 
 def run_gemm(mx, A, W, device, args, world):
-    """Block-scaled FP4 GEMM C = A^Q W^Q^T (MXFP4, NVFP4, and MBS operands on
-    the NVFP4 kind) and QSNR(AB)."""
+    """Block-scaled GEMM C = A^Q W^Q^T (MXFP4, NVFP4, MBS operands on the NVFP4
+    kind, MXFP6) and QSNR(AB)."""
     out = {}
     pk, pk_src = peaks()
-    fp4_peak = pk["bf16_tflops"] * 4.0      # nominal dense ratio fp4 : bf16 = 9 : 2.25
     stream = torch.cuda.current_stream(device)
     flop = 2.0 * M_TOK * N_OUT * K_DIM
     mbs = mx.Config(macro_block=128)
     for name, cfg in (("mxfp4", mx.Config(sf_layout=1)),
                       ("nvfp4", mx.Config(block=16, scale_fmt=1, rule=3, tensor_scale=1, sf_layout=1)),
-                      ("mbs_mxfp4_via_nvf4", mbs)):
+                      ("mbs_mxfp4_via_nvf4", mbs),
+                      ("mxfp6_e2m3", mx.Config(elem=mx.E2M3, sf_layout=1))):
         qa = mx.quantize(A, cfg, stats=False)
         qw = mx.quantize(W, cfg, stats=False)
         if cfg.macro_block:
@@ -440,10 +440,13 @@ def run_gemm(mx, A, W, device, args, world):
         torch.cuda.synchronize(device)
         ms = s.elapsed_time(e) / steps
         tf = flop / (ms * 1e-3) / 1e12
+        # FP6 runs at the FP8 rate (kind::mxf8f6f4): nominal 2x bf16; FP4 4x
+        ratio = 2.0 if cfg.elem in (mx.E2M3, mx.E3M2) else 4.0
+        peak = pk["bf16_tflops"] * ratio
         rec = {"TFLOPS": round(tf, 1), "ms": round(ms, 4), "unit": "TFLOP/s",
-               "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(fp4_peak, 1),
-                            "unit": "TFLOP/s", "frac": round(tf / fp4_peak, 4),
-                            "peak_source": f"{pk_src} bf16 x 4 (nominal fp4:bf16 dense ratio)"}}
+               "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(peak, 1),
+                            "unit": "TFLOP/s", "frac": round(tf / peak, 4),
+                            "peak_source": f"{pk_src} bf16 x {ratio:g} (nominal dense ratio to bf16)"}}
         try:
             st = mx.gemm_qsnr(A, W, qa, qw)
             torch.cuda.synchronize(device)
@@ -548,8 +551,9 @@ def kernel_case(args):
     res = {"case": case, "stats": not args.no_stats}
     if case.startswith("gemm"):
         M, N, K = M_TOK, N_OUT, K_DIM
-        cfg = (mx.Config(sf_layout=1) if case == "gemm_mxfp4" else
-               mx.Config(block=16, scale_fmt=1, rule=3, tensor_scale=1, sf_layout=1))
+        cfg = {"gemm_mxfp4": mx.Config(sf_layout=1),
+               "gemm_nvfp4": mx.Config(block=16, scale_fmt=1, rule=3, tensor_scale=1, sf_layout=1),
+               "gemm_mxfp6": mx.Config(elem=mx.E2M3, sf_layout=1)}[case]
         a = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
         w = (torch.randn(N, K, generator=g, device=dev) * 0.02).to(torch.bfloat16)
         qa, qw = mx.quantize(a, cfg, stats=False), mx.quantize(w, cfg, stats=False)

@@ -79,6 +79,13 @@ extern "C" {
 #define MX_RULE_CEIL    1
 #define MX_RULE_OAS     2
 #define MX_RULE_NEAREST 3
+/* MSE: per-block MSE-optimal E8M0 scale (a per-block scale search; the pages
+ * suggest optimising scales for MSE but fix no search): the exponent among
+ * k_floor and k_floor + 1 whose nearest-even codes leave the smaller block
+ * squared error, 4^k sum (v - q)^2 with v = binary32(x 2^-k), each sum in
+ * binary64 in element order, ties to k_floor.  E8M0, MX_ROUND_RTNE, row
+ * axis, block 32, symmetric, no macro scale or rotation. */
+#define MX_RULE_MSE     4
 
 /* ---- element rounding ([MX-TRAIN]) ------------------------------------- */
 #define MX_ROUND_RTNE       0   /* nearest, ties to the even code, saturating */
@@ -116,7 +123,11 @@ typedef struct {
                               only; rows % 128 == 0, (cols / block) % 4 == 0): for row r and
                               scale j of a row holding S = cols / block scales, byte
                               ((r/128)*(S/4) + j/4)*512 + (r%32)*16 + ((r/32)%4)*4 + j%4,
-                              the layout mx_gemm copies into tensor memory */
+                              the layout mx_gemm copies into tensor memory.  With FP6
+                              elements it also sets the code layout to the tensor core's
+                              operand form: every 16 codes of a row in 12 bytes (code i at
+                              bits [6i, 6i+6) of the little-endian group) and 4 zero bytes,
+                              still one byte per element; FP4 codes are unchanged */
     uint64_t seed;         /* stochastic-rounding key */
 } mx_config;
 
@@ -247,7 +258,9 @@ int mx_qsnr(const void *x, int32_t x_dtype, const void *x_hat, int32_t x_hat_dty
  * tcgen05 chunk layout (ca/cb->sf_layout = 1, as mx_quantize wrote them).
  * MXFP4: block 32, E8M0 (ca/cb rule FLOOR, CEIL or OAS).  NVFP4: block 16,
  * UE4M3 NEAREST with tensor scales tsA/tsB (device floats; used when
- * ca/cb->tensor_scale != MX_TS_NONE, else 1).  C: device, bf16 or fp32
+ * ca/cb->tensor_scale != MX_TS_NONE, else 1).  MXFP6 ([MX-TRAIN]'s MX6;
+ * tcgen05 kind::mxf8f6f4): E2M3 and / or E3M2 codes, one per byte as
+ * mx_quantize writes them, block 32, E8M0; N % 256 == 0.  C: device, bf16 or fp32
  * (c_dtype), row-major M x N.  M % 128 == 0, N % 128 == 0, K % 256 == 0.
  * Tiles: 128 x 256 per SM (persistent) when N % 256 == 0, else 128 x 128.
  */

@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libmx_b200.so")
 MX_OK = 0
 E2M1, E3M0, E2M3, E3M2, INT4 = 0, 1, 2, 3, 4
 SCALE_E8M0, SCALE_UE4M3, SCALE_UE5M3 = 0, 1, 2
-RULE_FLOOR, RULE_CEIL, RULE_OAS, RULE_NEAREST = 0, 1, 2, 3
+RULE_FLOOR, RULE_CEIL, RULE_OAS, RULE_NEAREST, RULE_MSE = 0, 1, 2, 3, 4
 ROUND_RTNE, ROUND_CEIL, ROUND_STOCHASTIC = 0, 1, 2
 AXIS_ROW, AXIS_COL, AXIS_2D = 0, 1, 2
 DT_BF16, DT_FP32 = 0, 1

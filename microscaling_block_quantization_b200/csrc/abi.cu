@@ -71,7 +71,11 @@ int check_config(const mx_config *c, int64_t rows, int64_t cols, bool want_had)
     if (c->sf_layout == 1 && c->axis != MX_AXIS_ROW) return MX_ERR_UNSUPPORTED;
     if (c->elem < MX_E2M1 || c->elem > MX_INT4) return MX_ERR_INVALID;
     if (c->scale_fmt < MX_SCALE_E8M0 || c->scale_fmt > MX_SCALE_UE5M3) return MX_ERR_INVALID;
-    if (c->rule < MX_RULE_FLOOR || c->rule > MX_RULE_NEAREST) return MX_ERR_INVALID;
+    if (c->rule < MX_RULE_FLOOR || c->rule > MX_RULE_MSE) return MX_ERR_INVALID;
+    if (c->rule == MX_RULE_MSE &&
+        (c->scale_fmt != MX_SCALE_E8M0 || c->round != MX_ROUND_RTNE || c->axis != MX_AXIS_ROW ||
+         c->block != 32 || c->asymmetric || c->macro_block || c->hadamard || c->tensor_scale != MX_TS_NONE))
+        return MX_ERR_UNSUPPORTED;
     if (c->round < MX_ROUND_RTNE || c->round > MX_ROUND_STOCHASTIC) return MX_ERR_INVALID;
     if (c->axis < MX_AXIS_ROW || c->axis > MX_AXIS_2D) return MX_ERR_INVALID;
     if (c->asymmetric != 0 && c->asymmetric != 1) return MX_ERR_INVALID;
@@ -208,7 +212,8 @@ int quantize_impl(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t 
     p.stats = stats;
     p.count = (double)n;
     p.ticket = need_ws ? reinterpret_cast<unsigned int *>(ws + kWsTicket) : nullptr;
-    const int fast = cfg->elem == MX_E2M1 && cfg->round == MX_ROUND_RTNE && !cfg->asymmetric;
+    const int fast = cfg->elem == MX_E2M1 && cfg->round == MX_ROUND_RTNE && !cfg->asymmetric &&
+                     cfg->rule != MX_RULE_MSE;
     int grid = 0;
     if (launch_quantize(p, cfg->axis, in_fp32, fast, st, &grid)) return MX_ERR_CUDA;
     return MX_OK;

@@ -116,8 +116,13 @@ __global__ void __launch_bounds__(kThreads) k_dequant_chunk(const DParams p)
             } else {
                 const uint4 u0 = reinterpret_cast<const uint4 *>(p.codes)[2 * (size_t)c];
                 const uint4 u1 = reinterpret_cast<const uint4 *>(p.codes)[2 * (size_t)c + 1];
-                w[0] = u0.x; w[1] = u0.y; w[2] = u0.z; w[3] = u0.w;
-                w[4] = u1.x; w[5] = u1.y; w[6] = u1.z; w[7] = u1.w;
+                if (p.sf_gemm) {                    // tensor-core operand layout
+                    fp6_group_unpack(u0, w);
+                    fp6_group_unpack(u1, w + 4);
+                } else {
+                    w[0] = u0.x; w[1] = u0.y; w[2] = u0.z; w[3] = u0.w;
+                    w[4] = u1.x; w[5] = u1.y; w[6] = u1.z; w[7] = u1.w;
+                }
             }
             if (FAST) {
                 // E2M1, symmetric, power-of-two or NEAREST scales, row or 2D axis, no MBS

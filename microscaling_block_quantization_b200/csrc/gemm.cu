@@ -38,7 +38,7 @@ constexpr int kTmemCols = 256;
 constexpr int kTileBytes = BM * 128;              // one operand tile: 128 rows x 128 bytes
 constexpr uint64_t kWaitNs = 2000000000ull;       // bound of one mbarrier wait: 2 s
 
-enum { KIND_BF16 = 0, KIND_MXF4 = 1, KIND_NVF4 = 2 };
+enum { KIND_BF16 = 0, KIND_MXF4 = 1, KIND_NVF4 = 2, KIND_MXF6 = 3 };
 enum { EPI_BF16 = 0, EPI_F32 = 1, EPI_QSNR = 2 };
 
 // device status word of the bounded waits (read and cleared by mx_device_status)
@@ -51,6 +51,7 @@ struct GParams {
     void *C;                     // EPI_BF16 / EPI_F32 output, row-major M x N
     const float *Cq;             // EPI_QSNR: the quantized product, fp32 M x N
     double *partials;            // EPI_QSNR: per-CTA [sum C^2, sum (C - Cq)^2]
+    uint32_t ab_fmt;             // KIND_MXF6: A / B element formats of the instruction descriptor
 };
 
 template <int KIND>
@@ -176,6 +177,10 @@ __device__ __forceinline__ void mma(uint32_t dt, uint64_t ad, uint64_t bd, uint3
     } else if constexpr (KIND == KIND_MXF4) {
         asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
                      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+                     ::"r"(dt), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
+    } else if constexpr (KIND == KIND_MXF6) {
+        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
                      ::"r"(dt), "l"(ad), "l"(bd), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb));
     } else {
         asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
@@ -395,7 +400,10 @@ constexpr int kTmemColsP = 512;
 
 template <int KIND>
 struct KindP {
-    static constexpr int kChunks = KIND == KIND_MXF4 ? 2 : 4;       // 4-scale chunks per stage (K = 256)
+    // 4-scale chunks per stage: a stage is 128 bytes of every row, K = 256
+    // E2M1 elements (MXF4: 8 blocks of 32, NVF4: 16 of 16) or K = 128 FP6
+    // elements in byte containers (MXF6: 4 blocks of 32)
+    static constexpr int kChunks = KIND == KIND_MXF4 ? 2 : KIND == KIND_MXF6 ? 1 : 4;
     static constexpr int kSfaBytes = kChunks * 512;                  // 128 rows of A
     static constexpr int kSfbBytes = 2 * kChunks * 512;              // 256 rows of B
     static constexpr int kABytes = BM * 128, kBBytes = BNP * 128;
@@ -404,10 +412,11 @@ struct KindP {
 };
 
 template <int KIND>
-__device__ __forceinline__ uint32_t idesc_p()
+__device__ __forceinline__ uint32_t idesc_p(uint32_t ab_fmt)
 {
-    uint32_t d = (1u << 7) | (1u << 10);          // A, B E2M1
-    if (KIND == KIND_MXF4) d |= 1u << 23;        // UE8M0 scales
+    // A, B formats: E2M1 (kind::mxf4 / mxf4nvf4), or E2M3 = 3 / E3M2 = 4 (kind::mxf8f6f4)
+    uint32_t d = KIND == KIND_MXF6 ? ab_fmt : (1u << 7) | (1u << 10);
+    if (KIND != KIND_NVF4) d |= 1u << 23;        // UE8M0 scales
     d |= (uint32_t)(BNP >> 3) << 17;
     d |= (uint32_t)(BM >> 4) << 24;
     return d;
@@ -433,7 +442,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ntn = p.N / BNP, ntm = p.M / BM;
     const int ntiles = ntn * ntm;
-    const int ktiles = p.K / 256;
+    const int ktiles = p.K / (KIND == KIND_MXF6 ? 128 : 256);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStagesP; ++s) {
@@ -458,7 +467,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            const int sf_chunks_row = (p.K / (KIND == KIND_MXF4 ? 32 : 16)) / 4;
+            const int sf_chunks_row = (p.K / (KIND == KIND_NVF4 ? 16 : 32)) / 4;
             uint32_t it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
@@ -481,7 +490,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idesc0 = idesc_p<KIND>();
+            const uint32_t idesc0 = idesc_p<KIND>(p.ab_fmt);
             uint32_t it = 0, tcount = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tcount) {
@@ -510,10 +519,17 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                     for (int k = 0; k < 4; ++k) {
                         uint32_t idesc = idesc0, sfa, sfb;
                         if constexpr (KIND == KIND_MXF4) {
+                            // K = 64: two 32-blocks, scale bytes 0-1 or 2-3 of a chunk column
                             const uint32_t id = (k & 1) * 2;
                             idesc |= (id << 29) | (id << 4);
                             sfa = sfa_t + 4 * (k >> 1);
                             sfb = sfb_t + 8 * (k >> 1);
+                        } else if constexpr (KIND == KIND_MXF6) {
+                            // K = 32: one 32-block, scale byte k of the stage's chunk column
+                            const uint32_t id = (uint32_t)k;
+                            idesc |= (id << 29) | (id << 4);
+                            sfa = sfa_t;
+                            sfb = sfb_t;
                         } else {
                             sfa = sfa_t + 4 * k;
                             sfb = sfb_t + 8 * k;
@@ -627,13 +643,16 @@ EncodeTiled encoder()
 }
 
 // rows x row_bytes operand, box of 128 rows x 128 bytes, 128-byte swizzle
-bool make_map(CUtensorMap *m, const void *base, int rows, int K, bool bf16, unsigned box_rows = 128)
+// elem_bits: 16 (bf16), 4 (packed E2M1) or 8 (FP6 codes, one per byte)
+bool make_map(CUtensorMap *m, const void *base, int rows, int K, int elem_bits, unsigned box_rows = 128)
 {
     EncodeTiled enc = encoder();
     if (!enc) return false;
-    const cuuint64_t inner = bf16 ? (cuuint64_t)K : (cuuint64_t)K / 2;
+    const bool bf16 = elem_bits == 16;
+    const cuuint64_t row_bytes = (cuuint64_t)K * elem_bits / 8;
+    const cuuint64_t inner = bf16 ? (cuuint64_t)K : row_bytes;
     const cuuint64_t dims[2] = {inner, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {bf16 ? (cuuint64_t)K * 2 : (cuuint64_t)K / 2};
+    const cuuint64_t strides[1] = {row_bytes};
     const cuuint32_t box[2] = {bf16 ? 64u : 128u, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
@@ -646,8 +665,8 @@ template <int KIND, int EPI>
 int launch(const GParams &p, const void *A, const void *B, cudaStream_t st)
 {
     CUtensorMap ta, tb;
-    const bool bf16 = KIND == KIND_BF16;
-    if (!make_map(&ta, A, p.M, p.K, bf16) || !make_map(&tb, B, p.N, p.K, bf16)) return MX_ERR_CUDA;
+    const int bits = KIND == KIND_BF16 ? 16 : 4;
+    if (!make_map(&ta, A, p.M, p.K, bits) || !make_map(&tb, B, p.N, p.K, bits)) return MX_ERR_CUDA;
     using KT = Kind<KIND>;
     const int smem = 1024 + kStages * KT::kStageBytes + 256;
     auto k = k_gemm<KIND, EPI>;
@@ -667,7 +686,8 @@ template <int KIND, int EPI>
 int launch_p(const GParams &p, const void *A, const void *B, cudaStream_t st)
 {
     CUtensorMap ta, tb;
-    if (!make_map(&ta, A, p.M, p.K, false, 128) || !make_map(&tb, B, p.N, p.K, false, 256)) return MX_ERR_CUDA;
+    const int bits = KIND == KIND_MXF6 ? 8 : 4;
+    if (!make_map(&ta, A, p.M, p.K, bits, 128) || !make_map(&tb, B, p.N, p.K, bits, 256)) return MX_ERR_CUDA;
     using KT = KindP<KIND>;
     const int smem = 1024 + kStagesP * KT::kStageBytes + 256;
     auto k = k_gemm_p<KIND, EPI>;
@@ -689,17 +709,30 @@ int launch_p(const GParams &p, const void *A, const void *B, cudaStream_t st)
 int fp4_kind(const mx_config *a, const mx_config *b)
 {
     if (!a || !b) return -1;
-    auto same = [](const mx_config *c) {
-        return c->elem == MX_E2M1 && c->axis == MX_AXIS_ROW && c->sf_layout == 1 && !c->asymmetric &&
-               !c->macro_block;
+    auto layout = [](const mx_config *c) {
+        return c->axis == MX_AXIS_ROW && c->sf_layout == 1 && !c->asymmetric && !c->macro_block && !c->hadamard;
     };
-    if (!same(a) || !same(b)) return -1;
+    if (!layout(a) || !layout(b)) return -1;
+    auto fp6 = [](const mx_config *c) { return c->elem == MX_E2M3 || c->elem == MX_E3M2; };
+    if (fp6(a) && fp6(b)) {
+        if (a->scale_fmt == MX_SCALE_E8M0 && b->scale_fmt == MX_SCALE_E8M0 && a->block == 32 && b->block == 32)
+            return KIND_MXF6;
+        return -1;
+    }
+    if (a->elem != MX_E2M1 || b->elem != MX_E2M1) return -1;
     if (a->scale_fmt == MX_SCALE_E8M0 && b->scale_fmt == MX_SCALE_E8M0 && a->block == 32 && b->block == 32)
         return KIND_MXF4;
     if (a->scale_fmt == MX_SCALE_UE4M3 && b->scale_fmt == MX_SCALE_UE4M3 && a->rule == MX_RULE_NEAREST &&
         b->rule == MX_RULE_NEAREST && a->block == 16 && b->block == 16)
         return KIND_NVF4;
     return -1;
+}
+
+// kind::mxf8f6f4 operand formats (instruction descriptor bits 7-9 and 10-12)
+uint32_t fp6_formats(const mx_config *a, const mx_config *b)
+{
+    const uint32_t fa = a->elem == MX_E2M3 ? 3u : 4u, fb = b->elem == MX_E2M3 ? 3u : 4u;
+    return (fa << 7) | (fb << 10);
 }
 
 bool shapes_ok(int64_t M, int64_t N, int64_t K)
@@ -748,6 +781,13 @@ int mx_gemm(const mx_config *ca, const mx_config *cb, const void *Aq, const uint
     }
     p.C = C;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (kind == KIND_MXF6) {
+        // MXFP6: the persistent 128 x 256 kernel only
+        if (N % BNP) return MX_ERR_UNSUPPORTED;
+        p.ab_fmt = fp6_formats(ca, cb);
+        return c_dtype == MX_DT_BF16 ? launch_p<KIND_MXF6, EPI_BF16>(p, Aq, Bq, st)
+                                     : launch_p<KIND_MXF6, EPI_F32>(p, Aq, Bq, st);
+    }
     if (N % BNP == 0) {
         if (kind == KIND_MXF4)
             return c_dtype == MX_DT_BF16 ? launch_p<KIND_MXF4, EPI_BF16>(p, Aq, Bq, st)

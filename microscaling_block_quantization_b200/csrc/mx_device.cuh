@@ -21,7 +21,7 @@ namespace mxk {
 
 enum { E2M1 = 0, E3M0 = 1, E2M3 = 2, E3M2 = 3, INT4 = 4 };
 enum { S_E8M0 = 0, S_UE4M3 = 1, S_UE5M3 = 2 };
-enum { R_FLOOR = 0, R_CEIL = 1, R_OAS = 2, R_NEAREST = 3 };
+enum { R_FLOOR = 0, R_CEIL = 1, R_OAS = 2, R_NEAREST = 3, R_MSE = 4 };
 enum { RD_RTNE = 0, RD_CEIL = 1, RD_SR = 2 };
 enum { AX_ROW = 0, AX_COL = 1, AX_2D = 2 };
 enum { TS_NONE = 0, TS_COMPUTE = 1, TS_GIVEN = 2 };
@@ -150,6 +150,37 @@ __device__ __forceinline__ float decode_elem(const ElemDesc &d, uint32_t code)
     uint32_t sbit = 1u << (d.code_bits - 1);
     float mv = mag_value(d, (int)(code & (sbit - 1)));
     return (code & sbit) ? -mv : mv;
+}
+
+// FP6 codes of 32 elements, one per byte (4 per word, code j in byte j % 4
+// of word j / 4), <-> the tensor-core operand layout: each 16 codes packed
+// into 12 bytes (code i at bits [6i, 6i + 6) of the little-endian 96-bit
+// group), then 4 zero bytes.
+__device__ __forceinline__ uint4 fp6_group_pack(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3)
+{
+    uint32_t c[16];
+    const uint32_t w[4] = {w0, w1, w2, w3};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) c[i] = (w[i >> 2] >> (8 * (i & 3))) & 0x3fu;
+    uint4 r;
+    r.x = c[0] | (c[1] << 6) | (c[2] << 12) | (c[3] << 18) | (c[4] << 24) | (c[5] << 30);
+    r.y = (c[5] >> 2) | (c[6] << 4) | (c[7] << 10) | (c[8] << 16) | (c[9] << 22) | (c[10] << 28);
+    r.z = (c[10] >> 4) | (c[11] << 2) | (c[12] << 8) | (c[13] << 14) | (c[14] << 20) | (c[15] << 26);
+    r.w = 0u;
+    return r;
+}
+__device__ __forceinline__ void fp6_group_unpack(uint4 g, uint32_t w[4])
+{
+    const uint64_t lo = (uint64_t)g.x | ((uint64_t)g.y << 32);
+    const uint64_t hi = (uint64_t)g.y | ((uint64_t)g.z << 32);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w[k] = 0u;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int bit = 6 * i;
+        const uint32_t c = bit < 32 + 26 ? (uint32_t)(lo >> bit) & 0x3fu : (uint32_t)(hi >> (bit - 32)) & 0x3fu;
+        w[i >> 2] |= c << (8 * (i & 3));
+    }
 }
 
 // E2M1 fast path: eight binary32 values -> eight nibbles, element j in bits

@@ -102,6 +102,45 @@ __device__ __forceinline__ uint32_t encode_grid(float v, uint32_t u, float &q)
     }
 }
 
+// MSE-optimal E8M0 scale of a 32-element block (alpha > 0 finite): the
+// exponent among k_floor and k_floor + 1 whose nearest-even codes leave the
+// smaller squared error, 4^k sum (v - q)^2 with v = RN(y 2^-k); the two sums
+// are accumulated in binary64 in element order (every term exact) and
+// compared as S(k_floor) <= 4 S(k_floor + 1), ties to k_floor.
+template <int ELEM>
+__device__ __forceinline__ BlockScale mse_block_scale(const float y[32], float alpha, int emax)
+{
+    const uint32_t b = __float_as_uint(alpha);
+    const int kf = (b >> 23) == 0 ? -1000 : (int)(b >> 23) - 127 - emax;
+    const int k0 = min(max(kf, -127), 127), k1 = min(max(kf + 1, -127), 127);
+    int k = k0;
+    if (k1 != k0) {
+        double sum[2];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const float inv = exp2i(-(c ? k1 : k0));
+            double acc = 0.0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const float v = __fmul_rn(y[j], inv);
+                float q;
+                (void)encode_grid<ELEM, RD_RTNE, false>(v, 0u, q);
+                const double d = (double)v - (double)q;
+                acc = __dadd_rn(acc, __dmul_rn(d, d));
+            }
+            sum[c] = acc;
+        }
+        k = (sum[0] <= 4.0 * sum[1]) ? k0 : k1;
+    }
+    BlockScale r;
+    r.code = (uint32_t)(k + 127);
+    r.inv = exp2i(-k);
+    r.deq = exp2i(k);
+    r.zero = 0;
+    r.nan = 0;
+    return r;
+}
+
 // nearest-even conversion instructions: two binary32 values -> two codes
 __device__ __forceinline__ uint32_t cvt_e2m3x2(float a0, float a1)
 {
@@ -177,7 +216,9 @@ __global__ void __launch_bounds__(kRingThreads, 2) k_quant_gen(const QParams p, 
                 }
                 a = ra;
             }
-            const BlockScale bs = block_scale(p.ed, p.sd, bad ? 0.0f : a, bad, sT);
+            const BlockScale bs = (!ASYM && p.sd.rule == R_MSE && !bad && a > 0.0f)
+                                      ? mse_block_scale<ELEM>(y, a, p.ed.emax)
+                                      : block_scale(p.ed, p.sd, bad ? 0.0f : a, bad, sT);
             const float2 inv2 = make_float2(bs.inv, bs.inv);
 
             // element codes and grid values
@@ -235,9 +276,15 @@ __global__ void __launch_bounds__(kRingThreads, 2) k_quant_gen(const QParams p, 
                     reinterpret_cast<uint4 *>(p.codes)[c] = make_uint4(words[0], words[1], words[2], words[3]);
                 } else {
                     uint4 *dst = reinterpret_cast<uint4 *>(p.codes) + 2 * (size_t)c;
-                    dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-                    dst[NW > 4 ? 1 : 0] = make_uint4(words[NW > 4 ? 4 : 0], words[NW > 4 ? 5 : 0],
-                                                     words[NW > 4 ? 6 : 0], words[NW > 4 ? 7 : 0]);
+                    if (p.sf_gemm) {                // tensor-core operand layout
+                        dst[0] = fp6_group_pack(words[0], words[1], words[2], words[3]);
+                        dst[NW > 4 ? 1 : 0] = fp6_group_pack(words[NW > 4 ? 4 : 0], words[NW > 4 ? 5 : 0],
+                                                             words[NW > 4 ? 6 : 0], words[NW > 4 ? 7 : 0]);
+                    } else {
+                        dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+                        dst[NW > 4 ? 1 : 0] = make_uint4(words[NW > 4 ? 4 : 0], words[NW > 4 ? 5 : 0],
+                                                         words[NW > 4 ? 6 : 0], words[NW > 4 ? 7 : 0]);
+                    }
                 }
                 if (p.sf_gemm) {
                     const uint32_t S = (uint32_t)(p.cols / 32), r = c / S;

@@ -232,8 +232,15 @@ __global__ void __launch_bounds__(kThreads) k_quant_row(const QParams p)
                 reinterpret_cast<uint4 *>(p.codes)[c] = make_uint4(words[0], words[1], words[2], words[3]);
             } else {
                 uint4 *dst = reinterpret_cast<uint4 *>(p.codes) + 2 * (size_t)c;
-                dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-                dst[1] = make_uint4(words[FAST ? 0 : 4], words[FAST ? 0 : 5], words[FAST ? 0 : 6], words[FAST ? 0 : 7]);
+                if (p.sf_gemm) {                    // tensor-core operand layout
+                    dst[0] = fp6_group_pack(words[0], words[1], words[2], words[3]);
+                    dst[1] = fp6_group_pack(words[FAST ? 0 : 4], words[FAST ? 0 : 5], words[FAST ? 0 : 6],
+                                            words[FAST ? 0 : 7]);
+                } else {
+                    dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+                    dst[1] = make_uint4(words[FAST ? 0 : 4], words[FAST ? 0 : 5], words[FAST ? 0 : 6],
+                                        words[FAST ? 0 : 7]);
+                }
             }
             // scales (and offsets): NB per thread, or one per G lanes
             if (G == 1 || (lane & (G - 1)) == 0) {

@@ -21,7 +21,7 @@ from . import build as _build
 # enumeration values (the library's interface convention)
 E2M1, E3M0, E2M3, E3M2, INT4 = 0, 1, 2, 3, 4
 E8M0, UE4M3, UE5M3 = 0, 1, 2
-FLOOR, CEIL, OAS, NEAREST = 0, 1, 2, 3
+FLOOR, CEIL, OAS, NEAREST, MSE = 0, 1, 2, 3, 4
 RTNE, RCEIL, SR = 0, 1, 2
 ROW, COL, TWO_D = 0, 1, 2
 BF16, FP32 = 0, 1
@@ -73,6 +73,8 @@ def lib():
         L.orc_dequantize.restype = C.c_int
         L.orc_pack.argtypes = [C.c_int, P, i64, i64, P]
         L.orc_unpack.argtypes = [C.c_int, P, i64, i64, P]
+        L.orc_pack_tc.argtypes = [C.c_int, P, i64, i64, P]
+        L.orc_unpack_tc.argtypes = [C.c_int, P, i64, i64, P]
         L.orc_packed_bytes.argtypes = [C.c_int, i64, i64]
         L.orc_packed_bytes.restype = i64
         L.orc_stats.argtypes = [P, P, i64, i64, C.c_int, C.c_int, P, P]
@@ -170,6 +172,22 @@ def pack(elem: int, codes: np.ndarray) -> np.ndarray:
     out = np.zeros(nbytes, np.uint8)
     lib().orc_pack(elem, _ptr(np.ascontiguousarray(codes)), rows, cols, _ptr(out))
     return out.reshape(rows, -1)
+
+
+def pack_tc(elem: int, codes: np.ndarray) -> np.ndarray:
+    """Codes in the tensor-core operand layout (FP6: 16 codes in 12 bytes + 4
+    zero bytes; FP4 as `pack`)."""
+    rows, cols = codes.shape
+    nbytes = lib().orc_packed_bytes(elem, rows, cols)
+    out = np.zeros(nbytes, np.uint8)
+    lib().orc_pack_tc(elem, _ptr(np.ascontiguousarray(codes)), rows, cols, _ptr(out))
+    return out.reshape(rows, -1)
+
+
+def unpack_tc(elem: int, packed: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    out = np.zeros((rows, cols), np.uint8)
+    lib().orc_unpack_tc(elem, _ptr(np.ascontiguousarray(packed)), rows, cols, _ptr(out))
+    return out
 
 
 def unpack(elem: int, packed: np.ndarray, rows: int, cols: int) -> np.ndarray:

@@ -50,7 +50,7 @@
 /* ------------------------------------------------------------------------ */
 enum { E_E2M1 = 0, E_E3M0 = 1, E_E2M3 = 2, E_E3M2 = 3, E_INT4 = 4 };
 enum { S_E8M0 = 0, S_UE4M3 = 1, S_UE5M3 = 2 };
-enum { R_FLOOR = 0, R_CEIL = 1, R_OAS = 2, R_NEAREST = 3 };
+enum { R_FLOOR = 0, R_CEIL = 1, R_OAS = 2, R_NEAREST = 3, R_MSE = 4 };
 enum { RD_RTNE = 0, RD_CEIL = 1, RD_SR = 2 };
 enum { AX_ROW = 0, AX_COL = 1, AX_2D = 2 };
 enum { DT_BF16 = 0, DT_FP32 = 1 };
@@ -459,6 +459,37 @@ static int pow2_exponent(const grid_t *g, int rule, float tau, float alpha)
     return k;
 }
 
+/* (READING) MSE-optimal power-of-two scale (a per-block MSE-min scale     */
+/* search, the third follow-up after the core path): among the E8M0         */
+/* exponents k_floor and k_floor + 1 (clamped), the one whose block of     */
+/* nearest-even element codes has the smaller squared error; ties keep     */
+/* k_floor.  The error of exponent k is 4^k sum (v_t - q_t)^2 with          */
+/* v_t = binary32(r_t 2^-k) and q_t its grid value, so the two sums are    */
+/* compared as S(k_floor) against 4 S(k_floor + 1), each accumulated in    */
+/* binary64 in element order (every term is exact there).                  */
+/* Pinned: brute force against an independent grid rounding (tests), and  */
+/* the closed forms of constant blocks.                                    */
+static int mse_exponent(const grid_t *g, int asym, const float *res, int L, float alpha)
+{
+    int kf = pow2_exponent(g, R_FLOOR, 0.0f, alpha);
+    int k0 = kf < -127 ? -127 : kf > 127 ? 127 : kf;
+    int k1 = kf + 1 < -127 ? -127 : kf + 1 > 127 ? 127 : kf + 1;
+    if (k0 == k1) return k0;
+    double sum[2];
+    for (int c = 0; c < 2; c++) {
+        float inv = pow2f(-(c ? k1 : k0));
+        double acc = 0.0;
+        for (int t = 0; t < L; t++) {
+            float v = res[t] * inv;
+            float q = decode_elem(g, asym, encode_elem(g, asym, RD_RTNE, v, 0u));
+            double d = (double)v - (double)q;
+            acc += d * d;
+        }
+        sum[c] = acc;
+    }
+    return (sum[0] <= 4.0 * sum[1]) ? k0 : k1;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Quantize                                                                 */
 /* ------------------------------------------------------------------------ */
@@ -603,7 +634,8 @@ int orc_quantize(const orc_cfg *cfg, const void *x, int dtype, int64_t rows, int
             if (nonfinite) { scode = 0xff; zero_block = 1; }
             else if (alpha == 0.0f) { scode = 0; zero_block = 1; }
             else {
-                int k = pow2_exponent(&g, cfg->rule, cfg->oas_tau, alpha);
+                int k = (cfg->rule == R_MSE) ? mse_exponent(&g, asym, res, L, alpha)
+                                             : pow2_exponent(&g, cfg->rule, cfg->oas_tau, alpha);
                 if (k < -127) k = -127;
                 if (k > 127) k = 127;
                 scode = (uint8_t)(k + 127);
@@ -681,6 +713,40 @@ void orc_pack(int elem, const uint8_t *codes, int64_t rows, int64_t cols, uint8_
         for (int64_t j = 0; j < cols / 2; j++) {
             uint8_t lo = codes[r * cols + 2 * j] & 0xf, hi = codes[r * cols + 2 * j + 1] & 0xf;
             packed[r * (cols / 2) + j] = (uint8_t)(lo | (hi << 4));
+        }
+}
+
+/* (READING) Tensor-core operand layout of FP6 codes (the library's
+ * sf_layout = 1): every 16 consecutive codes of a row are packed into 12
+ * bytes, code i at bits [6i, 6i + 6) of the little-endian 96-bit value,
+ * followed by 4 zero bytes; 16 bytes per 16 elements.  The layout CUDA's
+ * tensor-map documentation gives for 16 x U6 values in shared memory.  FP4
+ * codes keep their packing (two per byte). */
+void orc_pack_tc(int elem, const uint8_t *codes, int64_t rows, int64_t cols, uint8_t *packed)
+{
+    grid_t g; make_grid(elem, 0, &g);
+    if (g.bits != 6) { orc_pack(elem, codes, rows, cols, packed); return; }
+    for (int64_t i0 = 0; i0 < rows * cols; i0 += 16) {
+        uint8_t *dst = packed + i0;
+        memset(dst, 0, 16);
+        for (int i = 0; i < 16; i++) {
+            unsigned v = codes[i0 + i] & 0x3fu;
+            for (int b = 0; b < 6; b++)
+                if (v & (1u << b)) dst[(6 * i + b) / 8] |= (uint8_t)(1u << ((6 * i + b) % 8));
+        }
+    }
+}
+
+void orc_unpack_tc(int elem, const uint8_t *packed, int64_t rows, int64_t cols, uint8_t *codes)
+{
+    grid_t g; make_grid(elem, 0, &g);
+    if (g.bits != 6) { orc_unpack(elem, packed, rows, cols, codes); return; }
+    for (int64_t i0 = 0; i0 < rows * cols; i0 += 16)
+        for (int i = 0; i < 16; i++) {
+            unsigned v = 0;
+            for (int b = 0; b < 6; b++)
+                if (packed[i0 + (6 * i + b) / 8] & (1u << ((6 * i + b) % 8))) v |= 1u << b;
+            codes[i0 + i] = (uint8_t)v;
         }
 }
 

@@ -70,6 +70,10 @@ def test_query_sizes_host_only(mx):
     (dict(block=16), 64, 16, -1),                         # cols % 32 (lanes walk 32-element chunks)
     (dict(rule=2, oas_tau=float("nan")), 64, 64, -1),
     (dict(elem=9), 64, 64, -1),
+    (dict(rule=5), 64, 64, -1),
+    (dict(rule=4, block=16), 64, 64, -2),                 # MSE rule: blocks of 32 only
+    (dict(rule=4, round=2), 64, 64, -2),                  # ... and nearest-even rounding
+    (dict(rule=4, axis=1), 64, 64, -2),
 ])
 def test_invalid_configs_rejected_on_host(mx, cfg, rows, cols, rc):
     c = mx.Config(**cfg)

@@ -210,3 +210,65 @@ def test_mbs_gemm_scales_rejects_other_configs(mx):
     q = mx.quantize(x, mx.MXFP4, stats=False)
     with pytest.raises(ValueError):
         mx.mbs_gemm_operand(q)
+
+
+@pytest.mark.parametrize("ea,eb", [(2, 2), (3, 3), (2, 3)])
+@pytest.mark.parametrize("shape", [(128, 256, 256), (256, 512, 768), (384, 256, 1024)])
+def test_mxfp6_gemm(mx, orc, ea, eb, shape):
+    """MXFP6 operands (E2M3 / E3M2 codes, one per byte, E8M0 scales per 32) on
+    the tcgen05 kind::mxf8f6f4: C equals the binary64 product of the
+    oracle's dequantized operands (products of FP6 values and powers of two
+    are exact; FP32 accumulation)."""
+    M, N, K = shape
+    a = inputs.laplace_outlier_cols(M, K, seed=6, n_outlier_cols=2)
+    w = inputs.normal(N, K, sigma=0.02, seed=7)
+    ca, cw = mx.Config(elem=ea, sf_layout=1), mx.Config(elem=eb, sf_layout=1)
+    qa = mx.quantize(a.cuda(), ca, stats=False)
+    qw = mx.quantize(w.cuda(), cw, stats=False)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        c = mx.gemm(qa, qw, out_dtype=out_dtype)
+        torch.cuda.synchronize()
+        assert mx.mx_device_status() == 0
+        oa, ow = orc.Cfg(elem=ea), orc.Cfg(elem=eb)
+        ra, rw = orc.quantize(oa, a), orc.quantize(ow, w)
+        S = K // 32
+        assert np.array_equal(qa.scales.cpu().numpy(), chunk_layout(ra["scales"], M, S))
+        # codes in the tensor-core operand layout (16 codes in 12 bytes + 4 zero bytes)
+        assert np.array_equal(qa.codes.cpu().numpy(),
+                              orc.pack_tc(ea, orc.unpack(ea, ra["packed"], M, K)).ravel())
+        ah = orc.dequantize(oa, ra["packed"], ra["scales"], ra["tensor_scale"], None, None, M, K)
+        wh = orc.dequantize(ow, rw["packed"], rw["scales"], rw["tensor_scale"], None, None, N, K)
+        # the library's dequantizer reads the tensor-core layout back
+        xh = mx.dequantize(qa, torch.float32).cpu().numpy()
+        assert np.array_equal(xh.view(np.uint32), ah.view(np.uint32))
+        ref = ah.astype(np.float64) @ wh.astype(np.float64).T
+        got = c.float().cpu().numpy().astype(np.float64)
+        tol = 1e-3 if out_dtype == torch.float32 else 8e-3
+        assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < tol
+        rms = np.sqrt(np.mean(ref ** 2))
+        assert np.max(np.abs(got - ref)) <= tol * rms + tol * np.abs(ref).max() * (out_dtype != torch.float32)
+
+
+def test_mxfp6_gemm_qsnr(mx, orc):
+    M, N, K = 256, 256, 512
+    a = inputs.laplace_outlier_cols(M, K, seed=6, n_outlier_cols=2)
+    w = inputs.normal(N, K, sigma=0.02, seed=7)
+    cfg = mx.Config(elem=2, sf_layout=1)
+    qa = mx.quantize(a.cuda(), cfg, stats=False)
+    qw = mx.quantize(w.cuda(), cfg, stats=False)
+    st = mx.gemm_qsnr(a.cuda(), w.cuda(), qa, qw).cpu().numpy()
+    oc = orc.Cfg(elem=2)
+    ra, rw = orc.quantize(oc, a), orc.quantize(oc, w)
+    ah = orc.dequantize(oc, ra["packed"], ra["scales"], ra["tensor_scale"], None, None, M, K)
+    wh = orc.dequantize(oc, rw["packed"], rw["scales"], rw["tensor_scale"], None, None, N, K)
+    o = orc.gemm_qsnr(orc.input_f32(a), orc.input_f32(w), ah, wh)
+    assert abs(st[0] - o[0]) <= 1e-3 * o[0]
+    assert abs(st[1] - o[1]) <= 1e-3 * o[1]
+
+
+def test_mxfp6_gemm_needs_n_multiple_of_256(mx):
+    a = torch.zeros(128, 256, dtype=torch.bfloat16, device="cuda")
+    q = mx.quantize(a, mx.Config(elem=2, sf_layout=1), stats=False)
+    with pytest.raises(mx.MXError) as e:
+        mx.gemm(q, q)
+    assert e.value.code == -2

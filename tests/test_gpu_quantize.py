@@ -215,6 +215,27 @@ def test_general_quantizer_matrix(mx, orc, elem, rnd, asym, dtype):
 
 
 @pytest.mark.parametrize("elem", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_mse_rule(mx, orc, elem, dtype):
+    """MSE-optimal E8M0 scales (k_floor or k_floor + 1 per block, the smaller
+    nearest-even squared error): codes, scales and statistics against the
+    oracle on a ragged shape, with zero / NaN blocks planted."""
+    x = inputs.laplace_outlier_cols(72, 544, seed=4, n_outlier_cols=4, dtype=torch.float32)
+    x[3, 32:64] = 0.0
+    x[7, 100] = float("nan")
+    x = x.to(dtype)
+    run_case(mx, orc, x, mx.Config(elem=elem, rule=mx.RULE_MSE))
+
+
+def test_mse_rule_lowers_mse(mx):
+    """The MSE rule never leaves a larger tensor MSE than the floor rule."""
+    x = inputs.laplace_outlier_cols(512, 1024, seed=4).cuda()
+    a = mx.quantize(x, mx.Config(rule=mx.RULE_MSE)).stats.cpu().numpy()
+    b = mx.quantize(x, mx.Config(rule=mx.RULE_FLOOR)).stats.cpu().numpy()
+    assert a[5] <= b[5]
+
+
+@pytest.mark.parametrize("elem", [0, 1, 2, 3, 4])
 @pytest.mark.parametrize("rnd", [0, 1, 2])
 def test_general_grid_sweep(mx, orc, elem, rnd):
     """Scaled values swept densely across each grid (multiples of 2^-7, so every

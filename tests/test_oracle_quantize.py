@@ -382,3 +382,67 @@ def test_trend_small_block_inversion_ue4m3(orc):
     assert mse(orc.UE4M3, 8, orc.TS_NONE) > mse(orc.UE4M3, 16, orc.TS_NONE)
     assert mse(orc.UE5M3, 8, orc.TS_NONE) < mse(orc.UE5M3, 16, orc.TS_NONE)
     assert mse(orc.UE4M3, 8, orc.TS_COMPUTE) < mse(orc.UE4M3, 16, orc.TS_COMPUTE)
+
+
+def _grid(elem):
+    """Magnitude grids, built here from their definitions (independent of the
+    oracle's tables): E2M1 as printed on the page, the others from their
+    exponent / mantissa fields."""
+    if elem == 0:
+        return np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+    if elem == 1:
+        return np.array([0] + [2.0 ** (f - 3) for f in range(1, 8)], np.float64)
+    if elem in (2, 3):
+        mb, bias = (3, 1) if elem == 2 else (2, 3)
+        out = []
+        for c in range(32):
+            e, m = c >> mb, c & ((1 << mb) - 1)
+            out.append(m / 2.0 ** mb * 2.0 ** (1 - bias) if e == 0 else (1 + m / 2.0 ** mb) * 2.0 ** (e - bias))
+        return np.array(out, np.float64)
+    return np.arange(8, dtype=np.float64)
+
+
+def _sse_nearest(v, grid):
+    """Sum of (v - q)^2, q the nearest grid magnitude (ties to the even index,
+    saturating), by brute force over the grid, accumulated in element order."""
+    acc = 0.0
+    for x in v:
+        a = abs(float(x))
+        d = np.abs(grid - a)
+        best = np.flatnonzero(d == d.min())
+        i = best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
+        if a >= grid[-1]:
+            i = len(grid) - 1
+        acc += (a - grid[i]) ** 2
+    return acc
+
+
+@pytest.mark.parametrize("elem", [0, 1, 2, 3, 4])
+def test_mse_rule_brute_force(orc, elem):
+    """MSE-optimal scale: the chosen E8M0 exponent is the one of k_floor,
+    k_floor + 1 whose block squared error (in x units: 4^k sum) is smaller,
+    ties to k_floor, checked against a brute-force grid rounding."""
+    rng = np.random.default_rng(11 + elem)
+    grid = _grid(elem)
+    emax = {0: 2, 1: 4, 2: 2, 3: 4, 4: 2}[elem]
+    x = (rng.standard_normal((64, 32)) * np.exp(rng.uniform(-3, 3, (64, 1)))).astype(np.float32)
+    x[::7] *= 1.9                       # push some block maxima towards saturation
+    r = orc.quantize(orc.Cfg(elem=elem, rule=orc.MSE), torch.from_numpy(x))
+    for b in range(64):
+        v = x[b]
+        alpha = float(np.max(np.abs(v)))
+        kf = math.frexp(alpha)[1] - 1 - emax
+        sse = [_sse_nearest((v.astype(np.float32) * np.float32(2.0 ** -k)).astype(np.float32), grid)
+               for k in (kf, kf + 1)]
+        want = kf if sse[0] <= 4.0 * sse[1] else kf + 1
+        assert int(r["scales"][b]) == want + 127, (b, sse)
+
+
+def test_mse_rule_constant_blocks(orc):
+    """Closed forms for E2M1 constant blocks: 7.0 and 5.0 tie (error 1 either
+    way) and keep k_floor; 7.5 has error 1.5 at k_floor against 0.5 at
+    k_floor + 1 (3.75 rounds to 4, i.e. 8)."""
+    for val, k in ((7.0, 0), (5.0, 0), (7.5, 1), (6.0, 0)):
+        x = torch.full((1, 32), val, dtype=torch.float32)
+        r = orc.quantize(orc.Cfg(rule=orc.MSE), x)
+        assert int(r["scales"][0]) == 127 + k, (val, r["scales"][0])
