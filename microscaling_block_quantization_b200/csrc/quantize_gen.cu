@@ -219,17 +219,51 @@ __global__ void __launch_bounds__(kRingThreads, 2) k_quant_gen(const QParams p, 
             const BlockScale bs = (!ASYM && p.sd.rule == R_MSE && !bad && a > 0.0f)
                                       ? mse_block_scale<ELEM>(y, a, p.ed.emax)
                                       : block_scale(p.ed, p.sd, bad ? 0.0f : a, bad, sT);
-            const float2 inv2 = make_float2(bs.inv, bs.inv);
+            // a flushed block (x_hat = 0, or o with an offset; not NaN): the
+            // residuals are the (offset-removed) values themselves
+            const bool flushed = bs.zero && !bs.nan;
+            const float inv = flushed ? 1.0f : bs.inv;
+            const float2 inv2 = make_float2(inv, inv);
+            float deqT = bs.nan ? __uint_as_float(0x7fc00000u) : nearest ? __fmul_rn(bs.deq, sT) : bs.deq;
+            if (flushed) deqT = 1.0f;
 
-            // element codes and grid values
+            // element codes and grid values; the statistics on the scaled
+            // values: y - x_hat = deqT (v - q), exact for power-of-two scales
+            // without an offset, within an ulp of y otherwise
             uint32_t words[NW];
 #pragma unroll
             for (int w = 0; w < NW; ++w) words[w] = 0;
-            float q[32];
+            float2 re2 = make_float2(0.f, 0.f), rb2 = re2, sx2 = re2;
+            int qz = 0, xhz = 0;
+            const float2 m1 = make_float2(-1.0f, -1.0f);
+            // residual sums of one pair (v, q); q = 0 in a flushed block
+            auto pair_stats = [&](float2 v, float q0, float q1, float x0, float x1) {
+                if (bs.zero) { q0 = 0.0f; q1 = 0.0f; }
+                const float2 d = __ffma2_rn(make_float2(q0, q1), m1, v);
+                re2 = __ffma2_rn(d, d, re2);
+                rb2 = __fadd2_rn(rb2, d);
+                const float2 yv = make_float2(x0, x1);
+                sx2 = __ffma2_rn(yv, yv, sx2);
+                if (ASYM || nearest) {
+                    // x_hat exactly as the dequantizer forms it (zero test)
+                    float h0, h1;
+                    if (bs.nan) { h0 = h1 = __uint_as_float(0x7fc00000u); }
+                    else if (nearest) {
+                        h0 = __fmul_rn(__fmul_rn(q0, bs.deq), sT);
+                        h1 = __fmul_rn(__fmul_rn(q1, bs.deq), sT);
+                    } else {
+                        h0 = __fadd_rn(__fmul_rn(q0, bs.deq), o);
+                        h1 = __fadd_rn(__fmul_rn(q1, bs.deq), o);
+                    }
+                    xhz += (h0 == 0.0f && x0 != 0.0f) + (h1 == 0.0f && x1 != 0.0f);
+                } else {
+                    qz += (q0 == 0.0f) + (q1 == 0.0f);
+                }
+            };
             if constexpr (HW && ELEM == E2M1) {
 #pragma unroll
                 for (int j = 0; j < 32; j += 8) {
-                    float s8[8];
+                    float s8[8], q8[8];
 #pragma unroll
                     for (int e = 0; e < 8; e += 2) {
                         const float2 r = ASYM ? make_float2(__fsub_rn(y[j + e], o), __fsub_rn(y[j + e + 1], o))
@@ -239,7 +273,12 @@ __global__ void __launch_bounds__(kRingThreads, 2) k_quant_gen(const QParams p, 
                         s8[e + 1] = v.y;
                     }
                     words[j >> 3] = cvt_e2m1x8(s8);
-                    e2m1x8_values_alu(words[j >> 3], q + j);
+                    if (stats) {
+                        e2m1x8_values_alu(words[j >> 3], q8);
+#pragma unroll
+                        for (int e = 0; e < 8; e += 2)
+                            pair_stats(make_float2(s8[e], s8[e + 1]), q8[e], q8[e + 1], y[j + e], y[j + e + 1]);
+                    }
                 }
             } else {
                 uint4 rw = make_uint4(0, 0, 0, 0);
@@ -248,27 +287,25 @@ __global__ void __launch_bounds__(kRingThreads, 2) k_quant_gen(const QParams p, 
                     const float2 r = ASYM ? make_float2(__fsub_rn(y[j], o), __fsub_rn(y[j + 1], o))
                                           : make_float2(y[j], y[j + 1]);
                     const float2 v = __fmul2_rn(r, inv2);
+                    float2 qq;
                     if constexpr (HW) {
                         const uint32_t pair = ELEM == E2M3 ? cvt_e2m3x2(v.x, v.y) : cvt_e3m2x2(v.x, v.y);
-                        const float2 qq = ELEM == E2M3 ? e2m3x2_values(pair) : e3m2x2_values(pair);
-                        q[j] = qq.x;
-                        q[j + 1] = qq.y;
+                        if (stats) qq = ELEM == E2M3 ? e2m3x2_values(pair) : e3m2x2_values(pair);
                         words[j >> 2] |= pair << (8 * (j & 3));
                     } else {
                         if (RD == RD_SR && (j & 3) == 0) rw = element_words(p.seed, ((uint64_t)c * 32 + j) >> 2);
                         const uint32_t u0 = (j & 3) ? rw.z : rw.x, u1 = (j & 3) ? rw.w : rw.y;
-                        const uint32_t c0 = encode_grid<ELEM, RD, ASYM>(v.x, u0, q[j]);
-                        const uint32_t c1 = encode_grid<ELEM, RD, ASYM>(v.y, u1, q[j + 1]);
+                        const uint32_t c0 = encode_grid<ELEM, RD, ASYM>(v.x, u0, qq.x);
+                        const uint32_t c1 = encode_grid<ELEM, RD, ASYM>(v.y, u1, qq.y);
                         if constexpr (F::BITS == 4) words[j >> 3] |= (c0 | (c1 << 4)) << (4 * (j & 7));
                         else words[j >> 2] |= (c0 | (c1 << 8)) << (8 * (j & 3));
                     }
+                    if (stats) pair_stats(v, qq.x, qq.y, y[j], y[j + 1]);
                 }
             }
             if (bs.zero) {
 #pragma unroll
                 for (int w = 0; w < NW; ++w) words[w] = 0;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) q[j] = 0.0f;
             }
 
             if (ok) {
@@ -296,32 +333,18 @@ __global__ void __launch_bounds__(kRingThreads, 2) k_quant_gen(const QParams p, 
             }
 
             if (stats && ok) {
-                // dequantized values as the dequantizer forms them
-                float sx = 0.f, se = 0.f, sb = 0.f;
-                int z = 0, f = 0;
+                const double X = (double)deqT;
+                acc.e2 += (double)(re2.x + re2.y) * X * X;
+                acc.e -= (double)(rb2.x + rb2.y) * X;
+                acc.x2 += (double)(sx2.x + sx2.y);
+                // exact zeros (rare): the block's minimum magnitude is zero
+                int xz = 0;
+                if (absmin<32>(y) == 0.0f)
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float xv = y[j];
-                    float xh;
-                    if (bs.nan) xh = __uint_as_float(0x7fc00000u);
-                    else if (nearest) xh = __fmul_rn(__fmul_rn(q[j], bs.deq), sT);
-                    else {
-                        xh = __fmul_rn(q[j], bs.deq);
-                        if (ASYM) xh = __fadd_rn(xh, o);
-                    }
-                    const float d = __fsub_rn(xv, xh);
-                    sx = fmaf(xv, xv, sx);
-                    se = fmaf(d, d, se);
-                    sb -= d;
-                    const int nzj = xv != 0.0f;
-                    z += nzj;
-                    f += nzj & (xh == 0.0f);
-                }
-                acc.x2 += (double)sx;
-                acc.e2 += (double)se;
-                acc.e += (double)sb;
-                acc.nz += (double)z;
-                acc.ftz += (double)f;
+                    for (int j = 0; j < 32; ++j) xz += (y[j] == 0.0f);
+                acc.nz += (double)(32 - xz);
+                if (ASYM || nearest) acc.ftz += (double)xhz;
+                else if (!bs.nan) acc.ftz += (double)(qz - xz);
             }
         }
     }
