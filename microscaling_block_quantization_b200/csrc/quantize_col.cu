@@ -150,6 +150,157 @@ __device__ __forceinline__ void stage_block(const QParams &p, const LaneTile<CPT
     if constexpr (HAD) rotate_tile<AXIS>(t, p.had, RB, lane);
 }
 
+// E2M1 round-to-nearest-even, no macro scale or offset, on one staged RB-row
+// tile (lane's CPT columns at t): one statistic pass (NaN-propagating abs
+// max) and one encode pass with packed binary32 pairs; codes, scales and
+// the fidelity sums.
+template <int CPT, int AXIS>
+__device__ __forceinline__ void col_fast_tile(const QParams &p, const LaneTile<CPT> &t, int64_t r0, int64_t c0,
+                                              int RB, bool ok, int lane, float sT, bool stats, Acc &acc)
+{
+    constexpr int G2 = 32 / CPT;            // lanes of a 2D tile row
+        constexpr int NSF = (AXIS == AX_COL) ? CPT : 1;
+        float a[NSF], mabs[NSF];
+#pragma unroll
+        for (int s2 = 0; s2 < NSF; ++s2) { a[s2] = 0.0f; mabs[s2] = FLT_MAX; }
+        if constexpr (CPT == 8) {
+            // bf16 pairs straight from the tile: |x| by masking the
+            // sign bits, NaN-propagating max and min per column pair
+            __nv_bfloat162 am[4], mn[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                am[i] = __float2bfloat162_rn(0.0f);
+                mn[i] = __float2bfloat162_rn(__uint_as_float(0x7f800000u));
+            }
+            for (int r = 0; r < RB; ++r) {
+                const uint4 u = t.base[r * 32];
+                const uint32_t wv[4] = {u.x & 0x7fff7fffu, u.y & 0x7fff7fffu, u.z & 0x7fff7fffu,
+                                        u.w & 0x7fff7fffu};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&wv[i]);
+                    am[i] = __hmax2_nan(am[i], b);
+                    mn[i] = __hmin2(mn[i], b);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 fa = __bfloat1622float2(am[i]), fm = __bfloat1622float2(mn[i]);
+                const int s0 = (AXIS == AX_COL) ? 2 * i : 0, s1 = (AXIS == AX_COL) ? 2 * i + 1 : 0;
+                a[s0] = fmax_nan(a[s0], fa.x);
+                a[s1] = fmax_nan(a[s1], fa.y);
+                mabs[s0] = fminf(mabs[s0], fm.x);
+                mabs[s1] = fminf(mabs[s1], fm.y);
+            }
+        } else {
+            for (int r = 0; r < RB; ++r) {
+                float v[CPT];
+                t.get(r, v);
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) {
+                    const int s2 = (AXIS == AX_COL) ? j : 0;
+                    a[s2] = fmax_nan(a[s2], fabsf(v[j]));
+                    mabs[s2] = fminf(mabs[s2], fabsf(v[j]));
+                }
+            }
+        }
+        BlockScale bsf[NSF];
+#pragma unroll
+        for (int s2 = 0; s2 < NSF; ++s2) {
+            int bad = !(a[s2] <= FLT_MAX);
+            float aa = bad ? 0.0f : a[s2];
+            if (AXIS == AX_2D) {
+                aa = grp_max(aa, G2);
+                bad = grp_or(bad, G2);
+                mabs[s2] = grp_min(mabs[s2], G2);
+            }
+            bsf[s2] = block_scale(p.ed, p.sd, aa, bad, sT);
+        }
+        if (ok) {
+            if (AXIS == AX_COL) {
+                uint8_t *dst = p.scales + (r0 / RB) * p.cols + c0;
+                uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+                for (int j = 0; j < CPT; ++j) {
+                    if (j < 4) w0 |= bsf[(AXIS == AX_COL) ? j : 0].code << (8 * j);
+                    else w1 |= bsf[(AXIS == AX_COL) ? j : 0].code << (8 * (j - 4));
+                }
+                if constexpr (CPT == 8) *reinterpret_cast<uint2 *>(dst) = make_uint2(w0, w1);
+                else *reinterpret_cast<uint32_t *>(dst) = w0;
+            } else if ((lane & (G2 - 1)) == 0) {
+                p.scales[(r0 / 32) * (p.cols / 32) + c0 / 32] = (uint8_t)bsf[0].code;
+            }
+        }
+        const bool nearest = p.sd.fmt != S_E8M0 && p.sd.rule == R_NEAREST;
+        float deqT[NSF];
+#pragma unroll
+        for (int s2 = 0; s2 < NSF; ++s2)
+            deqT[s2] = bsf[s2].nan ? __uint_as_float(0x7fc00000u)
+                     : nearest ? __fmul_rn(bsf[s2].deq, sT) : bsf[s2].deq;
+        float2 sx2 = make_float2(0.f, 0.f), se2 = sx2, sb2 = sx2;
+        int qz = 0;                      // zero-magnitude codes of the lane
+        for (int r = 0; r < RB; ++r) {
+            const int64_t e0 = (r0 + r) * p.cols + c0;
+            float v[CPT];
+            t.get(r, v);
+            float s8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+            for (int j = 0; j < CPT; j += 2) {
+                const int sa = (AXIS == AX_COL) ? j : 0, sb_ = (AXIS == AX_COL) ? j + 1 : 0;
+                const float2 pr = __fmul2_rn(make_float2(v[j], v[j + 1]),
+                                             make_float2(bsf[sa].inv, bsf[sb_].inv));
+                s8[j] = bsf[sa].zero ? 0.0f : pr.x;
+                s8[j + 1] = bsf[sb_].zero ? 0.0f : pr.y;
+            }
+            uint32_t lo = cvt_e2m1x8(s8);
+            if (CPT == 4) lo &= 0xffffu;
+            if (ok) {
+                uint8_t *dst = static_cast<uint8_t *>(p.codes) + e0 / 2;
+                if constexpr (CPT == 8) *reinterpret_cast<uint32_t *>(dst) = lo;
+                else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)lo;
+            }
+            if (stats && ok) {
+                float q[8];
+                e2m1x8_values_alu(lo, q);
+#pragma unroll
+                for (int j = 0; j < CPT; j += 2) {
+                    const int sa = (AXIS == AX_COL) ? j : 0, sb_ = (AXIS == AX_COL) ? j + 1 : 0;
+                    const float2 yv = make_float2(v[j], v[j + 1]);
+                    const float2 d = __ffma2_rn(make_float2(q[j], q[j + 1]),
+                                                make_float2(-deqT[sa], -deqT[sb_]), yv);
+                    se2 = __ffma2_rn(d, d, se2);
+                    sx2 = __ffma2_rn(yv, yv, sx2);
+                    sb2 = __fadd2_rn(sb2, d);
+                }
+                qz += e2m1_zero_codes8(lo) - (8 - CPT);
+            }
+        }
+        if (stats && ok) {
+            acc.x2 += (double)(sx2.x + sx2.y);
+            acc.e2 += (double)(se2.x + se2.y);
+            acc.e += -(double)(sb2.x + sb2.y);
+            // flushed = zero codes - exact zeros, NaN blocks (all codes
+            // zero) left out
+            int ftz = qz;
+#pragma unroll
+            for (int s2 = 0; s2 < NSF; ++s2) {
+                int xz = 0;
+                if (mabs[s2] == 0.0f)
+                    for (int r = 0; r < RB; ++r) {
+                        float v[CPT];
+                        t.get(r, v);
+#pragma unroll
+                        for (int j = 0; j < CPT; ++j)
+                            if ((AXIS == AX_COL) ? j == s2 : true) xz += (v[j] == 0.0f);
+                    }
+                const int n_lane = (AXIS == AX_COL) ? RB : RB * CPT;
+                acc.nz += (double)(n_lane - xz);
+                ftz -= bsf[s2].nan ? n_lane : xz;
+            }
+            acc.ftz += (double)ftz;
+        }
+}
+
 template <typename InT, int CPT, int AXIS, bool FAST, bool HAD>
 __global__ void __launch_bounds__(kColThreads) k_quant_col(const QParams p)
 {
@@ -237,146 +388,7 @@ __global__ void __launch_bounds__(kColThreads) k_quant_col(const QParams p)
             // packed binary32 pairs
             if constexpr (FAST) {
                 if (!p.mbs) {
-                    constexpr int NSF = (AXIS == AX_COL) ? CPT : 1;
-                    float a[NSF], mabs[NSF];
-#pragma unroll
-                    for (int s2 = 0; s2 < NSF; ++s2) { a[s2] = 0.0f; mabs[s2] = FLT_MAX; }
-                    if constexpr (CPT == 8) {
-                        // bf16 pairs straight from the tile: |x| by masking the
-                        // sign bits, NaN-propagating max and min per column pair
-                        __nv_bfloat162 am[4], mn[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            am[i] = __float2bfloat162_rn(0.0f);
-                            mn[i] = __float2bfloat162_rn(__uint_as_float(0x7f800000u));
-                        }
-                        for (int r = 0; r < RB; ++r) {
-                            const uint4 u = t.base[r * 32];
-                            const uint32_t wv[4] = {u.x & 0x7fff7fffu, u.y & 0x7fff7fffu, u.z & 0x7fff7fffu,
-                                                    u.w & 0x7fff7fffu};
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&wv[i]);
-                                am[i] = __hmax2_nan(am[i], b);
-                                mn[i] = __hmin2(mn[i], b);
-                            }
-                        }
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float2 fa = __bfloat1622float2(am[i]), fm = __bfloat1622float2(mn[i]);
-                            const int s0 = (AXIS == AX_COL) ? 2 * i : 0, s1 = (AXIS == AX_COL) ? 2 * i + 1 : 0;
-                            a[s0] = fmax_nan(a[s0], fa.x);
-                            a[s1] = fmax_nan(a[s1], fa.y);
-                            mabs[s0] = fminf(mabs[s0], fm.x);
-                            mabs[s1] = fminf(mabs[s1], fm.y);
-                        }
-                    } else {
-                        for (int r = 0; r < RB; ++r) {
-                            float v[CPT];
-                            t.get(r, v);
-#pragma unroll
-                            for (int j = 0; j < CPT; ++j) {
-                                const int s2 = (AXIS == AX_COL) ? j : 0;
-                                a[s2] = fmax_nan(a[s2], fabsf(v[j]));
-                                mabs[s2] = fminf(mabs[s2], fabsf(v[j]));
-                            }
-                        }
-                    }
-                    BlockScale bsf[NSF];
-#pragma unroll
-                    for (int s2 = 0; s2 < NSF; ++s2) {
-                        int bad = !(a[s2] <= FLT_MAX);
-                        float aa = bad ? 0.0f : a[s2];
-                        if (AXIS == AX_2D) {
-                            aa = grp_max(aa, G2);
-                            bad = grp_or(bad, G2);
-                            mabs[s2] = grp_min(mabs[s2], G2);
-                        }
-                        bsf[s2] = block_scale(p.ed, p.sd, aa, bad, sT);
-                    }
-                    if (ok) {
-                        if (AXIS == AX_COL) {
-                            uint8_t *dst = p.scales + (r0 / RB) * p.cols + c0;
-                            uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-                            for (int j = 0; j < CPT; ++j) {
-                                if (j < 4) w0 |= bsf[(AXIS == AX_COL) ? j : 0].code << (8 * j);
-                                else w1 |= bsf[(AXIS == AX_COL) ? j : 0].code << (8 * (j - 4));
-                            }
-                            if constexpr (CPT == 8) *reinterpret_cast<uint2 *>(dst) = make_uint2(w0, w1);
-                            else *reinterpret_cast<uint32_t *>(dst) = w0;
-                        } else if ((lane & (G2 - 1)) == 0) {
-                            p.scales[(r0 / 32) * (p.cols / 32) + c0 / 32] = (uint8_t)bsf[0].code;
-                        }
-                    }
-                    const bool nearest = p.sd.fmt != S_E8M0 && p.sd.rule == R_NEAREST;
-                    float deqT[NSF];
-#pragma unroll
-                    for (int s2 = 0; s2 < NSF; ++s2)
-                        deqT[s2] = bsf[s2].nan ? __uint_as_float(0x7fc00000u)
-                                 : nearest ? __fmul_rn(bsf[s2].deq, sT) : bsf[s2].deq;
-                    float2 sx2 = make_float2(0.f, 0.f), se2 = sx2, sb2 = sx2;
-                    int qz = 0;                      // zero-magnitude codes of the lane
-                    for (int r = 0; r < RB; ++r) {
-                        const int64_t e0 = (r0 + r) * p.cols + c0;
-                        float v[CPT];
-                        t.get(r, v);
-                        float s8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll
-                        for (int j = 0; j < CPT; j += 2) {
-                            const int sa = (AXIS == AX_COL) ? j : 0, sb_ = (AXIS == AX_COL) ? j + 1 : 0;
-                            const float2 pr = __fmul2_rn(make_float2(v[j], v[j + 1]),
-                                                         make_float2(bsf[sa].inv, bsf[sb_].inv));
-                            s8[j] = bsf[sa].zero ? 0.0f : pr.x;
-                            s8[j + 1] = bsf[sb_].zero ? 0.0f : pr.y;
-                        }
-                        uint32_t lo = cvt_e2m1x8(s8);
-                        if (CPT == 4) lo &= 0xffffu;
-                        if (ok) {
-                            uint8_t *dst = static_cast<uint8_t *>(p.codes) + e0 / 2;
-                            if constexpr (CPT == 8) *reinterpret_cast<uint32_t *>(dst) = lo;
-                            else *reinterpret_cast<uint16_t *>(dst) = (uint16_t)lo;
-                        }
-                        if (stats && ok) {
-                            float q[8];
-                            e2m1x8_values_alu(lo, q);
-#pragma unroll
-                            for (int j = 0; j < CPT; j += 2) {
-                                const int sa = (AXIS == AX_COL) ? j : 0, sb_ = (AXIS == AX_COL) ? j + 1 : 0;
-                                const float2 yv = make_float2(v[j], v[j + 1]);
-                                const float2 d = __ffma2_rn(make_float2(q[j], q[j + 1]),
-                                                            make_float2(-deqT[sa], -deqT[sb_]), yv);
-                                se2 = __ffma2_rn(d, d, se2);
-                                sx2 = __ffma2_rn(yv, yv, sx2);
-                                sb2 = __fadd2_rn(sb2, d);
-                            }
-                            qz += e2m1_zero_codes8(lo) - (8 - CPT);
-                        }
-                    }
-                    if (stats && ok) {
-                        acc.x2 += (double)(sx2.x + sx2.y);
-                        acc.e2 += (double)(se2.x + se2.y);
-                        acc.e += -(double)(sb2.x + sb2.y);
-                        // flushed = zero codes - exact zeros, NaN blocks (all codes
-                        // zero) left out
-                        int ftz = qz;
-#pragma unroll
-                        for (int s2 = 0; s2 < NSF; ++s2) {
-                            int xz = 0;
-                            if (mabs[s2] == 0.0f)
-                                for (int r = 0; r < RB; ++r) {
-                                    float v[CPT];
-                                    t.get(r, v);
-#pragma unroll
-                                    for (int j = 0; j < CPT; ++j)
-                                        if ((AXIS == AX_COL) ? j == s2 : true) xz += (v[j] == 0.0f);
-                                }
-                            const int n_lane = (AXIS == AX_COL) ? RB : RB * CPT;
-                            acc.nz += (double)(n_lane - xz);
-                            ftz -= bsf[s2].nan ? n_lane : xz;
-                        }
-                        acc.ftz += (double)ftz;
-                    }
+                    col_fast_tile<CPT, AXIS>(p, t, r0, c0, RB, ok, lane, sT, stats, acc);
                     continue;
                 }
             }

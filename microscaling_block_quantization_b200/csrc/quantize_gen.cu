@@ -33,9 +33,7 @@ template <> struct GFmt<E2M3> { static constexpr int M = 3, EMIN = 0, MAXC = 31,
 template <> struct GFmt<E3M2> { static constexpr int M = 2, EMIN = -2, MAXC = 31, BITS = 6; static constexpr bool INT = false; };
 template <> struct GFmt<INT4> { static constexpr int M = 0, EMIN = 0, MAXC = 7, BITS = 4; static constexpr bool INT = true; };
 
-// largest magnitude and its code (INT4 with an offset: unsigned 0..15)
-template <int ELEM, bool ASYM>
-__device__ __forceinline__ constexpr int max_code() { return (GFmt<ELEM>::INT && ASYM) ? 15 : GFmt<ELEM>::MAXC; }
+// largest magnitude (INT4 with an offset: unsigned 0..15)
 template <int ELEM, bool ASYM>
 __device__ __forceinline__ float max_value()
 {
@@ -52,8 +50,10 @@ template <int ELEM, int RD, bool ASYM>
 __device__ __forceinline__ uint32_t round_grid(float a, uint32_t u, float &qm)
 {
     using F = GFmt<ELEM>;
-    const float maxv = max_value<ELEM, ASYM>();
-    if (!(a < maxv)) { qm = maxv; return (uint32_t)max_code<ELEM, ASYM>(); }
+    // saturation without a branch: the maximum is a grid point, so a clamped
+    // magnitude lands on it with a zero remainder under every mode (NaN and
+    // +inf clamp to it as well)
+    a = fminf(a, max_value<ELEM, ASYM>());
     float sc = 1.0f, isc = 1.0f;
     int cbase = 0;
     if constexpr (!F::INT) {
@@ -90,8 +90,7 @@ __device__ __forceinline__ uint32_t encode_grid(float v, uint32_t u, float &q)
 {
     using F = GFmt<ELEM>;
     if constexpr (F::INT && ASYM) {
-        if (!(v > 0.0f)) { q = 0.0f; return 0u; }
-        return round_grid<ELEM, RD, ASYM>(v, u, q);
+        return round_grid<ELEM, RD, ASYM>(fmaxf(v, 0.0f), u, q);      // negatives (and NaN) -> 0
     } else {
         const uint32_t neg = __float_as_uint(v) >> 31;
         float m;
