@@ -259,8 +259,15 @@ int mx_qsnr(const void *x, int32_t x_dtype, const void *x_hat, int32_t x_hat_dty
  * MXFP4: block 32, E8M0 (ca/cb rule FLOOR, CEIL or OAS).  NVFP4: block 16,
  * UE4M3 NEAREST with tensor scales tsA/tsB (device floats; used when
  * ca/cb->tensor_scale != MX_TS_NONE, else 1).  MXFP6 ([MX-TRAIN]'s MX6;
- * tcgen05 kind::mxf8f6f4): E2M3 and / or E3M2 codes, one per byte as
- * mx_quantize writes them, block 32, E8M0; N % 256 == 0.  C: device, bf16 or fp32
+ * tcgen05 kind::mxf8f6f4): E2M3 and / or E3M2 codes in the tensor-core
+ * operand layout mx_quantize writes with sf_layout = 1 (16 codes in 12 bytes
+ * + 4 zero bytes), block 32, E8M0; N % 256 == 0.  The same kind takes one
+ * FP6 operand with one MXFP4 operand (E2M1 + E8M0 / 32, packed codes; the
+ * packed operand's pointer 32-byte aligned): [MX-TRAIN]'s MX6 weights and
+ * activations against MX4 gradients.  Operands rotated by mx_hadamard_quantize
+ * are accepted when both carry the same rotation (cfg->hadamard), since
+ * (A H)(B H)^T = A B^T ([BRIDGING] sec. 2.3: rotated operands into the FP4
+ * GEMM).  Any other pair: MX_ERR_UNSUPPORTED.  C: device, bf16 or fp32
  * (c_dtype), row-major M x N.  M % 128 == 0, N % 128 == 0, K % 256 == 0.
  * Tiles: 128 x 256 per SM (persistent) when N % 256 == 0, else 128 x 128.
  */

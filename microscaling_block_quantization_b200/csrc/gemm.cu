@@ -39,6 +39,7 @@ constexpr int kTileBytes = BM * 128;              // one operand tile: 128 rows 
 constexpr uint64_t kWaitNs = 2000000000ull;       // bound of one mbarrier wait: 2 s
 
 enum { KIND_BF16 = 0, KIND_MXF4 = 1, KIND_NVF4 = 2, KIND_MXF6 = 3 };
+constexpr uint32_t kFmtE2M1 = 5;     // E2M1 in the kind::mxf8f6f4 instruction descriptor
 enum { EPI_BF16 = 0, EPI_F32 = 1, EPI_QSNR = 2 };
 
 // device status word of the bounded waits (read and cleared by mx_device_status)
@@ -52,6 +53,7 @@ struct GParams {
     const float *Cq;             // EPI_QSNR: the quantized product, fp32 M x N
     double *partials;            // EPI_QSNR: per-CTA [sum C^2, sum (C - Cq)^2]
     uint32_t ab_fmt;             // KIND_MXF6: A / B element formats of the instruction descriptor
+    uint32_t stage_tx;           // KIND_MXF6: bytes the TMA brings per stage (A, B and scales)
 };
 
 template <int KIND>
@@ -403,6 +405,9 @@ struct KindP {
     // 4-scale chunks per stage: a stage is 128 bytes of every row, K = 256
     // E2M1 elements (MXF4: 8 blocks of 32, NVF4: 16 of 16) or K = 128 FP6
     // elements in byte containers (MXF6: 4 blocks of 32)
+    // (an E2M1 operand of kind::mxf8f6f4 also takes one byte per element in
+    // shared memory: the TMA expands each 8-byte group of 16 packed codes to
+    // 16 bytes, the upper 8 left zero)
     static constexpr int kChunks = KIND == KIND_MXF4 ? 2 : KIND == KIND_MXF6 ? 1 : 4;
     static constexpr int kSfaBytes = kChunks * 512;                  // 128 rows of A
     static constexpr int kSfbBytes = 2 * kChunks * 512;              // 256 rows of B
@@ -475,7 +480,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                 for (int kt = 0; kt < ktiles; ++kt, ++it) {
                     const int s = it % kStagesP;
                     if (it >= (uint32_t)kStagesP && !mbar_wait(&empty[s], ((it / kStagesP) - 1) & 1, 11)) { ok = false; break; }
-                    mbar_expect_tx(&full[s], KT::kStageBytes);
+                    mbar_expect_tx(&full[s], KIND == KIND_MXF6 ? p.stage_tx : (uint32_t)KT::kStageBytes);
                     tma_load_2d(sA + s * KT::kABytes, &tmA, &full[s], kt * 128, m0);
                     tma_load_2d(sB + s * KT::kBBytes, &tmB, &full[s], kt * 128, n0);
                     const size_t ca = ((size_t)(m0 / 128) * sf_chunks_row + (size_t)kt * KT::kChunks) * 512;
@@ -648,6 +653,18 @@ bool make_map(CUtensorMap *m, const void *base, int rows, int K, int elem_bits, 
 {
     EncodeTiled enc = encoder();
     if (!enc) return false;
+    if (elem_bits == -4) {
+        // packed E2M1 codes read for kind::mxf8f6f4: boxes of 128 elements
+        // (64 bytes) land as 128 bytes in shared memory, every 8 bytes of codes
+        // followed by 8 zero bytes
+        const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+        const cuuint64_t strides[1] = {(cuuint64_t)K / 2};
+        const cuuint32_t box[2] = {128u, box_rows};
+        const cuuint32_t estr[2] = {1, 1};
+        return enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    }
     const bool bf16 = elem_bits == 16;
     const cuuint64_t row_bytes = (cuuint64_t)K * elem_bits / 8;
     const cuuint64_t inner = bf16 ? (cuuint64_t)K : row_bytes;
@@ -686,9 +703,18 @@ template <int KIND, int EPI>
 int launch_p(const GParams &p, const void *A, const void *B, cudaStream_t st)
 {
     CUtensorMap ta, tb;
-    const int bits = KIND == KIND_MXF6 ? 8 : 4;
-    if (!make_map(&ta, A, p.M, p.K, bits, 128) || !make_map(&tb, B, p.N, p.K, bits, 256)) return MX_ERR_CUDA;
     using KT = KindP<KIND>;
+    int abits = 4, bbits = 4;
+    GParams q = p;
+    if (KIND == KIND_MXF6) {
+        // per operand: FP6 codes one per byte, or packed E2M1 expanded by the TMA
+        const bool a4 = ((p.ab_fmt >> 7) & 7u) == kFmtE2M1, b4 = ((p.ab_fmt >> 10) & 7u) == kFmtE2M1;
+        abits = a4 ? -4 : 8;
+        bbits = b4 ? -4 : 8;
+        q.stage_tx = (uint32_t)((a4 ? KT::kABytes / 2 : KT::kABytes) + (b4 ? KT::kBBytes / 2 : KT::kBBytes) +
+                                KT::kSfaBytes + KT::kSfbBytes);
+    }
+    if (!make_map(&ta, A, p.M, p.K, abits, 128) || !make_map(&tb, B, p.N, p.K, bbits, 256)) return MX_ERR_CUDA;
     const int smem = 1024 + kStagesP * KT::kStageBytes + 256;
     auto k = k_gemm_p<KIND, EPI>;
     static bool attr = false;
@@ -700,7 +726,7 @@ int launch_p(const GParams &p, const void *A, const void *B, cudaStream_t st)
     const int tiles = (p.M / BM) * (p.N / BNP);
     int grid = mxk::device_sm_count();
     if (grid > tiles) grid = tiles;
-    k<<<grid, kThreadsP, smem, st>>>(p, ta, tb);
+    k<<<grid, kThreadsP, smem, st>>>(q, ta, tb);
     return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
 
@@ -709,13 +735,18 @@ int launch_p(const GParams &p, const void *A, const void *B, cudaStream_t st)
 int fp4_kind(const mx_config *a, const mx_config *b)
 {
     if (!a || !b) return -1;
+    // rotated operands are accepted when both carry the same rotation along
+    // K: (A H)(B H)^T = A B^T for the orthonormal block Hadamard H
     auto layout = [](const mx_config *c) {
-        return c->axis == MX_AXIS_ROW && c->sf_layout == 1 && !c->asymmetric && !c->macro_block && !c->hadamard;
+        return c->axis == MX_AXIS_ROW && c->sf_layout == 1 && !c->asymmetric && !c->macro_block;
     };
-    if (!layout(a) || !layout(b)) return -1;
+    if (!layout(a) || !layout(b) || a->hadamard != b->hadamard) return -1;
     auto fp6 = [](const mx_config *c) { return c->elem == MX_E2M3 || c->elem == MX_E3M2; };
-    if (fp6(a) && fp6(b)) {
-        if (a->scale_fmt == MX_SCALE_E8M0 && b->scale_fmt == MX_SCALE_E8M0 && a->block == 32 && b->block == 32)
+    if (fp6(a) || fp6(b)) {
+        // kind::mxf8f6f4: FP6 x FP6, or FP6 with an E2M1 operand (E8M0, blocks of 32)
+        const bool elems = (fp6(a) || a->elem == MX_E2M1) && (fp6(b) || b->elem == MX_E2M1);
+        if (elems && a->scale_fmt == MX_SCALE_E8M0 && b->scale_fmt == MX_SCALE_E8M0 && a->block == 32 &&
+            b->block == 32)
             return KIND_MXF6;
         return -1;
     }
@@ -728,11 +759,12 @@ int fp4_kind(const mx_config *a, const mx_config *b)
     return -1;
 }
 
-// kind::mxf8f6f4 operand formats (instruction descriptor bits 7-9 and 10-12)
+// kind::mxf8f6f4 operand formats (instruction descriptor bits 7-9 and 10-12):
+// E2M3 = 3, E3M2 = 4, E2M1 = 5
 uint32_t fp6_formats(const mx_config *a, const mx_config *b)
 {
-    const uint32_t fa = a->elem == MX_E2M3 ? 3u : 4u, fb = b->elem == MX_E2M3 ? 3u : 4u;
-    return (fa << 7) | (fb << 10);
+    auto f = [](const mx_config *c) { return c->elem == MX_E2M3 ? 3u : c->elem == MX_E3M2 ? 4u : kFmtE2M1; };
+    return (f(a) << 7) | (f(b) << 10);
 }
 
 bool shapes_ok(int64_t M, int64_t N, int64_t K)
@@ -782,8 +814,11 @@ int mx_gemm(const mx_config *ca, const mx_config *cb, const void *Aq, const uint
     p.C = C;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (kind == KIND_MXF6) {
-        // MXFP6: the persistent 128 x 256 kernel only
+        // MXFP6 (and FP6 x E2M1): the persistent 128 x 256 kernel only
         if (N % BNP) return MX_ERR_UNSUPPORTED;
+        // the expanding TMA form wants 32-byte aligned packed E2M1 operands
+        if ((ca->elem == MX_E2M1 && ((uintptr_t)Aq & 31u)) || (cb->elem == MX_E2M1 && ((uintptr_t)Bq & 31u)))
+            return MX_ERR_ALIGN;
         p.ab_fmt = fp6_formats(ca, cb);
         return c_dtype == MX_DT_BF16 ? launch_p<KIND_MXF6, EPI_BF16>(p, Aq, Bq, st)
                                      : launch_p<KIND_MXF6, EPI_F32>(p, Aq, Bq, st);

@@ -101,6 +101,23 @@ def test_alignment_and_workspace_rejected_on_host(mx):
                                    None) == -2
 
 
+def test_gemm_operand_pairs_checked_on_host(mx):
+    """mx_gemm rejects operand pairs it has no tensor-core kind for, and the
+    misaligned packed E2M1 operand of the FP6 x FP4 kind, before any launch."""
+    P = C.c_void_p
+    def gemm(ca, cb, a=4096, b=4096, M=128, N=256, K=256):
+        return mx.mx_gemm(ca, cb, P(a), P(4096), P(b), P(4096), None, None, M, N, K, P(4096), 1, None)
+    g = dict(sf_layout=1)
+    assert gemm(mx.Config(hadamard=32, **g), mx.Config(**g)) == -2         # rotation on one side only
+    assert gemm(mx.Config(hadamard=16, **g), mx.Config(hadamard=32, **g)) == -2
+    assert gemm(mx.Config(elem=2, **g), mx.Config(elem=4, **g)) == -2       # FP6 x INT4
+    nv = mx.Config(block=16, scale_fmt=mx.SCALE_UE4M3, rule=mx.RULE_NEAREST, tensor_scale=mx.TS_COMPUTE, **g)
+    assert gemm(mx.Config(elem=2, **g), nv) == -2                           # FP6 x NVFP4
+    assert gemm(mx.Config(elem=2, **g), mx.Config(**g), b=4112) == -3       # packed E2M1 wants 32 bytes
+    assert gemm(mx.Config(elem=2, **g), mx.Config(**g), N=128) == -2        # FP6 kinds: N % 256
+    assert gemm(mx.Config(**g), mx.Config(**g), K=128) == -1                # K % 256
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     import microscaling_block_quantization_b200 as m
     monkeypatch.setattr(m, "_lib", None)

@@ -249,6 +249,76 @@ def test_mxfp6_gemm(mx, orc, ea, eb, shape):
         assert np.max(np.abs(got - ref)) <= tol * rms + tol * np.abs(ref).max() * (out_dtype != torch.float32)
 
 
+@pytest.mark.parametrize("ea,eb", [(2, 0), (0, 3), (3, 0), (0, 2)])
+@pytest.mark.parametrize("shape", [(128, 256, 256), (256, 512, 768)])
+def test_fp6_fp4_mixed_gemm(mx, orc, ea, eb, shape):
+    """One FP6 operand (E2M3 / E3M2) and one MXFP4 operand (packed E2M1) on
+    kind::mxf8f6f4, the MX6 weight / activation with MX4 gradient pairing of
+    MX training: the packed E2M1 codes are expanded by the TMA to the
+    kind's one-byte-per-element shared-memory form.  C equals the binary64
+    product of the oracle's dequantized operands within FP32 accumulation."""
+    M, N, K = shape
+    a = inputs.laplace_outlier_cols(M, K, seed=6, n_outlier_cols=2)
+    w = inputs.normal(N, K, sigma=0.02, seed=7)
+    ca, cw = mx.Config(elem=ea, sf_layout=1), mx.Config(elem=eb, sf_layout=1)
+    qa = mx.quantize(a.cuda(), ca, stats=False)
+    qw = mx.quantize(w.cuda(), cw, stats=False)
+    oa, ow = orc.Cfg(elem=ea), orc.Cfg(elem=eb)
+    ra, rw = orc.quantize(oa, a), orc.quantize(ow, w)
+    ah = orc.dequantize(oa, ra["packed"], ra["scales"], ra["tensor_scale"], None, None, M, K)
+    wh = orc.dequantize(ow, rw["packed"], rw["scales"], rw["tensor_scale"], None, None, N, K)
+    ref = ah.astype(np.float64) @ wh.astype(np.float64).T
+    for out_dtype in (torch.float32, torch.bfloat16):
+        c = mx.gemm(qa, qw, out_dtype=out_dtype)
+        torch.cuda.synchronize()
+        assert mx.mx_device_status() == 0
+        got = c.float().cpu().numpy().astype(np.float64)
+        tol = 1e-3 if out_dtype == torch.float32 else 8e-3
+        assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < tol
+        rms = np.sqrt(np.mean(ref ** 2))
+        assert np.max(np.abs(got - ref)) <= tol * rms + tol * np.abs(ref).max() * (out_dtype != torch.float32)
+
+
+@pytest.mark.parametrize("had", [16, 32])
+@pytest.mark.parametrize("elem", [0, 2])
+def test_rotated_operand_gemm(mx, orc, had, elem):
+    """Both operands rotated by the same block Hadamard along K, quantized and
+    multiplied: (A H)(W H)^T = A W^T.  The GEMM equals the binary64 product of
+    the oracle's dequantized rotated operands, and its QSNR against A W^T
+    beats the unrotated MXFP4 product on outlier-column activations."""
+    M, N, K = 256, 256, 512
+    a = inputs.laplace_outlier_cols(M, K, seed=6, n_outlier_cols=2)
+    w = inputs.normal(N, K, sigma=0.02, seed=7)
+    cfg = mx.Config(elem=elem, hadamard=had, sf_layout=1)
+    qa = mx.quantize(a.cuda(), cfg, stats=False)
+    qw = mx.quantize(w.cuda(), cfg, stats=False)
+    c = mx.gemm(qa, qw, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert mx.mx_device_status() == 0
+    oc = orc.Cfg(elem=elem, hadamard=had)
+    ra, rw = orc.quantize(oc, a), orc.quantize(oc, w)
+    ah = orc.dequantize(oc, ra["packed"], ra["scales"], ra["tensor_scale"], None, None, M, K)
+    wh = orc.dequantize(oc, rw["packed"], rw["scales"], rw["tensor_scale"], None, None, N, K)
+    ref = ah.astype(np.float64) @ wh.astype(np.float64).T
+    got = c.cpu().numpy().astype(np.float64)
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < 1e-3
+    exact = orc.input_f32(a).astype(np.float64) @ orc.input_f32(w).astype(np.float64).T
+    if elem == 0:
+        q0 = mx.quantize(a.cuda(), mx.Config(sf_layout=1), stats=False)
+        w0 = mx.quantize(w.cuda(), mx.Config(sf_layout=1), stats=False)
+        c0 = mx.gemm(q0, w0, out_dtype=torch.float32).cpu().numpy().astype(np.float64)
+        assert np.linalg.norm(exact - got) < np.linalg.norm(exact - c0)
+
+
+def test_gemm_rejects_mismatched_rotation(mx):
+    x = torch.zeros(128, 256, dtype=torch.bfloat16, device="cuda")
+    qa = mx.quantize(x, mx.Config(hadamard=32, sf_layout=1), stats=False)
+    qb = mx.quantize(x, mx.Config(sf_layout=1), stats=False)
+    with pytest.raises(mx.MXError) as e:
+        mx.gemm(qa, qb)
+    assert e.value.code == -2
+
+
 def test_mxfp6_gemm_qsnr(mx, orc):
     M, N, K = 256, 256, 512
     a = inputs.laplace_outlier_cols(M, K, seed=6, n_outlier_cols=2)
