@@ -105,6 +105,9 @@ extern "C" {
 #define MX_TS_NONE    0   /* s_T = 1 */
 #define MX_TS_COMPUTE 1   /* s_T = amax_T / (max_elem * max_scale), written to *tensor_scale */
 #define MX_TS_GIVEN   2   /* s_T read from *tensor_scale (device) */
+#define MX_TS_AMAX    3   /* as MX_TS_COMPUTE, with amax_T taken from the workspace's amax
+                             word (left there by mx_tensor_amax, then reduced across the
+                             shards of a row-partitioned tensor) instead of a pre-pass */
 
 typedef struct {
     int32_t elem;          /* MX_E2M1 ... MX_INT4 */
@@ -204,7 +207,8 @@ int mx_quantize(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t ro
  *   capture.  Every call shares the one array (zero at load; every call
  *   leaves its control words zero), so calls that overlap on the
  *   GPU -- on different streams, or from different threads -- race: order them
- *   on one stream.  Rotation (mx_hadamard_quantize) is not covered.
+ *   on one stream.  Rotation (mx_hadamard_quantize) is not covered, nor
+ *   MX_TS_AMAX (its amax word is in a caller's workspace): MX_ERR_UNSUPPORTED.
  */
 int mx_quantize_noalloc(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t rows,
                         int64_t cols, void *codes, uint8_t *scales, float *tensor_scale,
@@ -224,6 +228,33 @@ int mx_hadamard_quantize(const mx_config *cfg, const void *x, int32_t x_dtype, i
                          int64_t cols, void *codes, uint8_t *scales, float *tensor_scale,
                          uint8_t *macro_scales, uint16_t *offsets, double *stats,
                          float *rotated, void *workspace, int64_t workspace_bytes, void *stream);
+
+/*
+ * mx_tensor_amax -- the tensor-amax pre-pass alone, for a tensor split by rows
+ * over several devices (one process per GPU): amax_T = max |x| (of the rotated
+ * y when cfg->hadamard), NaN ignored ([FINER] per-tensor scale), folded into
+ * the workspace's amax word (byte 0, the binary32 bits of amax_T, a max with
+ * what the word holds).  cfg->tensor_scale must be MX_TS_AMAX, and the word
+ * must hold zero or a partial amax.  The word keeps amax_T: the caller may
+ * reduce it across ranks (a max of the 32-bit words, which order like the
+ * non-negative floats they hold), then call mx_quantize /
+ * mx_hadamard_quantize with the same cfg and workspace, which derives
+ * s_T = amax_T / (max_elem * max_scale) from the word, writes it to
+ * *tensor_scale and clears the word.  Shapes and errors as mx_quantize; no
+ * outputs other than the word.  The pages have no multi-device procedure:
+ * this is how the per-tensor scale stays the one of the whole tensor.
+ */
+int mx_tensor_amax(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t rows, int64_t cols,
+                   void *workspace, int64_t workspace_bytes, void *stream);
+
+/*
+ * mx_stats_finalize -- recomputes the derived entries [5..9] of a `stats`
+ * buffer (device, MX_STATS_LEN doubles) from its sums [0..4] and element count
+ * [10]: after the sums of several shards' calls were added together (a sum
+ * reduction across ranks), the buffer then holds the whole tensor's MSE,
+ * R-MSE, QSNR, bias and flush share ([MXFP4-OAS] Sec.3 Eq. (1)).
+ */
+int mx_stats_finalize(double *stats, void *stream);
 
 /*
  * mx_dequantize -- x_hat from codes and scales ([MX-TRAIN] fake quantization).

@@ -32,7 +32,7 @@ RULE_FLOOR, RULE_CEIL, RULE_OAS, RULE_NEAREST, RULE_MSE = 0, 1, 2, 3, 4
 ROUND_RTNE, ROUND_CEIL, ROUND_STOCHASTIC = 0, 1, 2
 AXIS_ROW, AXIS_COL, AXIS_2D = 0, 1, 2
 DT_BF16, DT_FP32 = 0, 1
-TS_NONE, TS_COMPUTE, TS_GIVEN = 0, 1, 2
+TS_NONE, TS_COMPUTE, TS_GIVEN, TS_AMAX = 0, 1, 2, 3
 STATS_LEN = 16
 STAT_NAMES = ["sum_x2", "sum_e2", "sum_e", "n_ftz", "n_nonzero", "mse", "rmse", "qsnr_db",
               "bias", "ftz_frac", "count"]
@@ -113,11 +113,14 @@ def lib() -> C.CDLL:
         L.mx_gemm_qsnr.argtypes = [cfgp, cfgp, P, P, i64, i64, i64, P, P, P, P, P, P, P, P, i64, P]
         L.mx_mbs_gemm_scales.argtypes = [cfgp, P, P, i64, i64, P, P, P, i64, P]
         L.mx_device_status.argtypes = [P, C.POINTER(i32)]
+        L.mx_tensor_amax.argtypes = [cfgp, P, i32, i64, i64, P, i64, P]
+        L.mx_stats_finalize.argtypes = [P, P]
         L.mx_strerror.argtypes = [C.c_int]
         L.mx_strerror.restype = C.c_char_p
         L.mx_version.restype = C.c_char_p
         for f in ("mx_query_sizes", "mx_quantize", "mx_quantize_noalloc", "mx_hadamard_quantize", "mx_dequantize",
-                  "mx_qsnr", "mx_gemm", "mx_gemm_qsnr", "mx_mbs_gemm_scales", "mx_device_status"):
+                  "mx_qsnr", "mx_gemm", "mx_gemm_qsnr", "mx_mbs_gemm_scales", "mx_device_status",
+                  "mx_tensor_amax", "mx_stats_finalize"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -175,6 +178,15 @@ def mx_quantize(cfg: Config, x, x_dtype, rows, cols, codes, scales, tensor_scale
     c = cfg.c()
     return lib().mx_quantize(C.byref(c), x, x_dtype, rows, cols, codes, scales, tensor_scale,
                              macro, offsets, stats, workspace, workspace_bytes, stream)
+
+
+def mx_tensor_amax(cfg: Config, x, x_dtype, rows, cols, workspace, workspace_bytes, stream) -> int:
+    c = cfg.c()
+    return lib().mx_tensor_amax(C.byref(c), x, x_dtype, rows, cols, workspace, workspace_bytes, stream)
+
+
+def mx_stats_finalize(stats, stream) -> int:
+    return lib().mx_stats_finalize(stats, stream)
 
 
 def mx_quantize_noalloc(cfg: Config, x, x_dtype, rows, cols, codes, scales, tensor_scale, macro,
@@ -291,14 +303,17 @@ def alloc_outputs(cfg: Config, rows: int, cols: int, device, stats: bool = True,
 
 def quantize(x: torch.Tensor, cfg: Config = MXFP4, *, stats: bool = True,
              tensor_scale: torch.Tensor | None = None, rotated: bool = False,
-             out: Quantized | None = None, stream=None) -> Quantized:
+             out: Quantized | None = None, stream=None,
+             workspace: torch.Tensor | None = None) -> Quantized:
     """Block-quantize a 2-D bf16/fp32 CUDA tensor (``mx_quantize``, or
-    ``mx_hadamard_quantize`` when ``cfg.hadamard`` is set)."""
+    ``mx_hadamard_quantize`` when ``cfg.hadamard`` is set).  ``workspace``:
+    a caller's scratch (uint8, at least ``query_sizes(...).workspace_bytes``,
+    control words zero), needed with ``TS_AMAX`` to carry the amax."""
     _cuda2d(x, "x")
     rows, cols = x.shape
     q = out if out is not None else alloc_outputs(cfg, rows, cols, x.device, stats, rotated,
                                                   tensor_scale)
-    ws = _ws(query_sizes(cfg, rows, cols).workspace_bytes, x.device)
+    ws = workspace if workspace is not None else _ws(query_sizes(cfg, rows, cols).workspace_bytes, x.device)
     st = _stream(stream)
     if cfg.hadamard:
         rc = mx_hadamard_quantize(cfg, _p(x), _dtype_code(x), rows, cols, _p(q.codes), _p(q.scales),
@@ -311,6 +326,29 @@ def quantize(x: torch.Tensor, cfg: Config = MXFP4, *, stats: bool = True,
                          ws.numel(), st)
         _check("mx_quantize", rc)
     return q
+
+
+def tensor_amax(x: torch.Tensor, cfg: Config, workspace: torch.Tensor, stream=None) -> None:
+    """Fold max |x| (of the rotated tensor with ``cfg.hadamard``) into the
+    amax word at byte 0 of ``workspace`` (``mx_tensor_amax``; ``cfg`` with
+    ``tensor_scale=TS_AMAX``)."""
+    _cuda2d(x, "x")
+    rows, cols = x.shape
+    rc = mx_tensor_amax(cfg, _p(x), _dtype_code(x), rows, cols, _p(workspace), workspace.numel(),
+                        _stream(stream))
+    _check("mx_tensor_amax", rc)
+
+
+def stats_finalize(stats: torch.Tensor, stream=None) -> torch.Tensor:
+    """Recompute MSE / R-MSE / QSNR / bias / flush share of a stats buffer from
+    its sums and count, in place (``mx_stats_finalize``)."""
+    _check("mx_stats_finalize", mx_stats_finalize(_p(stats), _stream(stream)))
+    return stats
+
+
+def new_workspace(cfg: Config, rows: int, cols: int, device) -> torch.Tensor:
+    """A zeroed scratch buffer for ``quantize`` / ``tensor_amax``."""
+    return torch.zeros(query_sizes(cfg, rows, cols).workspace_bytes, dtype=torch.uint8, device=device)
 
 
 def dequantize(q: Quantized, out_dtype: torch.dtype = torch.float32, stream=None,

@@ -79,7 +79,7 @@ int check_config(const mx_config *c, int64_t rows, int64_t cols, bool want_had)
     if (c->round < MX_ROUND_RTNE || c->round > MX_ROUND_STOCHASTIC) return MX_ERR_INVALID;
     if (c->axis < MX_AXIS_ROW || c->axis > MX_AXIS_2D) return MX_ERR_INVALID;
     if (c->asymmetric != 0 && c->asymmetric != 1) return MX_ERR_INVALID;
-    if (c->tensor_scale < MX_TS_NONE || c->tensor_scale > MX_TS_GIVEN) return MX_ERR_INVALID;
+    if (c->tensor_scale < MX_TS_NONE || c->tensor_scale > MX_TS_AMAX) return MX_ERR_INVALID;
     if (c->macro_block != 0 && c->macro_block != 128) return MX_ERR_INVALID;
     if (c->hadamard != 0 && c->hadamard != 16 && c->hadamard != 32) return MX_ERR_INVALID;
     if (want_had != (c->hadamard != 0)) return MX_ERR_INVALID;
@@ -155,24 +155,28 @@ int cuda_ok(cudaError_t e) { return e == cudaSuccess ? MX_OK : MX_ERR_CUDA; }
 int quantize_impl(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t rows, int64_t cols,
                   void *codes, uint8_t *scales, float *tensor_scale, uint8_t *macro_scales,
                   uint16_t *offsets, double *stats, float *rotated, void *workspace,
-                  int64_t workspace_bytes, void *stream, bool want_had)
+                  int64_t workspace_bytes, void *stream, bool want_had, bool amax_only = false)
 {
     int rc = check_config(cfg, rows, cols, want_had);
     if (rc != MX_OK) return rc;
     if (x_dtype != MX_DT_BF16 && x_dtype != MX_DT_FP32) return MX_ERR_INVALID;
-    if (cfg->tensor_scale != MX_TS_NONE && !tensor_scale) return MX_ERR_INVALID;
-    if (cfg->macro_block && !macro_scales) return MX_ERR_INVALID;
-    if (cfg->asymmetric && !offsets) return MX_ERR_INVALID;
-    const bool need_ws = stats != nullptr || cfg->tensor_scale == MX_TS_COMPUTE;
+    if (!amax_only) {
+        if (cfg->tensor_scale != MX_TS_NONE && !tensor_scale) return MX_ERR_INVALID;
+        if (cfg->macro_block && !macro_scales) return MX_ERR_INVALID;
+        if (cfg->asymmetric && !offsets) return MX_ERR_INVALID;
+    }
+    const bool need_ws = stats != nullptr || cfg->tensor_scale == MX_TS_COMPUTE ||
+                         cfg->tensor_scale == MX_TS_AMAX || amax_only;
     if (need_ws && (!workspace || workspace_bytes < kWorkspaceBytes)) return MX_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t n = rows * cols;
     if (n == 0) {
+        if (amax_only) return MX_OK;
         if (stats) return launch_finalize_stats(nullptr, 0, 0.0, stats, st) ? MX_ERR_CUDA : MX_OK;
         return MX_OK;
     }
-    if (!x || !codes || !scales) return MX_ERR_INVALID;
-    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return MX_ERR_ALIGN;
+    if (!x || (!amax_only && (!codes || !scales))) return MX_ERR_INVALID;
+    if (!aligned16(x) || (!amax_only && (!aligned16(codes) || !aligned16(scales)))) return MX_ERR_ALIGN;
     if ((macro_scales && !aligned16(macro_scales)) || (offsets && !aligned16(offsets)) ||
         (rotated && !aligned16(rotated)) || (workspace && !aligned16(workspace)) ||
         (stats && ((uintptr_t)stats & 7u)) || (tensor_scale && ((uintptr_t)tensor_scale & 3u)))
@@ -197,7 +201,9 @@ int quantize_impl(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t 
     p.asym = cfg->asymmetric;
     p.mbs = cfg->macro_block;
     p.had = cfg->hadamard;
-    p.ts_mode = cfg->tensor_scale;
+    // a given amax (already in the workspace's amax word) is a computed
+    // tensor scale without the pre-pass
+    p.ts_mode = cfg->tensor_scale == MX_TS_AMAX ? (int)MX_TS_COMPUTE : cfg->tensor_scale;
     p.seed = cfg->seed;
     p.sf_gemm = cfg->sf_layout;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -206,8 +212,9 @@ int quantize_impl(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t 
     const int in_fp32 = x_dtype == MX_DT_FP32;
 
     // the tensor-amax pre-pass; the quantizer derives s_T from its word
-    if (cfg->tensor_scale == MX_TS_COMPUTE && launch_tensor_amax(p, cfg->axis, in_fp32, st))
+    if ((cfg->tensor_scale == MX_TS_COMPUTE || amax_only) && launch_tensor_amax(p, cfg->axis, in_fp32, st))
         return MX_ERR_CUDA;
+    if (amax_only) return MX_OK;
     p.partials = stats ? partials : nullptr;
     p.stats = stats;
     p.count = (double)n;
@@ -270,6 +277,22 @@ int mx_hadamard_quantize(const mx_config *cfg, const void *x, int32_t x_dtype, i
 {
     return quantize_impl(cfg, x, x_dtype, rows, cols, codes, scales, tensor_scale, macro_scales,
                          offsets, stats, rotated, workspace, workspace_bytes, stream, true);
+}
+
+int mx_tensor_amax(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t rows, int64_t cols,
+                   void *workspace, int64_t workspace_bytes, void *stream)
+{
+    if (!cfg) return MX_ERR_INVALID;
+    if (cfg->tensor_scale != MX_TS_AMAX) return MX_ERR_INVALID;
+    return quantize_impl(cfg, x, x_dtype, rows, cols, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                         nullptr, workspace, workspace_bytes, stream, cfg->hadamard != 0, true);
+}
+
+int mx_stats_finalize(double *stats, void *stream)
+{
+    if (!stats) return MX_ERR_INVALID;
+    if ((uintptr_t)stats & 7u) return MX_ERR_ALIGN;
+    return launch_stats_refinalize(stats, static_cast<cudaStream_t>(stream)) ? MX_ERR_CUDA : MX_OK;
 }
 
 int mx_dequantize(const mx_config *cfg, const void *codes, const uint8_t *scales,

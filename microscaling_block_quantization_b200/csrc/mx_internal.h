@@ -94,6 +94,7 @@ int launch_quantize_fast(const QParams &p, int in_fp32, cudaStream_t st, int *gr
 int launch_quantize_gen(const QParams &p, int in_fp32, cudaStream_t st, int *grid_out);
 // Read and clear the status words of the two persistent quantizers'
 // bounded waits (synchronise st); 0 when no wait gave up.
+int launch_stats_refinalize(double *stats, cudaStream_t st);
 int take_status_fast(cudaStream_t st, int *v);
 int take_status_gen(cudaStream_t st, int *v);
 

@@ -51,6 +51,8 @@ extern "C" int mx_quantize_noalloc(const mx_config *cfg, const void *x, int32_t 
     mx_sizes s;
     int rc = mx_query_sizes(cfg, rows, cols, &s);
     if (rc != MX_OK) return rc;
+    // a given amax lives in a caller's workspace, which this entry has none of
+    if (cfg->tensor_scale == MX_TS_AMAX) return MX_ERR_UNSUPPORTED;
     if (s.workspace_bytes > kScratchBytes) return MX_ERR_WORKSPACE;
     void *scratch = nullptr;
     rc = scratch_for_current_device(&scratch);

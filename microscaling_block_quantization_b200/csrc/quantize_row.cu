@@ -336,6 +336,14 @@ __global__ void __launch_bounds__(kThreads) k_amax_vec(const QParams p)
 
 // Sum the per-CTA records in a fixed order and derive MSE, R-MSE, QSNR (Eq. (1)),
 // bias and the flush-to-zero share.
+// derived statistics recomputed from the sums and the count already in
+// `stats` (after the sums of several calls were added together)
+__global__ void k_refinalize_stats(double *stats)
+{
+    const double s[5] = {stats[0], stats[1], stats[2], stats[3], stats[4]};
+    store_stats(stats, s, stats[10]);
+}
+
 __global__ void k_finalize_stats(const double *partials, int nparts, double count, double *stats)
 {
     __shared__ double sh[256][5];
@@ -456,6 +464,12 @@ int launch_finalize_stats(const double *partials, int nparts, double count, doub
                           cudaStream_t st)
 {
     k_finalize_stats<<<1, 256, 0, st>>>(partials, nparts, count, stats);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_stats_refinalize(double *stats, cudaStream_t st)
+{
+    k_refinalize_stats<<<1, 1, 0, st>>>(stats);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

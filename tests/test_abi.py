@@ -118,6 +118,24 @@ def test_gemm_operand_pairs_checked_on_host(mx):
     assert gemm(mx.Config(**g), mx.Config(**g), K=128) == -1                # K % 256
 
 
+def test_sharding_entry_points_checked_on_host(mx):
+    P = C.c_void_p
+    amax_cfg = mx.Config(block=16, scale_fmt=mx.SCALE_UE4M3, rule=mx.RULE_NEAREST, tensor_scale=mx.TS_AMAX)
+    # the amax pass wants the amax mode and a workspace
+    assert mx.mx_tensor_amax(mx.NVFP4, P(4096), 0, 64, 64, P(4096), 4096, None) == -1
+    assert mx.mx_tensor_amax(amax_cfg, P(4096), 0, 64, 64, None, 0, None) == -5
+    assert mx.mx_tensor_amax(amax_cfg, P(4100), 0, 64, 64, P(4096), 1 << 20, None) == -3
+    # the given-amax mode: a workspace carries the amax; not through the no-alloc entry
+    assert mx.mx_quantize(amax_cfg, P(4096), 0, 64, 64, P(4096), P(4096), P(4096), None, None, None,
+                          None, 0, None) == -5
+    assert mx.mx_quantize_noalloc(amax_cfg, P(4096), 0, 64, 64, P(4096), P(4096), P(4096), None, None,
+                                  None, None) == -2
+    assert mx.mx_quantize(mx.Config(block=16, scale_fmt=mx.SCALE_UE4M3, rule=mx.RULE_NEAREST, tensor_scale=4),
+                          P(4096), 0, 64, 64, P(4096), P(4096), P(4096), None, None, None, None, 0, None) == -1
+    assert mx.mx_stats_finalize(None, None) == -1
+    assert mx.mx_stats_finalize(P(4100), None) == -3
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     import microscaling_block_quantization_b200 as m
     monkeypatch.setattr(m, "_lib", None)
