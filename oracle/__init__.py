@@ -91,6 +91,8 @@ def lib():
         L.orc_fwht.argtypes = [C.c_int, P, C.c_int]
         L.orc_tensor_scale.argtypes = [C.c_int, C.c_int, P, i64]
         L.orc_tensor_scale.restype = C.c_float
+        L.orc_mse_grid_trace.argtypes = [C.c_int, C.c_int, P, C.c_int, i64, i64, C.c_int, P, P]
+        L.orc_mse_grid_trace.restype = C.c_float
         L.orc_gemm.argtypes = [P, P, i64, i64, i64, P]
         L.orc_gemm_qsnr.argtypes = [P, P, P, P, i64, i64, i64, P]
         L.orc_bf16_to_f32.argtypes = [C.c_uint16]
@@ -253,6 +255,18 @@ def scale_decode(fmt: int, code: int) -> float:
 
 def scale_encode_nearest(fmt: int, x: float) -> int:
     return int(lib().orc_scale_encode_nearest(fmt, x))
+
+
+def mse_grid_trace(scale_fmt: int, block: int, x, rounds: int = 4):
+    """The alternating global / group scale optimisation of the MSE rule with
+    a nearest scale format (row blocks): final s_T, the s_T before each group
+    step and the squared error after it (rounds + 1 entries each)."""
+    arr, dt = as_input(x)
+    rows, cols = arr.shape
+    st = np.zeros(rounds + 1, np.float32)
+    se = np.zeros(rounds + 1, np.float64)
+    s = lib().orc_mse_grid_trace(scale_fmt, block, _ptr(arr), dt, rows, cols, rounds, _ptr(st), _ptr(se))
+    return float(s), st, se
 
 
 def fwht(v: np.ndarray, normalise: bool = True) -> np.ndarray:

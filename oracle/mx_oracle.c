@@ -490,6 +490,101 @@ static int mse_exponent(const grid_t *g, int asym, const float *res, int L, floa
     return (sum[0] <= 4.0 * sum[1]) ? k0 : k1;
 }
 
+/* (READING) MSE-optimal UE4M3 / UE5M3 block scale for a given tensor scale */
+/* s_T ([BRIDGING] sec. 2.2: MSE-optimised grids, the group-scale half of   */
+/* the alternating optimisation): the pages name the objective, not the     */
+/* search, so the plainest reading is the exact argmin over every finite    */
+/* scale code c of the block's squared error                                */
+/*   SSE(c) = sum_t (x_t - x_hat_t)^2,  x_hat_t = (q_t s_c) s_T,             */
+/* q_t the nearest-even grid value of x_t * RN(1 / RN(s_c s_T)) (the        */
+/* element rule of the nearest-scale formats), a block of zeros when        */
+/* s_c = 0 or the reciprocal overflows.  Each SSE is accumulated in binary64 */
+/* in element order (x_t - x_hat_t rounded once to binary64, squared, added) */
+/* and ties keep the lower code.  Pinned: never above the nearest rule's    */
+/* block error; single values q s reproduced exactly (tests).               */
+static uint8_t mse_ue_code(const grid_t *g, int fmt, const float *res, int L, float sT, double *sse_out)
+{
+    ufmt_t u = ufmt(fmt);
+    int best = 0;
+    double best_sse = INFINITY;
+    for (int c = 0; c < u.nan_code; c++) {
+        float sb = orc_scale_decode(fmt, (uint8_t)c);
+        float d = sb * sT;
+        float inv = 1.0f / d;
+        int zero = (sb == 0.0f) || !(inv < INFINITY);
+        double acc = 0.0;
+        for (int t = 0; t < L; t++) {
+            float xh = 0.0f;
+            if (!zero) {
+                float v = res[t] * inv;
+                float q = decode_elem(g, 0, encode_elem(g, 0, RD_RTNE, v, 0u));
+                xh = (q * sb) * sT;
+            }
+            double e = (double)res[t] - (double)xh;
+            acc += e * e;
+        }
+        if (acc < best_sse) { best_sse = acc; best = c; }
+    }
+    if (sse_out) *sse_out = best_sse;
+    return (uint8_t)best;
+}
+
+/* (READING) the global-scale half ([BRIDGING] sec. 2.2: alternating        */
+/* optimisation of the global and the group scales).  Starting from the     */
+/* amax rule's s_T, each round takes the group step above for every block,  */
+/* then, with the codes and element values u_t = q_t s_c held fixed, the    */
+/* s_T minimising sum (x_t - u_t s_T)^2: the least-squares factor           */
+/* s_T = sum x_t u_t / sum u_t^2 (binary64 sums in block and element order,  */
+/* every product exact there; rounded once to binary32; kept when it is not */
+/* a positive finite number).  The pages give no round count: MSE_ROUNDS.   */
+/* Blocks with a non-finite value take no part.  The squared error after    */
+/* each group step cannot rise from one round to the next (up to binary32   */
+/* rounding of x_hat and s_T): the pin of the tests.                         */
+#define MSE_ROUNDS 4
+
+static float mse_grid_alternate(const grid_t *g, int fmt, int axis, int B, const float *y, int64_t rows,
+                                int64_t cols, float sT, int rounds, float *sT_trace, double *sse_trace)
+{
+    const int64_t nb = n_blocks(axis, B, rows, cols);
+    const int L = block_len(axis, B);
+    float *res = (float *)malloc((size_t)L * sizeof(float));
+    if (!res) return NAN;
+    for (int it = 0; ; it++) {
+        double num = 0.0, den = 0.0, sse = 0.0;
+        for (int64_t b = 0; b < nb; b++) {
+            int nonfinite = 0;
+            for (int t = 0; t < L; t++) {
+                int64_t r, c;
+                block_elem(axis, B, rows, cols, b, t, &r, &c);
+                res[t] = y[r * cols + c];
+                if (!isfinite(res[t])) nonfinite = 1;
+            }
+            if (nonfinite) continue;
+            double bsse;
+            uint8_t code = mse_ue_code(g, fmt, res, L, sT, &bsse);
+            sse += bsse;
+            float sb = orc_scale_decode(fmt, code);
+            float inv = 1.0f / (sb * sT);
+            if (sb == 0.0f || !(inv < INFINITY)) continue;
+            for (int t = 0; t < L; t++) {
+                float q = decode_elem(g, 0, encode_elem(g, 0, RD_RTNE, res[t] * inv, 0u));
+                float u = q * sb;
+                num += (double)res[t] * (double)u;
+                den += (double)u * (double)u;
+            }
+        }
+        if (sT_trace) sT_trace[it] = sT;
+        if (sse_trace) sse_trace[it] = sse;
+        if (it == rounds) break;
+        if (den > 0.0) {
+            float s = (float)(num / den);
+            if (s > 0.0f && isfinite(s)) sT = s;
+        }
+    }
+    free(res);
+    return sT;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Quantize                                                                 */
 /* ------------------------------------------------------------------------ */
@@ -537,6 +632,9 @@ int orc_quantize(const orc_cfg *cfg, const void *x, int dtype, int64_t rows, int
     float sT = 1.0f;
     if (cfg->tensor_scale == TS_COMPUTE) {
         sT = orc_tensor_scale(cfg->elem, cfg->scale_fmt, y, n);
+        /* MSE rule with a nearest-scale format: the alternating optimisation */
+        if (cfg->rule == R_MSE && cfg->scale_fmt != S_E8M0)
+            sT = mse_grid_alternate(&g, cfg->scale_fmt, cfg->axis, B, y, rows, cols, sT, MSE_ROUNDS, NULL, NULL);
         if (tensor_scale) *tensor_scale = sT;
     } else if (cfg->tensor_scale == TS_GIVEN) {
         sT = *tensor_scale;
@@ -641,12 +739,13 @@ int orc_quantize(const orc_cfg *cfg, const void *x, int dtype, int64_t rows, int
                 scode = (uint8_t)(k + 127);
                 inv = pow2f(-k);
             }
-        } else if (cfg->rule == R_NEAREST) {
+        } else if (cfg->rule == R_NEAREST || cfg->rule == R_MSE) {
             ufmt_t u = ufmt(cfg->scale_fmt);
             if (nonfinite) { scode = (uint8_t)u.nan_code; zero_block = 1; }
             else {
                 float sb_real = (alpha / grid_max(&g)) / sT;
-                scode = orc_scale_encode_nearest(cfg->scale_fmt, sb_real);
+                scode = cfg->rule == R_MSE ? mse_ue_code(&g, cfg->scale_fmt, res, L, sT, NULL)
+                                           : orc_scale_encode_nearest(cfg->scale_fmt, sb_real);
                 float sb = orc_scale_decode(cfg->scale_fmt, scode);
                 if (isnan(sb)) zero_block = 1;
                 else {
@@ -696,6 +795,23 @@ int orc_quantize(const orc_cfg *cfg, const void *x, int dtype, int64_t rows, int
 /* column in the low nibble; 6-bit codes one per byte (low 6 bits).          */
 /* Pinned: 4.25 / 4.5 bits per element for MXFP4 / NVFP4 storage.            */
 /* ------------------------------------------------------------------------ */
+/* The alternating optimisation's s_T and squared error after each group
+ * step (rounds + 1 entries each), for the tests: row-axis E2M1 blocks, a
+ * nearest scale format, bf16 or fp32 input.  Returns the final s_T. */
+float orc_mse_grid_trace(int scale_fmt, int block, const void *x, int dtype, int64_t rows, int64_t cols,
+                         int rounds, float *sT_trace, double *sse_trace)
+{
+    grid_t g; make_grid(0, 0, &g);
+    const int64_t n = rows * cols;
+    float *y = (float *)malloc((size_t)n * sizeof(float));
+    if (!y) return NAN;
+    load_input(x, dtype, n, y);
+    float sT = orc_tensor_scale(0, scale_fmt, y, n);
+    sT = mse_grid_alternate(&g, scale_fmt, AX_ROW, block, y, rows, cols, sT, rounds, sT_trace, sse_trace);
+    free(y);
+    return sT;
+}
+
 int64_t orc_packed_bytes(int elem, int64_t rows, int64_t cols)
 {
     grid_t g; make_grid(elem, 0, &g);
@@ -715,6 +831,8 @@ void orc_pack(int elem, const uint8_t *codes, int64_t rows, int64_t cols, uint8_
             packed[r * (cols / 2) + j] = (uint8_t)(lo | (hi << 4));
         }
 }
+
+void orc_unpack(int elem, const uint8_t *packed, int64_t rows, int64_t cols, uint8_t *codes);
 
 /* (READING) Tensor-core operand layout of FP6 codes (the library's
  * sf_layout = 1): every 16 consecutive codes of a row are packed into 12
@@ -797,7 +915,7 @@ int orc_dequantize(const orc_cfg *cfg, const uint8_t *packed, const uint8_t *sca
             float q = decode_elem(&g, asym, codes[idx]);
             float v;
             if (isnan(s)) v = NAN;
-            else if (cfg->scale_fmt != S_E8M0 && cfg->rule == R_NEAREST) v = (q * s) * sT;
+            else if (cfg->scale_fmt != S_E8M0 && (cfg->rule == R_NEAREST || cfg->rule == R_MSE)) v = (q * s) * sT;
             else {
                 v = q * s;
                 if (cfg->macro_block) v = v * e4m3_decode(macro[macro_index(cfg->axis, rows, cols, r, c)]);

@@ -446,3 +446,146 @@ def test_mse_rule_constant_blocks(orc):
         x = torch.full((1, 32), val, dtype=torch.float32)
         r = orc.quantize(orc.Cfg(rule=orc.MSE), x)
         assert int(r["scales"][0]) == 127 + k, (val, r["scales"][0])
+
+
+def _ue4m3_values():
+    """UE4M3 values of codes 0..126 from the format's fields (bias 7, three
+    mantissa bits, subnormals for exponent field 0)."""
+    out = []
+    for c in range(127):
+        e, m = c >> 3, c & 7
+        out.append(m / 8.0 * 2.0 ** -6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7))
+    return np.array(out, np.float64)
+
+
+def _nearest_even_e2m1(v):
+    grid = _grid(0)
+    a = abs(float(v))
+    if a >= 6.0:
+        return math.copysign(6.0, v)
+    d = np.abs(grid - a)
+    best = np.flatnonzero(d == d.min())
+    i = best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
+    return math.copysign(grid[i], v)
+
+
+def _brute_force_ue_code(v, sT):
+    """Argmin over every finite UE4M3 code of the block's squared error, with
+    the element rule of the nearest formats, evaluated from the definitions
+    (binary32 steps via numpy float32, binary64 sum in element order); ties
+    keep the lower code."""
+    f32 = np.float32
+    best, bc = math.inf, 0
+    for c, s in enumerate(_ue4m3_values()):
+        s = f32(s)
+        d = f32(s * f32(sT))
+        with np.errstate(divide="ignore", over="ignore"):
+            inv = f32(f32(1.0) / d)
+        zero = s == 0 or not np.isfinite(inv)
+        acc = 0.0
+        for x in v:
+            xh = f32(0.0)
+            if not zero:
+                q = f32(_nearest_even_e2m1(f32(f32(x) * inv)))
+                xh = f32(f32(q * s) * f32(sT))
+            e = float(x) - float(xh)
+            acc += e * e
+        if acc < best:
+            best, bc = acc, c
+    return bc
+
+
+@pytest.mark.parametrize("sT", [1.0, 0.0123, 3.7e-4])
+def test_mse_ue_group_step_brute_force(orc, sT):
+    """MSE rule with UE4M3 scales and a given tensor scale: every block's code
+    is the brute-force argmin over all 127 finite codes (checked here from
+    the format's and the grid's definitions)."""
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((12, 32)) * np.exp(rng.uniform(-2, 2, (12, 1)))).astype(np.float32)
+    x *= np.float32(sT * 200)
+    x[3, :16] = 0.0                              # an all-zero block
+    x[5, 3] *= 30                                # an outlier
+    cfg = orc.Cfg(block=16, scale_fmt=orc.UE4M3, rule=orc.MSE, tensor_scale=orc.TS_GIVEN)
+    r = orc.quantize(cfg, torch.from_numpy(x), tensor_scale=sT)
+    for b in range(24):
+        v = x.reshape(-1, 16)[b]
+        assert int(r["scales"][b]) == _brute_force_ue_code(v, sT), b
+
+
+def test_mse_ue_reproduces_single_values(orc):
+    """Closed form: a block holding one value v = q s (q on the E2M1 grid, s a
+    UE4M3 value) and zeros has a zero-error scale, so the MSE rule returns v
+    exactly; the nearest rule, which maps the block max to 6, misses many."""
+    vals = _ue4m3_values()[8::5]                 # normal scales across the range
+    misses = 0
+    for s in vals:
+        for q in (0.5, 1.0, 1.5, 3.0, 4.0, 6.0):
+            v = np.float32(q * s)
+            x = np.zeros((1, 32), np.float32)
+            x[0, 5] = v
+            x[0, 20] = -v
+            for rule in (orc.MSE, orc.NEAREST):
+                cfg = orc.Cfg(block=16, scale_fmt=orc.UE4M3, rule=rule)
+                r = orc.quantize(cfg, torch.from_numpy(x))
+                xh = orc.dequantize(cfg, r["packed"], r["scales"], 1.0, None, None, 1, 32)
+                if rule == orc.MSE:
+                    assert np.array_equal(xh, x), (q, s)
+                else:
+                    misses += int(not np.array_equal(xh, x))
+    assert misses > 0
+
+
+def _block_sse(x, xh, B):
+    d = x.astype(np.float64).reshape(-1, B) - xh.astype(np.float64).reshape(-1, B)
+    return (d * d).sum(axis=1)
+
+
+@pytest.mark.parametrize("B", [8, 16, 32])
+def test_mse_ue_never_worse_than_nearest(orc, B):
+    """Invariant: for the same tensor scale the MSE rule's block error is
+    never above the nearest rule's, block by block."""
+    from microscaling_block_quantization_b200 import inputs
+    for x in (inputs.laplace_outlier_cols(64, 256, seed=4, n_outlier_cols=4),
+              inputs.normal(64, 256, sigma=0.02, seed=7)):
+        near = orc.Cfg(block=B, scale_fmt=orc.UE4M3, rule=orc.NEAREST, tensor_scale=orc.TS_COMPUTE)
+        rn = orc.quantize(near, x)
+        sT = rn["tensor_scale"]
+        mse = orc.Cfg(block=B, scale_fmt=orc.UE4M3, rule=orc.MSE, tensor_scale=orc.TS_GIVEN)
+        rm = orc.quantize(mse, x, tensor_scale=sT)
+        xn = orc.dequantize(near, rn["packed"], rn["scales"], sT, None, None, 64, 256)
+        xm = orc.dequantize(mse, rm["packed"], rm["scales"], sT, None, None, 64, 256)
+        y = orc.input_f32(x)
+        sn, sm = _block_sse(y, xn, B), _block_sse(y, xm, B)
+        assert np.all(sm <= sn * (1 + 1e-12) + 1e-300)
+        assert sm.sum() < sn.sum()
+
+
+def test_mse_ue_alternation(orc):
+    """Alternating optimisation of the global and group scales: the squared
+    error after each group step does not rise (up to binary32 rounding of
+    x_hat and s_T); every global step is the least-squares factor of the
+    fixed element values u = q s_c (checked against numpy's sums, and as a
+    minimum: moving s_T either way raises the fixed-u error); the quantizer
+    with a computed tensor scale ends on the trace's last s_T."""
+    from microscaling_block_quantization_b200 import inputs
+    for x in (inputs.laplace_outlier_cols(128, 256, seed=4, n_outlier_cols=4),
+              inputs.normal(128, 256, sigma=0.02, seed=7)):
+        sfin, st, se = orc.mse_grid_trace(orc.UE4M3, 16, x, rounds=4)
+        assert np.all(se[1:] <= se[:-1] * (1 + 1e-6))
+        y = orc.input_f32(x).astype(np.float64)
+        for i in range(4):
+            cfg = orc.Cfg(block=16, scale_fmt=orc.UE4M3, rule=orc.MSE, tensor_scale=orc.TS_GIVEN)
+            r = orc.quantize(cfg, x, tensor_scale=float(st[i]))
+            # u = q s_c: the dequantized values with a unit tensor scale
+            u = orc.dequantize(cfg, r["packed"], r["scales"], 1.0, None, None, 128, 256).astype(np.float64)
+            s_ls = float((y * u).sum() / (u * u).sum())
+            assert st[i + 1] == pytest.approx(s_ls, rel=1e-6)
+            f = lambda s: float(((y - u * s) ** 2).sum())
+            assert f(s_ls) <= min(f(s_ls * (1 + 1e-3)), f(s_ls * (1 - 1e-3)))
+        cfg = orc.Cfg(block=16, scale_fmt=orc.UE4M3, rule=orc.MSE, tensor_scale=orc.TS_COMPUTE)
+        r = orc.quantize(cfg, x)
+        assert np.float32(r["tensor_scale"]) == np.float32(sfin) == st[-1]
+        near = orc.Cfg(block=16, scale_fmt=orc.UE4M3, rule=orc.NEAREST, tensor_scale=orc.TS_COMPUTE)
+        rn = orc.quantize(near, x)
+        xn = orc.dequantize(near, rn["packed"], rn["scales"], rn["tensor_scale"], None, None, 128, 256)
+        assert se[-1] < float(((y - xn) ** 2).sum())
