@@ -79,12 +79,23 @@ extern "C" {
 #define MX_RULE_CEIL    1
 #define MX_RULE_OAS     2
 #define MX_RULE_NEAREST 3
-/* MSE: per-block MSE-optimal E8M0 scale (a per-block scale search; the pages
- * suggest optimising scales for MSE but fix no search): the exponent among
- * k_floor and k_floor + 1 whose nearest-even codes leave the smaller block
- * squared error, 4^k sum (v - q)^2 with v = binary32(x 2^-k), each sum in
- * binary64 in element order, ties to k_floor.  E8M0, MX_ROUND_RTNE, row
- * axis, block 32, symmetric, no macro scale or rotation. */
+/* MSE: MSE-optimal block scales ([BRIDGING] sec. 2.2: MSE-optimised grids;
+ * the pages name the objective, not the search).  Row axis, MX_ROUND_RTNE,
+ * symmetric, no macro scale or rotation.
+ *   E8M0 (block 32, any element type): the exponent among k_floor and
+ *   k_floor + 1 whose nearest-even codes leave the smaller block squared
+ *   error, 4^k sum (v - q)^2 with v = binary32(x 2^-k), each sum in binary64
+ *   in element order, ties to k_floor.
+ *   UE4M3 / UE5M3 (E2M1, blocks of 8, 16 or 32): for the tensor scale s_T
+ *   (MX_TS_NONE: 1, MX_TS_GIVEN: *tensor_scale) every block takes the code
+ *   c, over all finite codes, with the smallest sum (x - x_hat)^2, x_hat =
+ *   (q s_c) s_T and q the nearest-even value of x * RN(1 / RN(s_c s_T));
+ *   binary64 differences, squares and element-order sums, ties to the lower
+ *   code.  With MX_TS_COMPUTE the global and the group scales alternate
+ *   (four rounds from the amax rule's s_T): the group step above, then
+ *   s_T = sum x u / sum u^2 with u = q s_c held fixed (binary64 sums rounded
+ *   once to binary32); the final s_T is written to *tensor_scale.  Dequantize
+ *   and GEMM read these scales like nearest ones. */
 #define MX_RULE_MSE     4
 
 /* ---- element rounding ([MX-TRAIN]) ------------------------------------- */

@@ -72,10 +72,20 @@ int check_config(const mx_config *c, int64_t rows, int64_t cols, bool want_had)
     if (c->elem < MX_E2M1 || c->elem > MX_INT4) return MX_ERR_INVALID;
     if (c->scale_fmt < MX_SCALE_E8M0 || c->scale_fmt > MX_SCALE_UE5M3) return MX_ERR_INVALID;
     if (c->rule < MX_RULE_FLOOR || c->rule > MX_RULE_MSE) return MX_ERR_INVALID;
-    if (c->rule == MX_RULE_MSE &&
-        (c->scale_fmt != MX_SCALE_E8M0 || c->round != MX_ROUND_RTNE || c->axis != MX_AXIS_ROW ||
-         c->block != 32 || c->asymmetric || c->macro_block || c->hadamard || c->tensor_scale != MX_TS_NONE))
-        return MX_ERR_UNSUPPORTED;
+    // MSE rule: E8M0 blocks of 32 (any element type), or E2M1 with a nearest
+    // scale format and blocks of 8 / 16 / 32 (the alternating optimisation
+    // with a computed tensor scale); row axis, nearest-even elements
+    if (c->rule == MX_RULE_MSE) {
+        if (c->round != MX_ROUND_RTNE || c->axis != MX_AXIS_ROW || c->asymmetric || c->macro_block ||
+            c->hadamard)
+            return MX_ERR_UNSUPPORTED;
+        if (c->scale_fmt == MX_SCALE_E8M0 && (c->block != 32 || c->tensor_scale != MX_TS_NONE))
+            return MX_ERR_UNSUPPORTED;
+        if (c->scale_fmt != MX_SCALE_E8M0 &&
+            (c->elem != MX_E2M1 || !(c->block == 8 || c->block == 16 || c->block == 32) ||
+             c->tensor_scale == MX_TS_AMAX))
+            return MX_ERR_UNSUPPORTED;
+    }
     if (c->round < MX_ROUND_RTNE || c->round > MX_ROUND_STOCHASTIC) return MX_ERR_INVALID;
     if (c->axis < MX_AXIS_ROW || c->axis > MX_AXIS_2D) return MX_ERR_INVALID;
     if (c->asymmetric != 0 && c->asymmetric != 1) return MX_ERR_INVALID;
@@ -100,7 +110,8 @@ int check_config(const mx_config *c, int64_t rows, int64_t cols, bool want_had)
         if (c->rule == MX_RULE_NEAREST) return MX_ERR_INVALID;
         if (c->tensor_scale != MX_TS_NONE) return MX_ERR_INVALID;
     } else {
-        if (c->rule != MX_RULE_NEAREST && c->tensor_scale != MX_TS_NONE) return MX_ERR_UNSUPPORTED;
+        if (c->rule != MX_RULE_NEAREST && c->rule != MX_RULE_MSE && c->tensor_scale != MX_TS_NONE)
+            return MX_ERR_UNSUPPORTED;
         if (c->asymmetric) return MX_ERR_UNSUPPORTED;
     }
     if (c->macro_block) {
@@ -221,6 +232,12 @@ int quantize_impl(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t 
     p.ticket = need_ws ? reinterpret_cast<unsigned int *>(ws + kWsTicket) : nullptr;
     const int fast = cfg->elem == MX_E2M1 && cfg->round == MX_ROUND_RTNE && !cfg->asymmetric &&
                      cfg->rule != MX_RULE_MSE;
+    if (cfg->rule == MX_RULE_MSE && cfg->scale_fmt != MX_SCALE_E8M0) {
+        // (a computed tensor scale: the global-step passes reduce through the
+        // workspace records and ticket, which need_ws has required)
+        float *chain = ws ? reinterpret_cast<float *>(ws + kWsMseChain) : nullptr;
+        return launch_quantize_mse(p, partials, chain, in_fp32, st) ? MX_ERR_CUDA : MX_OK;
+    }
     int grid = 0;
     if (launch_quantize(p, cfg->axis, in_fp32, fast, st, &grid)) return MX_ERR_CUDA;
     return MX_OK;
@@ -324,6 +341,8 @@ int mx_dequantize(const mx_config *cfg, const void *codes, const uint8_t *scales
     p.out_fp32 = out_dtype == MX_DT_FP32;
     if (!make_elem(cfg->elem, cfg->asymmetric, p.ed)) return MX_ERR_INVALID;
     if (!make_scale(cfg, p.sd)) return MX_ERR_INVALID;
+    // an MSE-chosen nearest-format scale dequantizes like a nearest one
+    if (p.sd.fmt != S_E8M0 && p.sd.rule == R_MSE) p.sd.rule = R_NEAREST;
     p.block = cfg->block;
     p.axis = cfg->axis;
     p.asym = cfg->asymmetric;

@@ -753,8 +753,10 @@ int fp4_kind(const mx_config *a, const mx_config *b)
     if (a->elem != MX_E2M1 || b->elem != MX_E2M1) return -1;
     if (a->scale_fmt == MX_SCALE_E8M0 && b->scale_fmt == MX_SCALE_E8M0 && a->block == 32 && b->block == 32)
         return KIND_MXF4;
-    if (a->scale_fmt == MX_SCALE_UE4M3 && b->scale_fmt == MX_SCALE_UE4M3 && a->rule == MX_RULE_NEAREST &&
-        b->rule == MX_RULE_NEAREST && a->block == 16 && b->block == 16)
+    // (UE4M3 scales chosen by the nearest or the MSE rule alike)
+    auto near = [](const mx_config *c) { return c->rule == MX_RULE_NEAREST || c->rule == MX_RULE_MSE; };
+    if (a->scale_fmt == MX_SCALE_UE4M3 && b->scale_fmt == MX_SCALE_UE4M3 && near(a) && near(b) &&
+        a->block == 16 && b->block == 16)
         return KIND_NVF4;
     return -1;
 }

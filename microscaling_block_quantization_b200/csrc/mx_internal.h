@@ -16,6 +16,9 @@ constexpr int kPartialDoubles = 8;
 // zero before a launch and the launch's last CTA leaves them zero.
 constexpr int64_t kWsHeader = 256;
 constexpr int64_t kWsTicket = 64;
+// the MSE rule's tensor scale of each alternation round (floats, cleared by
+// the call that used them)
+constexpr int64_t kWsMseChain = 192;
 constexpr int64_t kWorkspaceBytes = kWsHeader + (int64_t)kMaxPartials * kPartialDoubles * 8;
 
 struct QParams {
@@ -95,6 +98,7 @@ int launch_quantize_gen(const QParams &p, int in_fp32, cudaStream_t st, int *gri
 // Read and clear the status words of the two persistent quantizers'
 // bounded waits (synchronise st); 0 when no wait gave up.
 int launch_stats_refinalize(double *stats, cudaStream_t st);
+int launch_quantize_mse(const QParams &p, double *records, float *chain, int in_fp32, cudaStream_t st);
 int take_status_fast(cudaStream_t st, int *v);
 int take_status_gen(cudaStream_t st, int *v);
 

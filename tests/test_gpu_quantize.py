@@ -5,6 +5,7 @@ per-tensor scale, the rotated tensor and the dequantized values.
 Tolerance (binary64 sums of binary32 terms in a different order): 1e-4
 relative on the squared sums / MSE / R-MSE, 1e-3 dB on QSNR, exact counts.
 """
+import dataclasses
 import math
 
 import numpy as np
@@ -192,6 +193,72 @@ def test_given_tensor_scale(mx, orc):
 def test_elements_and_rounding(mx, orc, elem, rule, asym, rnd, dtype):
     x = inputs.gradient_like(64, 512, seed=5, dtype=dtype)
     run_case(mx, orc, x, mx.Config(elem=elem, rule=rule, asymmetric=asym, round=rnd, seed=12345))
+
+
+@pytest.mark.parametrize("block", [8, 16, 32])
+@pytest.mark.parametrize("fmt", [1, 2])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_mse_nearest_format_group_step(mx, orc, block, fmt, dtype):
+    """MSE rule with a UE4M3 / UE5M3 scale and a given (or unit) tensor
+    scale: every block's code is the exact argmin of its binary64 squared
+    error over all finite codes.  Codes, scales, x_hat and statistics against
+    the oracle on a ragged multi-CTA shape with zero / NaN blocks planted."""
+    x = inputs.laplace_outlier_cols(72, 544, seed=4, n_outlier_cols=4, dtype=torch.float32)
+    x[3, 32:64] = 0.0
+    x[7, 100] = float("nan")
+    x = x.to(dtype)
+    run_case(mx, orc, x, mx.Config(block=block, scale_fmt=fmt, rule=mx.RULE_MSE, tensor_scale=mx.TS_GIVEN),
+             given_ts=0.0123)
+    if fmt == 1:
+        run_case(mx, orc, x, mx.Config(block=block, scale_fmt=fmt, rule=mx.RULE_MSE))
+
+
+@pytest.mark.parametrize("shape", [(128, 512), (256, 1024)])
+@pytest.mark.parametrize("sf_layout", [0, 1])
+def test_mse_nearest_format_alternation(mx, orc, shape, sf_layout):
+    """NVFP4 with the alternating global / group scale optimisation: the
+    tensor scale is a binary32 result of binary64 reductions summed in a
+    different order than the oracle's, so it is compared to 1e-5; given that
+    scale, the oracle's group step must reproduce the codes and scales
+    exactly.  The squared error is below plain NVFP4's; the workspace header
+    is left zero; the GEMM takes the operand like an NVFP4 one."""
+    rows, cols = shape
+    x = inputs.laplace_outlier_cols(rows, cols, seed=4, n_outlier_cols=8)
+    cfg = mx.Config(block=16, scale_fmt=mx.SCALE_UE4M3, rule=mx.RULE_MSE, tensor_scale=mx.TS_COMPUTE,
+                    sf_layout=sf_layout)
+    ws = mx.new_workspace(cfg, rows, cols, "cuda")
+    q = mx.quantize(x.cuda(), cfg, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:256].count_nonzero()) == 0
+    sT = float(q.tensor_scale.item())
+    o = orc.quantize(ocfg(orc, dataclasses.replace(cfg, sf_layout=0)), x)
+    assert sT == pytest.approx(o["tensor_scale"], rel=1e-5)
+    og = ocfg(orc, dataclasses.replace(cfg, tensor_scale=mx.TS_GIVEN, sf_layout=0))
+    r = orc.quantize(og, x, tensor_scale=sT)
+    S = cols // 16
+    if sf_layout:
+        from tests.test_gpu_gemm import chunk_layout
+        assert np.array_equal(q.scales.cpu().numpy(), chunk_layout(r["scales"], rows, S))
+    else:
+        assert np.array_equal(q.scales.cpu().numpy(), r["scales"])
+    assert np.array_equal(q.codes.cpu().numpy(), r["packed"].ravel())
+    oxh = orc.dequantize(og, r["packed"], r["scales"], sT, None, None, rows, cols)
+    assert_stats(q.stats.cpu().numpy(), orc.stats(r["y"], oxh)[0], rows * cols)
+    if not sf_layout:
+        assert_same_f32(mx.dequantize(q, torch.float32).cpu().numpy(), oxh, "dequantized")
+    plain = mx.quantize(x.cuda(), mx.Config(block=16, scale_fmt=mx.SCALE_UE4M3, rule=mx.RULE_NEAREST,
+                                            tensor_scale=mx.TS_COMPUTE)).stats.cpu().numpy()
+    assert q.stats.cpu().numpy()[1] < plain[1]
+    if sf_layout and rows % 128 == 0 and rows >= 256:
+        w = inputs.normal(256, cols, sigma=0.02, seed=7)
+        qw = mx.quantize(w.cuda(), dataclasses.replace(cfg, sf_layout=1))
+        c = mx.gemm(q, qw, out_dtype=torch.float32).cpu().numpy().astype(np.float64)
+        torch.cuda.synchronize()
+        assert mx.mx_device_status() == 0
+        rw = orc.quantize(og, w, tensor_scale=float(qw.tensor_scale.item()))
+        wh = orc.dequantize(og, rw["packed"], rw["scales"], float(qw.tensor_scale.item()), None, None, 256, cols)
+        ref = oxh.astype(np.float64) @ wh.astype(np.float64).T
+        assert np.linalg.norm(c - ref) / np.linalg.norm(ref) < 1e-3
 
 
 @pytest.mark.parametrize("elem", [0, 1, 2, 3, 4])
