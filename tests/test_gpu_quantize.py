@@ -195,6 +195,29 @@ def test_elements_and_rounding(mx, orc, elem, rule, asym, rnd, dtype):
     run_case(mx, orc, x, mx.Config(elem=elem, rule=rule, asymmetric=asym, round=rnd, seed=12345))
 
 
+@pytest.mark.parametrize("fmt", [1, 2])
+def test_measured_mse_follows_the_model(mx, fmt):
+    """The quantizer's measured MSE on 4096 x 4096 N(0, sigma^2) tensors
+    (nearest UE4M3 / UE5M3 scales, no tensor scale) against the expected-MSE
+    model, and the block-size inversion of narrow distributions with UE4M3
+    (absent with UE5M3)."""
+    from oracle import mse_model
+    name = "ue4m3" if fmt == 1 else "ue5m3"
+    got = {}
+    for sigma in (0.002, 0.02):
+        x = inputs.normal(4096, 4096, sigma=sigma, seed=1, dtype=torch.float32).cuda()
+        for block in (8, 16, 32):
+            st = mx.quantize(x, mx.Config(block=block, scale_fmt=fmt, rule=mx.RULE_NEAREST)).stats.cpu().numpy()
+            want = mse_model.expected_mse(sigma, block, name)["mse"]
+            assert st[5] == pytest.approx(want, rel=5e-3), (sigma, block, st[5], want)
+            got[sigma, block] = st[5]
+    if fmt == 1:
+        assert got[0.002, 8] > got[0.002, 16] > got[0.002, 32]
+    else:
+        assert got[0.002, 8] < got[0.002, 16] < got[0.002, 32]
+    assert got[0.02, 8] < got[0.02, 16] < got[0.02, 32]
+
+
 @pytest.mark.parametrize("block", [8, 16, 32])
 @pytest.mark.parametrize("fmt", [1, 2])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
