@@ -302,6 +302,7 @@ def run_ours(args, rank, world, device):
                 "traffic": traffic,
                 "traffic_launch": "MXFP4 on W (dram read + write per launch, from the ncu capture of the "
                                   "16384 x 8192 case scaled by elements)",
+                "traffic_launch_algorithmic_bytes": algo_bytes(mx.MXFP4, N_OUT, K_DIM, "q"),
                 "algorithmic_bytes_per_step": qbytes,
                 "by_variant_frac": {n: round(rows[n]["GB_per_s"] / pk["hbm_gbs"], 4) for n in qnames}}
 
@@ -411,18 +412,36 @@ def run_e2e(mx, A_cpu, W_cpu, plan, outs, device, args, step_bytes, world):
 
 def run_gemm(mx, A, W, device, args, world):
     """Block-scaled GEMM C = A^Q W^Q^T (MXFP4, NVFP4, MBS operands on the NVFP4
-    kind, MXFP6) and QSNR(AB)."""
+    kind, MXFP6, MXFP6 activations with MXFP4 weights, Hadamard-rotated MXFP4,
+    NVFP4 with MSE-optimised scales) and QSNR(AB)."""
     out = {}
     pk, pk_src = peaks()
     stream = torch.cuda.current_stream(device)
     flop = 2.0 * M_TOK * N_OUT * K_DIM
     mbs = mx.Config(macro_block=128)
-    for name, cfg in (("mxfp4", mx.Config(sf_layout=1)),
-                      ("nvfp4", mx.Config(block=16, scale_fmt=1, rule=3, tensor_scale=1, sf_layout=1)),
-                      ("mbs_mxfp4_via_nvf4", mbs),
-                      ("mxfp6_e2m3", mx.Config(elem=mx.E2M3, sf_layout=1))):
+    fp4 = mx.Config(sf_layout=1)
+    nv = mx.Config(block=16, scale_fmt=1, rule=3, tensor_scale=1, sf_layout=1)
+    nv_mse = mx.Config(block=16, scale_fmt=1, rule=mx.RULE_MSE, tensor_scale=1, sf_layout=1)
+    for name, cfg, cfg_w in (("mxfp4", fp4, fp4),
+                             ("nvfp4", nv, nv),
+                             ("mbs_mxfp4_via_nvf4", mbs, mbs),
+                             ("mxfp6_e2m3", mx.Config(elem=mx.E2M3, sf_layout=1), mx.Config(elem=mx.E2M3, sf_layout=1)),
+                             ("mxfp6_e2m3_x_mxfp4", mx.Config(elem=mx.E2M3, sf_layout=1), fp4),
+                             ("had32_mxfp4", mx.Config(hadamard=32, sf_layout=1), mx.Config(hadamard=32, sf_layout=1)),
+                             ("nvfp4_mse_scales", nv_mse, nv_mse)):
         qa = mx.quantize(A, cfg, stats=False)
-        qw = mx.quantize(W, cfg, stats=False)
+        if cfg_w.rule == mx.RULE_MSE:
+            # the alternating global / group scale search on W: an offline
+            # weight step, timed once here (not part of the GEMM time)
+            torch.cuda.synchronize(device)
+            s0, e0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            qw = mx.quantize(W, cfg_w, stats=False)
+            e0.record(stream)
+            torch.cuda.synchronize(device)
+            mse_quant_ms = s0.elapsed_time(e0)
+        else:
+            qw = mx.quantize(W, cfg_w, stats=False)
         if cfg.macro_block:
             # Macro Block Scaling operands: S_M X folded into UE4M3 16-element
             # scales, the GEMM's NVFP4 kind (the fold is outside the timed GEMM)
@@ -449,8 +468,9 @@ def run_gemm(mx, A, W, device, args, world):
         torch.cuda.synchronize(device)
         ms = s.elapsed_time(e) / steps
         tf = flop / (ms * 1e-3) / 1e12
-        # FP6 runs at the FP8 rate (kind::mxf8f6f4): nominal 2x bf16; FP4 4x
-        ratio = 2.0 if cfg.elem in (mx.E2M3, mx.E3M2) else 4.0
+        # FP6 runs at the FP8 rate (kind::mxf8f6f4, with an FP4 operand too):
+        # nominal 2x bf16; FP4 kinds 4x
+        ratio = 2.0 if mx.E2M3 in (cfg.elem, cfg_w.elem) or mx.E3M2 in (cfg.elem, cfg_w.elem) else 4.0
         peak = pk["bf16_tflops"] * ratio
         rec = {"TFLOPS": round(tf, 1), "ms": round(ms, 4), "unit": "TFLOP/s",
                "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(peak, 1),
@@ -468,6 +488,9 @@ def run_gemm(mx, A, W, device, args, world):
             rec["device_status"] = mx.mx_device_status()
         except mx.MXError as e:
             rec["qsnr_ab"] = f"unavailable: {e}"
+        if cfg_w.rule == mx.RULE_MSE:
+            rec["w_quantize_ms"] = round(mse_quant_ms, 3)
+            rec["w_quantize_note"] = "alternating global / group scale search on W (4 rounds + writing pass), once"
         out[name] = rec
     if "mxfp4" in out and "TFLOPS" in out.get("mbs_mxfp4_via_nvf4", {}):
         # the pages quote MBS's GEMM overhead against plain MXFP4
@@ -562,10 +585,12 @@ def kernel_case(args):
         M, N, K = M_TOK, N_OUT, K_DIM
         cfg = {"gemm_mxfp4": mx.Config(sf_layout=1),
                "gemm_nvfp4": mx.Config(block=16, scale_fmt=1, rule=3, tensor_scale=1, sf_layout=1),
-               "gemm_mxfp6": mx.Config(elem=mx.E2M3, sf_layout=1)}[case]
+               "gemm_mxfp6": mx.Config(elem=mx.E2M3, sf_layout=1),
+               "gemm_mxfp6_x_mxfp4": mx.Config(elem=mx.E2M3, sf_layout=1)}[case]
+        cfg_w = mx.Config(sf_layout=1) if case == "gemm_mxfp6_x_mxfp4" else cfg
         a = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
         w = (torch.randn(N, K, generator=g, device=dev) * 0.02).to(torch.bfloat16)
-        qa, qw = mx.quantize(a, cfg, stats=False), mx.quantize(w, cfg, stats=False)
+        qa, qw = mx.quantize(a, cfg, stats=False), mx.quantize(w, cfg_w, stats=False)
         c = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         run = lambda: mx.gemm(qa, qw, out=c)
         work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
@@ -581,7 +606,8 @@ def kernel_case(args):
                "quant_e2m1_sr_grad": mx.Config(round=mx.ROUND_STOCHASTIC, seed=5),
                "quant_e2m3_grad": mx.Config(elem=mx.E2M3),
                "quant_int4_asym_grad": mx.Config(elem=mx.INT4, asymmetric=1, rule=mx.RULE_CEIL),
-               "quant_e3m0_ceil_grad": mx.Config(elem=mx.E3M0, rule=mx.RULE_CEIL)}[case]
+               "quant_e3m0_ceil_grad": mx.Config(elem=mx.E3M0, rule=mx.RULE_CEIL),
+               "quant_nvfp4_mse_row": mx.Config(block=16, scale_fmt=1, rule=mx.RULE_MSE, tensor_scale=1)}[case]
         q = mx.quantize(x, cfg, stats=not args.no_stats)
         if case.startswith("dequant"):
             out = torch.empty(R, Cc, dtype=torch.bfloat16, device=dev)
