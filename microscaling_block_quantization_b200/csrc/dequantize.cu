@@ -228,6 +228,8 @@ __global__ void __launch_bounds__(kThreads) k_dequant_oct(const DParams p, const
 {
     constexpr int U = 4;
     const uint32_t T = gridDim.x * blockDim.x;
+    pdl_trigger();
+    pdl_wait();
     const float sT = (p.ts_mode != TS_NONE && p.tensor_scale) ? *p.tensor_scale : 1.0f;
     const bool nearest = p.sd.fmt != S_E8M0 && p.sd.rule == R_NEAREST;
     const int lb = __ffs(p.block) - 1;
@@ -315,14 +317,15 @@ int launch_dequant_oct(const DParams &p, cudaStream_t st)
 {
     const uint64_t noct = (uint64_t)(p.rows * p.cols / 8);
     const FastDiv f = make_fast_div((uint32_t)(p.cols / 8));
+    cudaError_t e;
     if (p.out_fp32) {
         const int g = grid_of(k_dequant_oct<AXIS, true>, (int64_t)(noct / 4 + 255) / 256 * 8);
-        k_dequant_oct<AXIS, true><<<g, kThreads, 0, st>>>(p, f, (uint32_t)noct);
+        e = launch_pdl(k_dequant_oct<AXIS, true>, g, kThreads, 0, st, p, f, (uint32_t)noct);
     } else {
         const int g = grid_of(k_dequant_oct<AXIS, false>, (int64_t)(noct / 4 + 255) / 256 * 8);
-        k_dequant_oct<AXIS, false><<<g, kThreads, 0, st>>>(p, f, (uint32_t)noct);
+        e = launch_pdl(k_dequant_oct<AXIS, false>, g, kThreads, 0, st, p, f, (uint32_t)noct);
     }
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    return e == cudaSuccess ? 0 : -1;
 }
 
 // Column axis with the rotation along columns: thread = 4 columns x `block`

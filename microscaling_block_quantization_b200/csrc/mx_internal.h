@@ -86,6 +86,34 @@ int device_sm_count();
 // the shared-memory attribute are host work that would otherwise sit between
 // short kernels); raises the kernel's dynamic shared-memory limit as needed.
 int cached_occupancy(const void *kernel, int threads, size_t smem);
+
+// Programmatic dependent launch: a CTA lets the next launch on the stream
+// start (its CTAs take SMs as this grid's CTAs retire) and, before its first
+// global access, waits until the preceding grid has completed with its
+// memory visible.  Both are no-ops for a kernel launched without the
+// programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launch with programmatic stream serialization (the kernel pairs it with
+// pdl_trigger / pdl_wait): the launch may begin while the previous kernel on
+// the stream drains.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                              cudaStream_t st, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
 int launch_quantize_col(const QParams &p, int axis, int in_fp32, int fast, cudaStream_t st,
                         int *grid_out);
 int launch_amax_col(const QParams &p, int in_fp32, cudaStream_t st);

@@ -254,16 +254,30 @@ __device__ __forceinline__ void finish_launch(const QParams &p, const Acc &a)
         s_last = atomicAdd(p.ticket, 1u) == gridDim.x - 1;
     }
     __syncthreads();
-    if (!s_last || threadIdx.x >= 32) return;
+    if (!s_last) return;
     __threadfence();
     if (p.partials) {
+        // every thread of the last CTA takes a strided share of the records,
+        // then warps, then the CTA (a fixed order for a given launch shape)
+        __shared__ double red[32][5];
         double s[5] = {0, 0, 0, 0, 0};
-        for (unsigned i = threadIdx.x; i < gridDim.x; i += 32)
+        for (unsigned i = threadIdx.x; i < gridDim.x; i += blockDim.x)
 #pragma unroll
             for (int k = 0; k < 5; ++k) s[k] += __ldcg(p.partials + (size_t)i * kPartialDoubles + k);
 #pragma unroll
         for (int k = 0; k < 5; ++k) s[k] = warp_sum(s[k]);
-        if (threadIdx.x == 0) store_stats(p.stats, s, p.count);
+        const int w = threadIdx.x >> 5;
+        if ((threadIdx.x & 31) == 0)
+#pragma unroll
+            for (int k = 0; k < 5; ++k) red[w][k] = s[k];
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double t[5] = {0, 0, 0, 0, 0};
+            for (int v = 0; v < (int)(blockDim.x >> 5); ++v)
+#pragma unroll
+                for (int k = 0; k < 5; ++k) t[k] += red[v][k];
+            store_stats(p.stats, t, p.count);
+        }
     }
     if (threadIdx.x == 0) {
         if (p.ts_mode == TS_COMPUTE) *p.amax_word = 0u;

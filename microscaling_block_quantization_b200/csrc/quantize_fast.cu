@@ -83,7 +83,9 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t nch = (uint32_t)(p.rows * p.cols / 32);
     const uint32_t ntiles = (nch + kConsumers - 1) / kConsumers;
+    pdl_trigger();
     if (threadIdx.x == 0) ring.init();
+    pdl_wait();
     const float sT = launch_tensor_scale(p);
     // nearest scales: s_b s_T and its reciprocal for every scale code, once per CTA
     __shared__ float2 near_tab[NEAR ? 256 : 1];
@@ -268,9 +270,9 @@ int launch_fast_b(const QParams &p, cudaStream_t st, int *grid_out)
     if (ring_map<InT>(&tm, p.x, nch) != 0) return -1;
     auto k = k_quant_fast<InT, B, STATS, HADN, MBS, NEAR>;
     const unsigned g = ring_grid(reinterpret_cast<const void *>(k), RingCfg<InT>::kSmem, nch);
-    k<<<g, kFastThreads, RingCfg<InT>::kSmem, st>>>(p, tm);
+    const cudaError_t e = launch_pdl(k, g, kFastThreads, RingCfg<InT>::kSmem, st, p, tm);
     *grid_out = (int)g;
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    return e == cudaSuccess ? 0 : -1;
 }
 
 // statistics on / off; nearest (UE4M3 / UE5M3) or power-of-two scales (the

@@ -176,7 +176,9 @@ __global__ void __launch_bounds__(kRingThreads, 2) k_quant_gen(const QParams p, 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t nch = (uint32_t)(p.rows * p.cols / 32);
     const uint32_t ntiles = (nch + kRingConsumers - 1) / kRingConsumers;
+    pdl_trigger();
     if (threadIdx.x == 0) ring.init();
+    pdl_wait();
     __syncthreads();
 
     Acc acc = {0, 0, 0, 0, 0};
@@ -358,9 +360,9 @@ int launch_gen_k(const QParams &p, cudaStream_t st, int *grid_out)
     if (ring_map<InT>(&tm, p.x, nch) != 0) return -1;
     auto k = k_quant_gen<InT, ELEM, RD, ASYM>;
     const unsigned g = ring_grid(reinterpret_cast<const void *>(k), RingCfg<InT>::kSmem, nch);
-    k<<<g, kRingThreads, RingCfg<InT>::kSmem, st>>>(p, tm);
+    const cudaError_t e = launch_pdl(k, g, kRingThreads, RingCfg<InT>::kSmem, st, p, tm);
     *grid_out = (int)g;
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    return e == cudaSuccess ? 0 : -1;
 }
 
 template <typename InT, int ELEM, bool ASYM>

@@ -304,6 +304,8 @@ __global__ void __launch_bounds__(kThreads) k_amax_vec(const QParams p)
     const uint4 *x = static_cast<const uint4 *>(p.x);
     const uint64_t nv = (uint64_t)(p.rows * p.cols) * sizeof(InT) / 16;
     const uint64_t T = (uint64_t)gridDim.x * blockDim.x;
+    pdl_trigger();
+    pdl_wait();
     float m = 0.0f;
     __nv_bfloat162 m2 = __float2bfloat162_rn(0.0f);
     for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv; i += U * T) {
@@ -436,16 +438,17 @@ int launch_quantize(const QParams &p, int axis, int in_fp32, int fast, cudaStrea
 
 int launch_tensor_amax(const QParams &p, int axis, int in_fp32, cudaStream_t st)
 {
+    cudaError_t e = cudaSuccess;
     if (axis == AX_COL && p.had) {
         if (launch_amax_col(p, in_fp32, st)) return -1;
     } else if (!p.had) {
         const int64_t warps = (p.rows * p.cols / 8 / 4 + 31) / 32;
         if (in_fp32) {
             const int g = grid_for(k_amax_vec<float>, warps);
-            k_amax_vec<float><<<g, kThreads, 0, st>>>(p);
+            e = launch_pdl(k_amax_vec<float>, g, kThreads, 0, st, p);
         } else {
             const int g = grid_for(k_amax_vec<__nv_bfloat16>, warps);
-            k_amax_vec<__nv_bfloat16><<<g, kThreads, 0, st>>>(p);
+            e = launch_pdl(k_amax_vec<__nv_bfloat16>, g, kThreads, 0, st, p);
         }
     } else {
         const int64_t tiles = (p.rows * p.cols / 32 + 31) / 32;
@@ -457,7 +460,7 @@ int launch_tensor_amax(const QParams &p, int axis, int in_fp32, cudaStream_t st)
             k_amax_row<__nv_bfloat16><<<g, kThreads, 0, st>>>(p);
         }
     }
-    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+    return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? 0 : -1;
 }
 
 int launch_finalize_stats(const double *partials, int nparts, double count, double *stats,
