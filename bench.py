@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-gemm", action="store_true")
+    ap.add_argument("--one-stream", action="store_true",
+                    help="capture the step on one stream (default: two streams, see run_ours)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-case", default=None,
                     help="run one kernel alone (for ncu captures): quant_mxfp4_row, quant_nvfp4_row, "
@@ -204,29 +206,68 @@ def run_ours(args, rank, world, device):
             outs[key] = torch.empty(x.shape, dtype=torch.bfloat16, device=device)
             outs[(key, "src")] = src
 
-    def run_call(name, t, cfg, kind):
+    # each stream owns a workspace: concurrent calls must not share control words
+    ws_main = mx.new_workspace(mx.MXFP4, *A.shape, device)
+    ws_side = mx.new_workspace(mx.MXFP4, *A.shape, device)
+
+    def run_call(name, t, cfg, kind, stream=None, ws=None):
         # stream=None: the current stream, i.e. the capture stream inside a graph
         key = (name, t)
         if kind == "q":
-            mx.quantize(T[t], cfg, out=outs[key])
+            mx.quantize(T[t], cfg, out=outs[key], stream=stream, workspace=ws_main if ws is None else ws)
         else:
-            mx.dequantize(outs[(key, "src")], out=outs[key])
+            mx.dequantize(outs[(key, "src")], out=outs[key], stream=stream)
+
+    # The step's launches are independent problems except that each
+    # dequantizer reads the MXFP4 codes of its tensor.  They are captured on
+    # two streams so that HBM-bound work (the NVFP4 tensor-amax passes, the
+    # dequantizers) overlaps issue-bound quantizers: the MXFP4 / rotated / MBS
+    # quantizers on the capture stream, NVFP4 and the dequantizers (after an
+    # event on their codes) on a side stream, each stream with its own
+    # workspace.
+    side = torch.cuda.Stream(device)
+    SIDE = {"nvfp4_row", "dequant_mxfp4_bf16"}
+
+    def run_step():
+        if args.one_stream:
+            for call in plan:
+                run_call(*call)
+            return
+        main = torch.cuda.current_stream(device)
+        fork = torch.cuda.Event()
+        fork.record(main)
+        side.wait_event(fork)
+        codes_ready = {}
+        for call in plan:
+            name, t, cfg, kind = call
+            if name in SIDE:
+                if kind == "d":
+                    side.wait_event(codes_ready[t])
+                with torch.cuda.stream(side):
+                    run_call(*call, stream=side, ws=ws_side)
+            else:
+                run_call(*call)
+                if name == "mxfp4_row":
+                    ev = torch.cuda.Event()
+                    ev.record(main)
+                    codes_ready[t] = ev
+        join = torch.cuda.Event()
+        join.record(side)
+        main.wait_event(join)
 
     step_bytes = sum(algo_bytes(cfg, *T[t].shape, kind) for _, t, cfg, kind in plan)
     launches = sum(launches_per_call(cfg, kind) for _, _, cfg, kind in plan)
 
-    # eager warm-up (allocates the workspace, caches kernel attributes)
+    # eager warm-up (caches kernel attributes)
     for _ in range(max(1, args.warmup)):
-        for call in plan:
-            run_call(*call)
+        run_step()
     torch.cuda.synchronize(device)
 
     # the step, and every launch of it, captured as CUDA graphs: the kernels
     # run back to back with no host work between them
     step_graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(step_graph):
-        for call in plan:
-            run_call(*call)
+        run_step()
     call_graphs = []
     for call in plan:
         g = torch.cuda.CUDAGraph()
@@ -360,45 +401,76 @@ def run_extra_rows(mx, A, device, args):
 
 def run_e2e(mx, A_cpu, W_cpu, plan, outs, device, args, step_bytes, world):
     """Same step through the public API, inputs copied from pinned host memory
-    and the codes, scales and stats read back, inside the timed region."""
-    stream = torch.cuda.current_stream(device)
+    and the codes, scales and stats read back, inside the timed region.  The
+    copies run on their own streams: A's results go back to the host while W
+    comes in and is quantized (PCIe is full duplex), and the next step's
+    inputs come in while the previous step's results go out.  Events order
+    every reuse of a device buffer."""
+    compute = torch.cuda.current_stream(device)
+    h2d, d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
     hA = A_cpu.pin_memory()
     hW = W_cpu.pin_memory()
     dA = torch.empty_like(hA, device=device)
     dW = torch.empty_like(hW, device=device)
     T = {"A": dA, "W": dW}
-    back = []
+    back = {"A": [], "W": []}
     for name, t, cfg, kind in plan:
         if kind == "q":
             o = outs[(name, t)]
-            back.append((o.codes, torch.empty(o.codes.shape, dtype=torch.uint8).pin_memory()))
-            back.append((o.scales, torch.empty(o.scales.shape, dtype=torch.uint8).pin_memory()))
-            back.append((o.stats, torch.empty(o.stats.shape, dtype=torch.float64).pin_memory()))
-    h2d = hA.numel() * 2 + hW.numel() * 2
-    d2h = sum(d.numel() * d.element_size() for d, _ in back)
+            for d in (o.codes, o.scales, o.stats):
+                back[t].append((d, torch.empty(d.shape, dtype=d.dtype).pin_memory()))
+    h2d_bytes = hA.numel() * 2 + hW.numel() * 2
+    d2h_bytes = sum(d.numel() * d.element_size() for t in back for d, _ in back[t])
+    host = {"A": hA, "W": hW}
+    # per tensor: inputs landed, launches done, results read back
+    ev = {(k, t): None for k in ("in", "done", "out") for t in ("A", "W")}
 
     def one():
-        dA.copy_(hA, non_blocking=True)
-        dW.copy_(hW, non_blocking=True)
-        for name, t, cfg, kind in plan:
-            if kind == "q":
-                mx.quantize(T[t], cfg, out=outs[(name, t)], stream=stream)
-            else:
-                mx.dequantize(outs[("mxfp4_row", t)], out=outs[(name, t)], stream=stream)
-        for d, h in back:
-            h.copy_(d, non_blocking=True)
+        for t in ("A", "W"):
+            if ev[("done", t)] is not None:
+                h2d.wait_event(ev[("done", t)])          # the previous step has read T[t]
+            with torch.cuda.stream(h2d):
+                T[t].copy_(host[t], non_blocking=True)
+            ev[("in", t)] = torch.cuda.Event()
+            ev[("in", t)].record(h2d)
+        for t in ("A", "W"):
+            compute.wait_event(ev[("in", t)])
+            if ev[("out", t)] is not None:
+                compute.wait_event(ev[("out", t)])       # the previous results are on the host
+            for name, tt, cfg, kind in plan:
+                if tt != t:
+                    continue
+                if kind == "q":
+                    mx.quantize(T[t], cfg, out=outs[(name, t)], stream=compute)
+                else:
+                    mx.dequantize(outs[("mxfp4_row", t)], out=outs[(name, t)], stream=compute)
+            ev[("done", t)] = torch.cuda.Event()
+            ev[("done", t)].record(compute)
+            d2h.wait_event(ev[("done", t)])
+            with torch.cuda.stream(d2h):
+                for d, h in back[t]:
+                    h.copy_(d, non_blocking=True)
+            ev[("out", t)] = torch.cuda.Event()
+            ev[("out", t)].record(d2h)
+
+    def drain():
+        for t in ("A", "W"):
+            compute.wait_event(ev[("out", t)])
 
     steps = max(3, args.steps // 4)
     for _ in range(2):
         one()
+    drain()
     torch.cuda.synchronize(device)
     if world > 1:
         torch.distributed.barrier()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(stream)
+    s.record(compute)
+    h2d.wait_event(s)
     for _ in range(steps):
         one()
-    e.record(stream)
+    drain()
+    e.record(compute)
     torch.cuda.synchronize(device)
     ms = s.elapsed_time(e) / steps
     if world > 1:
@@ -406,8 +478,9 @@ def run_e2e(mx, A_cpu, W_cpu, plan, outs, device, args, step_bytes, world):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
     return {"value": round(world * step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3),
-            "steps": steps}
+            "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes, "ms_per_step": round(ms, 3),
+            "steps": steps,
+            "overlap": "copy-in, compute and copy-out on three streams (A's results out while W comes in)"}
 
 
 def run_gemm(mx, A, W, device, args, world):
@@ -680,7 +753,11 @@ def main():
         "config": {"workload": WORKLOAD, "step": [f"{n}:{t}" for n, t, _, _ in step_plan(__import__("microscaling_block_quantization_b200"))],
                    "step_algorithmic_bytes": r["step_bytes"], "hbm_frac_of_8TBs": round(r["value"] / world / 8000, 4),
                    "l2": "inputs larger than L2 (A+W 176 MiB > 126 MB); consecutive launches alternate tensors",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "streams": "one" if args.one_stream else
+                              "two: MXFP4 / rotated / MBS quantizers on one stream, NVFP4 (tensor-amax pass + "
+                              "quantizer) and the dequantizers (after their codes) on a second, each with its "
+                              "own workspace; per-row figures are sequential single-launch replays"},
         "roofline": r["roofline"],
         "cpu_baseline": cpu,
         "e2e": r["e2e"],
