@@ -138,10 +138,10 @@ typedef struct {
                               scale j of a row holding S = cols / block scales, byte
                               ((r/128)*(S/4) + j/4)*512 + (r%32)*16 + ((r/32)%4)*4 + j%4,
                               the layout mx_gemm copies into tensor memory.  With FP6
-                              elements it also sets the code layout to the tensor core's
-                              operand form: every 16 codes of a row in 12 bytes (code i at
-                              bits [6i, 6i+6) of the little-endian group) and 4 zero bytes,
-                              still one byte per element; FP4 codes are unchanged */
+                              elements it also sets the code layout to the dense operand
+                              form: every 16 codes of a row in 12 bytes (code i at bits
+                              [6i, 6i+6) of the little-endian group), groups back to back,
+                              6 bits per element; FP4 codes are unchanged */
     uint64_t seed;         /* stochastic-rounding key */
 } mx_config;
 
@@ -170,7 +170,8 @@ int mx_query_sizes(const mx_config *cfg, int64_t rows, int64_t cols, mx_sizes *o
  * ([MXFP4-OAS] Sec.2/Sec.4, [FINER], [MX-TRAIN]).
  *   x          device, bf16 or fp32 (x_dtype), row-major, 16-byte aligned.
  *   codes      device out.  4-bit formats: rows x cols/2 bytes, element (r, 2j)
- *              in the low nibble of byte (r, j); FP6: rows x cols bytes.
+ *              in the low nibble of byte (r, j); FP6: rows x cols bytes, or
+ *              rows x cols x 3/4 in the dense form of cfg->sf_layout == 1.
  *              The layout is the same for every axis.
  *   scales     device out, one byte per block: row axis [rows][cols/B], column
  *              axis [rows/B][cols], 2D [rows/32][cols/32] (cfg->sf_layout == 0), or
@@ -301,12 +302,13 @@ int mx_qsnr(const void *x, int32_t x_dtype, const void *x_hat, int32_t x_hat_dty
  * MXFP4: block 32, E8M0 (ca/cb rule FLOOR, CEIL or OAS).  NVFP4: block 16,
  * UE4M3 NEAREST with tensor scales tsA/tsB (device floats; used when
  * ca/cb->tensor_scale != MX_TS_NONE, else 1).  MXFP6 ([MX-TRAIN]'s MX6;
- * tcgen05 kind::mxf8f6f4): E2M3 and / or E3M2 codes in the tensor-core
- * operand layout mx_quantize writes with sf_layout = 1 (16 codes in 12 bytes
- * + 4 zero bytes), block 32, E8M0; N % 256 == 0.  The same kind takes one
- * FP6 operand with one MXFP4 operand (E2M1 + E8M0 / 32, packed codes; the
- * packed operand's pointer 32-byte aligned): [MX-TRAIN]'s MX6 weights and
- * activations against MX4 gradients.  Operands rotated by mx_hadamard_quantize
+ * tcgen05 kind::mxf8f6f4): E2M3 and / or E3M2 codes in the dense form
+ * mx_quantize writes with sf_layout = 1 (16 codes in 12 bytes), block 32,
+ * E8M0; N % 256 == 0; the copy into shared memory widens them to the
+ * kind's one byte per element.  The same kind takes one FP6 operand with
+ * one MXFP4 operand (E2M1 + E8M0 / 32, packed codes): [MX-TRAIN]'s MX6
+ * weights and activations against MX4 gradients.  On this kind both operand
+ * pointers must be 32-byte aligned.  Operands rotated by mx_hadamard_quantize
  * are accepted when both carry the same rotation (cfg->hadamard), since
  * (A H)(B H)^T = A B^T ([BRIDGING] sec. 2.3: rotated operands into the FP4
  * GEMM).  Any other pair: MX_ERR_UNSUPPORTED.  C: device, bf16 or fp32

@@ -158,7 +158,9 @@ int64_t nmacro_of(const mx_config *c, int64_t rows, int64_t cols)
 
 int64_t codes_bytes_of(const mx_config *c, int64_t rows, int64_t cols)
 {
-    return (c->elem == MX_E2M3 || c->elem == MX_E3M2) ? rows * cols : rows * cols / 2;
+    // FP6: one byte per code, or 6 bits per code in the dense tensor-core form
+    if (c->elem == MX_E2M3 || c->elem == MX_E3M2) return c->sf_layout == 1 ? rows * cols / 4 * 3 : rows * cols;
+    return rows * cols / 2;
 }
 
 int cuda_ok(cudaError_t e) { return e == cudaSuccess ? MX_OK : MX_ERR_CUDA; }

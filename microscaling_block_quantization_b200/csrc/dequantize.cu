@@ -114,12 +114,14 @@ __global__ void __launch_bounds__(kThreads) k_dequant_chunk(const DParams p)
                 const uint4 u = reinterpret_cast<const uint4 *>(p.codes)[c];
                 w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
             } else {
-                const uint4 u0 = reinterpret_cast<const uint4 *>(p.codes)[2 * (size_t)c];
-                const uint4 u1 = reinterpret_cast<const uint4 *>(p.codes)[2 * (size_t)c + 1];
-                if (p.sf_gemm) {                    // tensor-core operand layout
-                    fp6_group_unpack(u0, w);
-                    fp6_group_unpack(u1, w + 4);
+                if (p.sf_gemm) {                    // dense tensor-core operand form
+                    uint4 g0, g1;
+                    fp6_load_dense(static_cast<const uint8_t *>(p.codes) + 24 * (size_t)c, g0, g1);
+                    fp6_group_unpack(g0, w);
+                    fp6_group_unpack(g1, w + 4);
                 } else {
+                    const uint4 u0 = reinterpret_cast<const uint4 *>(p.codes)[2 * (size_t)c];
+                    const uint4 u1 = reinterpret_cast<const uint4 *>(p.codes)[2 * (size_t)c + 1];
                     w[0] = u0.x; w[1] = u0.y; w[2] = u0.z; w[3] = u0.w;
                     w[4] = u1.x; w[5] = u1.y; w[6] = u1.z; w[7] = u1.w;
                 }

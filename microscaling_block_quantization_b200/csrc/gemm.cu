@@ -648,21 +648,23 @@ EncodeTiled encoder()
 }
 
 // rows x row_bytes operand, box of 128 rows x 128 bytes, 128-byte swizzle
-// elem_bits: 16 (bf16), 4 (packed E2M1) or 8 (FP6 codes, one per byte)
+// elem_bits: 16 (bf16), 4 (packed E2M1 bytes for kind::mxf4 / mxf4nvf4), or -4 / -6
+// (packed E2M1 / dense FP6, widened to one byte per element for kind::mxf8f6f4)
 bool make_map(CUtensorMap *m, const void *base, int rows, int K, int elem_bits, unsigned box_rows = 128)
 {
     EncodeTiled enc = encoder();
     if (!enc) return false;
-    if (elem_bits == -4) {
-        // packed E2M1 codes read for kind::mxf8f6f4: boxes of 128 elements
-        // (64 bytes) land as 128 bytes in shared memory, every 8 bytes of codes
-        // followed by 8 zero bytes
+    if (elem_bits == -4 || elem_bits == -6) {
+        // packed sub-byte codes read for kind::mxf8f6f4: a box of 128 elements
+        // (64 bytes of E2M1, 96 of FP6) lands as 128 bytes in shared memory,
+        // every group of 16 codes widened to 16 bytes (8 / 4 zero bytes added)
         const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-        const cuuint64_t strides[1] = {(cuuint64_t)K / 2};
+        const cuuint64_t strides[1] = {(cuuint64_t)K * (elem_bits == -4 ? 4 : 6) / 8};
         const cuuint32_t box[2] = {128u, box_rows};
         const cuuint32_t estr[2] = {1, 1};
-        return enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void *>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        return enc(m, elem_bits == -4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_16U6_ALIGN16B,
+                   2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     }
     const bool bf16 = elem_bits == 16;
@@ -707,12 +709,14 @@ int launch_p(const GParams &p, const void *A, const void *B, cudaStream_t st)
     int abits = 4, bbits = 4;
     GParams q = p;
     if (KIND == KIND_MXF6) {
-        // per operand: FP6 codes one per byte, or packed E2M1 expanded by the TMA
+        // per operand: dense FP6 (6 bits per code) or packed E2M1, both widened
+        // to one byte per element by the TMA; the transaction counts the
+        // packed bytes read
         const bool a4 = ((p.ab_fmt >> 7) & 7u) == kFmtE2M1, b4 = ((p.ab_fmt >> 10) & 7u) == kFmtE2M1;
-        abits = a4 ? -4 : 8;
-        bbits = b4 ? -4 : 8;
-        q.stage_tx = (uint32_t)((a4 ? KT::kABytes / 2 : KT::kABytes) + (b4 ? KT::kBBytes / 2 : KT::kBBytes) +
-                                KT::kSfaBytes + KT::kSfbBytes);
+        abits = a4 ? -4 : -6;
+        bbits = b4 ? -4 : -6;
+        q.stage_tx = (uint32_t)((a4 ? KT::kABytes / 2 : KT::kABytes / 4 * 3) +
+                                (b4 ? KT::kBBytes / 2 : KT::kBBytes / 4 * 3) + KT::kSfaBytes + KT::kSfbBytes);
     }
     if (!make_map(&ta, A, p.M, p.K, abits, 128) || !make_map(&tb, B, p.N, p.K, bbits, 256)) return MX_ERR_CUDA;
     const int smem = 1024 + kStagesP * KT::kStageBytes + 256;
@@ -818,9 +822,8 @@ int mx_gemm(const mx_config *ca, const mx_config *cb, const void *Aq, const uint
     if (kind == KIND_MXF6) {
         // MXFP6 (and FP6 x E2M1): the persistent 128 x 256 kernel only
         if (N % BNP) return MX_ERR_UNSUPPORTED;
-        // the expanding TMA form wants 32-byte aligned packed E2M1 operands
-        if ((ca->elem == MX_E2M1 && ((uintptr_t)Aq & 31u)) || (cb->elem == MX_E2M1 && ((uintptr_t)Bq & 31u)))
-            return MX_ERR_ALIGN;
+        // the widening TMA types want 32-byte aligned operands
+        if (((uintptr_t)Aq & 31u) || ((uintptr_t)Bq & 31u)) return MX_ERR_ALIGN;
         p.ab_fmt = fp6_formats(ca, cb);
         return c_dtype == MX_DT_BF16 ? launch_p<KIND_MXF6, EPI_BF16>(p, Aq, Bq, st)
                                      : launch_p<KIND_MXF6, EPI_F32>(p, Aq, Bq, st);

@@ -153,9 +153,11 @@ __device__ __forceinline__ float decode_elem(const ElemDesc &d, uint32_t code)
 }
 
 // FP6 codes of 32 elements, one per byte (4 per word, code j in byte j % 4
-// of word j / 4), <-> the tensor-core operand layout: each 16 codes packed
-// into 12 bytes (code i at bits [6i, 6i + 6) of the little-endian 96-bit
-// group), then 4 zero bytes.
+// of word j / 4), <-> the dense tensor-core operand form: each 16 codes
+// packed into 12 bytes (code i at bits [6i, 6i + 6) of the little-endian
+// 96-bit group; the fourth word of the uint4 is unused), a 32-code chunk in
+// 24 consecutive bytes.  The GEMM's TMA expands every 12-byte group to the
+// 16-byte shared-memory form of kind::mxf8f6f4 (4 zero bytes added).
 __device__ __forceinline__ uint4 fp6_group_pack(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3)
 {
     uint32_t c[16];
@@ -168,6 +170,21 @@ __device__ __forceinline__ uint4 fp6_group_pack(uint32_t w0, uint32_t w1, uint32
     r.z = (c[10] >> 4) | (c[11] << 2) | (c[12] << 8) | (c[13] << 14) | (c[14] << 20) | (c[15] << 26);
     r.w = 0u;
     return r;
+}
+// 24 bytes of a chunk's two groups at dst (8-byte aligned), and back
+__device__ __forceinline__ void fp6_store_dense(uint8_t *dst, uint4 g0, uint4 g1)
+{
+    uint2 *d = reinterpret_cast<uint2 *>(dst);
+    d[0] = make_uint2(g0.x, g0.y);
+    d[1] = make_uint2(g0.z, g1.x);
+    d[2] = make_uint2(g1.y, g1.z);
+}
+__device__ __forceinline__ void fp6_load_dense(const uint8_t *src, uint4 &g0, uint4 &g1)
+{
+    const uint2 *s = reinterpret_cast<const uint2 *>(src);
+    const uint2 a = s[0], b = s[1], c = s[2];
+    g0 = make_uint4(a.x, a.y, b.x, 0u);
+    g1 = make_uint4(b.y, c.x, c.y, 0u);
 }
 __device__ __forceinline__ void fp6_group_unpack(uint4 g, uint32_t w[4])
 {

@@ -314,10 +314,11 @@ __global__ void __launch_bounds__(kRingThreads, 2) k_quant_gen(const QParams p, 
                     reinterpret_cast<uint4 *>(p.codes)[c] = make_uint4(words[0], words[1], words[2], words[3]);
                 } else {
                     uint4 *dst = reinterpret_cast<uint4 *>(p.codes) + 2 * (size_t)c;
-                    if (p.sf_gemm) {                // tensor-core operand layout
-                        dst[0] = fp6_group_pack(words[0], words[1], words[2], words[3]);
-                        dst[NW > 4 ? 1 : 0] = fp6_group_pack(words[NW > 4 ? 4 : 0], words[NW > 4 ? 5 : 0],
-                                                             words[NW > 4 ? 6 : 0], words[NW > 4 ? 7 : 0]);
+                    if (p.sf_gemm) {                // dense tensor-core operand form, 24 bytes
+                        fp6_store_dense(static_cast<uint8_t *>(p.codes) + 24 * (size_t)c,
+                                        fp6_group_pack(words[0], words[1], words[2], words[3]),
+                                        fp6_group_pack(words[NW > 4 ? 4 : 0], words[NW > 4 ? 5 : 0],
+                                                       words[NW > 4 ? 6 : 0], words[NW > 4 ? 7 : 0]));
                     } else {
                         dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
                         dst[NW > 4 ? 1 : 0] = make_uint4(words[NW > 4 ? 4 : 0], words[NW > 4 ? 5 : 0],

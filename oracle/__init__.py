@@ -89,6 +89,8 @@ def lib():
         L.orc_scale_encode_nearest.argtypes = [C.c_int, C.c_float]
         L.orc_scale_encode_nearest.restype = C.c_uint8
         L.orc_fwht.argtypes = [C.c_int, P, C.c_int]
+        L.orc_packed_tc_bytes.argtypes = [C.c_int, i64, i64]
+        L.orc_packed_tc_bytes.restype = i64
         L.orc_tensor_scale.argtypes = [C.c_int, C.c_int, P, i64]
         L.orc_tensor_scale.restype = C.c_float
         L.orc_mse_grid_trace.argtypes = [C.c_int, C.c_int, P, C.c_int, i64, i64, C.c_int, P, P]
@@ -177,10 +179,10 @@ def pack(elem: int, codes: np.ndarray) -> np.ndarray:
 
 
 def pack_tc(elem: int, codes: np.ndarray) -> np.ndarray:
-    """Codes in the tensor-core operand layout (FP6: 16 codes in 12 bytes + 4
-    zero bytes; FP4 as `pack`)."""
+    """Codes in the tensor-core operand form (FP6: every 16 codes in 12
+    bytes, 6 bits each; FP4 as `pack`)."""
     rows, cols = codes.shape
-    nbytes = lib().orc_packed_bytes(elem, rows, cols)
+    nbytes = lib().orc_packed_tc_bytes(elem, rows, cols)
     out = np.zeros(nbytes, np.uint8)
     lib().orc_pack_tc(elem, _ptr(np.ascontiguousarray(codes)), rows, cols, _ptr(out))
     return out.reshape(rows, -1)

@@ -834,19 +834,26 @@ void orc_pack(int elem, const uint8_t *codes, int64_t rows, int64_t cols, uint8_
 
 void orc_unpack(int elem, const uint8_t *packed, int64_t rows, int64_t cols, uint8_t *codes);
 
-/* (READING) Tensor-core operand layout of FP6 codes (the library's
+/* (READING) Tensor-core operand form of FP6 codes (the library's
  * sf_layout = 1): every 16 consecutive codes of a row are packed into 12
- * bytes, code i at bits [6i, 6i + 6) of the little-endian 96-bit value,
- * followed by 4 zero bytes; 16 bytes per 16 elements.  The layout CUDA's
- * tensor-map documentation gives for 16 x U6 values in shared memory.  FP4
- * codes keep their packing (two per byte). */
+ * bytes, code i at bits [6i, 6i + 6) of the little-endian 96-bit value, the
+ * groups back to back: 6 bits per element, 12 bytes per 16.  That is the
+ * packed global form of CUDA's 16 x U6 tensor-map type, which the copy into
+ * shared memory widens to 16 bytes per group.  FP4 codes keep their packing
+ * (two per byte). */
+int64_t orc_packed_tc_bytes(int elem, int64_t rows, int64_t cols)
+{
+    grid_t g; make_grid(elem, 0, &g);
+    return g.bits == 6 ? rows * cols / 16 * 12 : rows * (cols / 2);
+}
+
 void orc_pack_tc(int elem, const uint8_t *codes, int64_t rows, int64_t cols, uint8_t *packed)
 {
     grid_t g; make_grid(elem, 0, &g);
     if (g.bits != 6) { orc_pack(elem, codes, rows, cols, packed); return; }
     for (int64_t i0 = 0; i0 < rows * cols; i0 += 16) {
-        uint8_t *dst = packed + i0;
-        memset(dst, 0, 16);
+        uint8_t *dst = packed + i0 / 16 * 12;
+        memset(dst, 0, 12);
         for (int i = 0; i < 16; i++) {
             unsigned v = codes[i0 + i] & 0x3fu;
             for (int b = 0; b < 6; b++)
@@ -859,13 +866,15 @@ void orc_unpack_tc(int elem, const uint8_t *packed, int64_t rows, int64_t cols, 
 {
     grid_t g; make_grid(elem, 0, &g);
     if (g.bits != 6) { orc_unpack(elem, packed, rows, cols, codes); return; }
-    for (int64_t i0 = 0; i0 < rows * cols; i0 += 16)
+    for (int64_t i0 = 0; i0 < rows * cols; i0 += 16) {
+        const uint8_t *src = packed + i0 / 16 * 12;
         for (int i = 0; i < 16; i++) {
             unsigned v = 0;
             for (int b = 0; b < 6; b++)
-                if (packed[i0 + (6 * i + b) / 8] & (1u << ((6 * i + b) % 8))) v |= 1u << b;
+                if (src[(6 * i + b) / 8] & (1u << ((6 * i + b) % 8))) v |= 1u << b;
             codes[i0 + i] = (uint8_t)v;
         }
+    }
 }
 
 void orc_unpack(int elem, const uint8_t *packed, int64_t rows, int64_t cols, uint8_t *codes)

@@ -201,18 +201,20 @@ def test_philox_known_answers(orc):
 
 
 def test_fp6_tensor_core_layout(orc):
-    """FP6 codes in the tensor-core operand layout: 16 codes per 16 bytes,
-    code i at bits [6i, 6i + 6) of the little-endian 96-bit group, 4 zero
-    bytes; checked against an integer construction, and the round trip."""
+    """FP6 codes in the dense tensor-core operand form: 16 codes per 12
+    bytes, code i at bits [6i, 6i + 6) of the little-endian 96-bit group,
+    groups back to back (6 bits per element); checked against an integer
+    construction, and the round trip."""
     rng = np.random.default_rng(5)
     codes = rng.integers(0, 64, size=(4, 64), dtype=np.uint8)
-    got = orc.pack_tc(2, codes).reshape(-1, 16)
+    got = orc.pack_tc(2, codes)
+    assert got.size == codes.size * 6 // 8
+    got = got.reshape(-1, 12)
     flat = codes.reshape(-1, 16)
     for g in range(flat.shape[0]):
         v = 0
         for i in range(16):
             v |= int(flat[g, i]) << (6 * i)
-        want = list(v.to_bytes(12, "little")) + [0, 0, 0, 0]
-        assert list(got[g]) == want
+        assert list(got[g]) == list(v.to_bytes(12, "little"))
     assert np.array_equal(orc.unpack_tc(3, orc.pack_tc(3, codes), 4, 64), codes)
     assert np.array_equal(orc.pack_tc(0, codes & 15), orc.pack(0, codes & 15))   # FP4 unchanged
