@@ -102,9 +102,13 @@ struct Ring {
         constexpr uint32_t S = RingCfg<InT>::kStages;
         return ring_wait(&full[i % S], (i / S) & 1, where);
     }
-    // consumer warp: every lane has read its chunk of the i-th tile
+    // consumer warp: every lane has read its chunk of the i-th tile.  The
+    // slot's next fill is an async-proxy (TMA) write, so each lane's
+    // generic-proxy reads are ordered before it by a proxy fence ahead of the
+    // arrive.
     __device__ __forceinline__ void release(uint32_t i) const
     {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if ((threadIdx.x & 31) == 0)
             asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];"
