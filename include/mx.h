@@ -192,7 +192,7 @@ int mx_query_sizes(const mx_config *cfg, int64_t rows, int64_t cols, mx_sizes *o
  *              words: one launch per call (two with a computed tensor scale:
  *              the amax pre-pass, then the quantizer).
  * Shapes: cols % 32 == 0 always (lanes walk rows in 32-element chunks),
- * rows * cols < 2^36, cols % block == 0 (row), rows % block == 0 (column),
+ * rows * cols < 2^32, cols % block == 0 (row), rows % block == 0 (column),
  * rows % 32 == 0 (2D), % 128 along the axis for MBS.  Block non-finite
  * values give the NaN scale code and zero element codes.
  */
@@ -285,8 +285,9 @@ int mx_dequantize(const mx_config *cfg, const void *codes, const uint8_t *scales
  * mx_qsnr -- fidelity reductions of x_hat against x ([MXFP4-OAS] Sec.3 Eq. (1);
  * [MX-TRAIN] R-MSE; [FINER] per-block MSE): stats as above, and when
  * per_block_mse != NULL the mean squared error of every block of the given
- * block size and axis (layout of `scales`).  x, x_hat: device, bf16 or fp32.
- * Reduction order is fixed: results are reproducible run to run.
+ * block size and axis (layout of `scales`).  x, x_hat: device, bf16 or fp32;
+ * rows * cols < 2^32.  Reduction order is fixed: results are reproducible
+ * run to run.
  */
 int64_t mx_qsnr_workspace_bytes(int64_t rows, int64_t cols);
 int mx_qsnr(const void *x, int32_t x_dtype, const void *x_hat, int32_t x_hat_dtype, int64_t rows,

@@ -123,8 +123,8 @@ int check_config(const mx_config *c, int64_t rows, int64_t cols, bool want_had)
     if (rows == 0 || cols == 0) return MX_OK;
     // kernels walk rows in 32-element chunks (one per lane)
     if (cols % 32) return MX_ERR_INVALID;
-    // fewer than 2^31 chunks: 32-bit chunk indices and TMA coordinates
-    if (rows > ((INT64_C(1) << 36) - 1) / cols) return MX_ERR_INVALID;
+    // fewer than 2^32 elements: 32-bit element, code-word and block indices
+    if (rows > (kMaxElements - 1) / cols) return MX_ERR_INVALID;
     if (c->axis == MX_AXIS_ROW && cols % B) return MX_ERR_INVALID;
     if (c->sf_layout == 1 && (rows % 128 || (cols / B) % 4)) return MX_ERR_INVALID;
     if (c->axis == MX_AXIS_COL && rows % B) return MX_ERR_INVALID;
@@ -367,6 +367,7 @@ int mx_qsnr(const void *x, int32_t x_dtype, const void *x_hat, int32_t x_hat_dty
             void *workspace, int64_t workspace_bytes, void *stream)
 {
     if (rows < 0 || cols < 0 || !stats) return MX_ERR_INVALID;
+    if (cols > 0 && rows > (kMaxElements - 1) / cols) return MX_ERR_INVALID;
     if ((x_dtype != MX_DT_BF16 && x_dtype != MX_DT_FP32) ||
         (x_hat_dtype != MX_DT_BF16 && x_hat_dtype != MX_DT_FP32))
         return MX_ERR_INVALID;

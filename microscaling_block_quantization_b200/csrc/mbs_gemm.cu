@@ -105,7 +105,7 @@ extern "C" int mx_mbs_gemm_scales(const mx_config *cfg, const uint8_t *scales, c
         cfg->axis != MX_AXIS_ROW || cfg->asymmetric || cfg->sf_layout != 0 || cfg->hadamard)
         return MX_ERR_UNSUPPORTED;
     if (rows <= 0 || cols <= 0 || rows % 128 || cols % 128) return MX_ERR_INVALID;
-    if (rows > ((INT64_C(1) << 36) - 1) / cols || rows >= (INT64_C(1) << 31)) return MX_ERR_INVALID;
+    if (rows > (kMaxElements - 1) / cols) return MX_ERR_INVALID;
     if (workspace_bytes < kWsHeader) return MX_ERR_WORKSPACE;
     if (((uintptr_t)workspace & 15u) || ((uintptr_t)sf16 & 15u) || ((uintptr_t)tensor_scale & 3u))
         return MX_ERR_ALIGN;

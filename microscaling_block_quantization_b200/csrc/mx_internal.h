@@ -15,6 +15,9 @@ constexpr int kPartialDoubles = 8;
 // tensor-amax accumulator at byte 0, the launch ticket at byte 64.  Both are
 // zero before a launch and the launch's last CTA leaves them zero.
 constexpr int64_t kWsHeader = 256;
+// Largest tensor a call takes (elements, exclusive): the kernels index
+// elements, 8-element code words and blocks in 32 bits.
+constexpr int64_t kMaxElements = INT64_C(1) << 32;
 constexpr int64_t kWsTicket = 64;
 // the MSE rule's tensor scale of each alternation round (floats, cleared by
 // the call that used them)

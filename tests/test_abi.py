@@ -136,6 +136,18 @@ def test_sharding_entry_points_checked_on_host(mx):
     assert mx.mx_stats_finalize(P(4100), None) == -3
 
 
+def test_element_limit_checked_on_host(mx):
+    """Calls take fewer than 2^32 elements (32-bit indices in the kernels)."""
+    P = C.c_void_p
+    s = mx.mx_sizes()
+    assert mx.lib().mx_query_sizes(C.byref(mx.MXFP4.c()), 1 << 16, (1 << 16) - 32, C.byref(s)) == 0
+    assert mx.lib().mx_query_sizes(C.byref(mx.MXFP4.c()), 1 << 16, 1 << 16, C.byref(s)) == -1
+    assert mx.mx_quantize(mx.MXFP4, P(4096), 0, 1 << 17, 1 << 15, P(4096), P(4096), None, None, None, None,
+                          None, 0, None) == -1
+    ws = 1 << 20
+    assert mx.mx_qsnr(P(4096), 0, P(4096), 0, 1 << 17, 1 << 15, 0, 0, P(4096), None, P(4096), ws, None) == -1
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     import microscaling_block_quantization_b200 as m
     monkeypatch.setattr(m, "_lib", None)
