@@ -308,7 +308,9 @@ def quantize(x: torch.Tensor, cfg: Config = MXFP4, *, stats: bool = True,
     """Block-quantize a 2-D bf16/fp32 CUDA tensor (``mx_quantize``, or
     ``mx_hadamard_quantize`` when ``cfg.hadamard`` is set).  ``workspace``:
     a caller's scratch (uint8, at least ``query_sizes(...).workspace_bytes``,
-    control words zero), needed with ``TS_AMAX`` to carry the amax."""
+    control words zero), needed with ``TS_AMAX`` to carry the amax.  Without
+    it the call uses one scratch per device, so calls that may run at the
+    same time on different streams must each pass their own."""
     _cuda2d(x, "x")
     rows, cols = x.shape
     q = out if out is not None else alloc_outputs(cfg, rows, cols, x.device, stats, rotated,

@@ -471,6 +471,36 @@ def test_qsnr_and_per_block_mse(mx, orc, axis, block):
     assert_stats(st2.cpu().numpy(), ost2, x.numel())
 
 
+def test_concurrent_streams_with_own_workspaces(mx):
+    """Quantizer calls running at the same time on two streams, each with its
+    own workspace (control words and statistics records), give exactly the
+    results of the same calls one after the other."""
+    a = inputs.laplace_outlier_cols(2048, 4096, seed=4).cuda()
+    w = inputs.normal(4096, 4096, sigma=0.02, seed=7).cuda()
+    cfgs = [mx.MXFP4, mx.NVFP4, mx.Config(hadamard=32)]
+    ref = [(mx.quantize(x, c), c) for c in cfgs for x in (a, w)]
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    w1, w2 = mx.new_workspace(mx.MXFP4, 1, 32, "cuda"), mx.new_workspace(mx.MXFP4, 1, 32, "cuda")
+    outs = []
+    for _ in range(3):
+        for c in cfgs:
+            with torch.cuda.stream(s1):
+                q1 = mx.quantize(a, c, stream=s1, workspace=w1)
+            with torch.cuda.stream(s2):
+                q2 = mx.quantize(w, c, stream=s2, workspace=w2)
+            outs += [q1, q2]
+    torch.cuda.synchronize()
+    assert mx.mx_device_status() == 0
+    for k, q in enumerate(outs):
+        r, _ = ref[k % len(ref)]
+        assert torch.equal(q.codes, r.codes) and torch.equal(q.scales, r.scales)
+        assert torch.equal(q.tensor_scale, r.tensor_scale)
+        assert np.array_equal(q.stats.cpu().numpy(), r.stats.cpu().numpy())
+    for ws in (w1, w2):
+        assert int(ws[:256].count_nonzero()) == 0
+
+
 def test_stats_reproducible(mx):
     x = inputs.laplace_outlier_cols(512, 1024, seed=4).cuda()
     a = mx.quantize(x, mx.MXFP4).stats.cpu().numpy()
