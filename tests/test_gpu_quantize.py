@@ -402,7 +402,8 @@ def test_special_values(mx, orc):
         run_case(mx, orc, x, mx.Config(**cfg), check_stats=False)
     x16 = torch.from_numpy(pats.view(np.int16)).view(torch.bfloat16)      # 2048 x 32, 16-blocks
     for cfg in (dict(block=16, scale_fmt=1, rule=3), dict(block=16, scale_fmt=2, rule=3),
-                dict(block=16, scale_fmt=1, rule=0)):
+                dict(block=16, scale_fmt=1, rule=0), dict(block=16, scale_fmt=1, rule=4),
+                dict(block=32, scale_fmt=2, rule=4), dict(rule=4), dict(elem=4, asymmetric=1, rule=1)):
         run_case(mx, orc, x16, mx.Config(**cfg), check_stats=False)
 
 
