@@ -17,7 +17,7 @@
 //   warps 2..5   epilogue: tcgen05.ld of the accumulator lanes of their
 //                quadrant, per-tensor scales, and either the C store or the
 //                QSNR sums against a previously computed C_q.
-// No TMA multicast anywhere; every wait on an mbarrier is bounded and sets a
+// Every TMA load targets its own CTA only; every wait on an mbarrier is bounded and sets a
 // device status word instead of hanging.
 #include <cuda.h>
 #include <cuda_bf16.h>
