@@ -420,6 +420,7 @@ __device__ __forceinline__ float div_by_recip(float a, float b, float y)
 struct NearScale {
     float maxv, r_max;      // largest element magnitude and RN(1 / maxv)
     float sT, r_T;          // tensor scale and RN(1 / sT); r_T = 0: IEEE division
+    float c;                // UE4M3 shortcut: RN(1 / RN(maxv sT)), or 0 (no shortcut)
     const float2 *tab;      // per scale code: {RN(s_b sT), RN(1 / RN(s_b sT))}; NaN code: {NaN, 0}
 };
 
@@ -427,15 +428,32 @@ struct NearScale {
 // s_b = RTNE((alpha / max) / s_T) through div_by_recip; the dequantization
 // factor s_b s_T (in deq) and the element multiplier from the launch's table.
 // A zero block: s_b = 0 (1/0 = +inf).
+//
+// UE4M3 shortcut: v = RN(alpha c) with c = RN(1 / RN(maxv sT)) is within
+// 5 ulp of the two-quotient value w (each of the three roundings in v and the
+// two in w is at most half an ulp, relative 2^-24, and the ulp of a binade
+// is at least 2^-24 of its values), so when v lies in E4M3's normal range and
+// more than 6 ulp from a rounding midpoint of E4M3 (mantissa bits below the
+// top 3 equal to 1000...0, i.e. low 20 bits 0x80000), v and w round to the
+// same code; every other block takes the two quotients.
 __device__ __forceinline__ BlockScale near_block_scale(const ScaleDesc &s, const NearScale &ns, float alpha,
                                                        int nonfinite)
 {
     BlockScale r;
-    const float q1 = div_by_recip(alpha, ns.maxv, ns.r_max);
-    const float sb_real = ns.sT == 1.0f ? q1
-                        : ns.r_T != 0.0f ? div_by_recip(q1, ns.sT, ns.r_T) : __fdiv_rn(q1, ns.sT);
-    r.code = nonfinite ? (uint32_t)s.ue_nan_code
-                       : (s.fmt == S_UE4M3) ? ue4m3_encode_hw(sb_real) : ue_encode_rtne(s, sb_real);
+    uint32_t code;
+    const float v = __fmul_rn(alpha, ns.c);
+    const uint32_t mid = (__float_as_uint(v) & 0xfffffu) - 0x80000u + 6u;
+    if (s.fmt == S_UE4M3 && v >= 0x1p-6f && v <= 0x1p100f && mid > 12u) {
+        uint16_t h;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(0.0f), "f"(v));
+        code = h & 0xffu;
+    } else {
+        const float q1 = div_by_recip(alpha, ns.maxv, ns.r_max);
+        const float sb_real = ns.sT == 1.0f ? q1
+                            : ns.r_T != 0.0f ? div_by_recip(q1, ns.sT, ns.r_T) : __fdiv_rn(q1, ns.sT);
+        code = (s.fmt == S_UE4M3) ? ue4m3_encode_hw(sb_real) : ue_encode_rtne(s, sb_real);
+    }
+    r.code = nonfinite ? (uint32_t)s.ue_nan_code : code;
     const float2 t = ns.tab[r.code];
     r.deq = t.x;
     r.inv = t.y;

@@ -101,6 +101,11 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) 
     ns.r_max = __fdiv_rn(1.0f, p.ed.maxv);
     ns.sT = sT;
     ns.r_T = (sT >= 0x1p-125f && sT <= 0x1p125f) ? __fdiv_rn(1.0f, sT) : 0.0f;
+    {
+        // the UE4M3 shortcut's constant, when max_elem s_T and its reciprocal are normal
+        const float ms = __fmul_rn(p.ed.maxv, sT);
+        ns.c = (ms >= 0x1p-125f && ms <= 0x1p125f) ? __fdiv_rn(1.0f, ms) : 0.0f;
+    }
     ns.tab = near_tab;
 
     Acc acc = {0, 0, 0, 0, 0};
