@@ -21,7 +21,8 @@
  *                 minimum 2^-17, per-tensor FP32 scale (UE4M3-S).
  *   [BRIDGING]   "Bridging the Gap Between Promise and Performance for
  *                 Microscaling FP4 Quantization": sec. 2.1/2.2 block-wise
- *                 Hadamard rotation before quantization.
+ *                 Hadamard rotation before quantization, MSE-optimised
+ *                 grids (alternating global / group scales).
  *   [MX-TRAIN]   fmread summary of Yang et al., "MX quantization for LLM
  *                 training" (ARITH 2025): element types E2M1/E3M0/INT4,
  *                 RTNE / Ceil / stochastic rounding, asymmetric scaling,
@@ -32,8 +33,9 @@
  *
  * Precision: every decision that produces an integer code (scale exponent,
  * element code) is taken with single IEEE binary32 operations in the order
- * written here (compile with -ffp-contract=off, no fast-math); the fidelity
- * reductions are accumulated in binary64.
+ * written here (compile with -ffp-contract=off, no fast-math), except the
+ * MSE rules, which compare block squared errors summed in binary64 in
+ * element order; the fidelity reductions are accumulated in binary64.
  *
  * Parity status of each function is stated beside it: "pinned" functions are
  * checked by the CPU tests against values fixed by the pages or by
