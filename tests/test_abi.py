@@ -148,6 +148,37 @@ def test_element_limit_checked_on_host(mx):
     assert mx.mx_qsnr(P(4096), 0, P(4096), 0, 1 << 17, 1 << 15, 0, 0, P(4096), None, P(4096), ws, None) == -1
 
 
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/mx.h compiles as strict C11 (no C++ in the boundary), and a C
+    program calling every declared entry point links against the library."""
+    import re
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no gcc")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    hdr = open(os.path.join(root, "include", "mx.h")).read()
+    names = sorted(set(re.findall(r"^\s*(?:int|int64_t|const char \*)\s*\**(mx_\w+)\(", hdr, re.M)))
+    assert "mx_quantize" in names and "mx_gemm_qsnr" in names
+    src = tmp_path / "use.c"
+    src.write_text('#include "mx.h"\n#include <stdio.h>\ntypedef void (*fn)(void);\n'
+                   + "static const fn all[] = {" + ", ".join(f"(fn){n}" for n in names) + "};\n"
+                   + "int main(void) {\n    unsigned i, k = 0;\n"
+                   + "    for (i = 0; i < sizeof all / sizeof all[0]; ++i) k += all[i] != 0;\n"
+                   + '    printf("%u\\n", k);\n    return 0;\n}\n')
+    lib = os.path.dirname(mx_lib_path())
+    cmd = ["gcc", "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(root, "include"),
+           "-I", "/usr/local/cuda/include", str(src), "-o", str(tmp_path / "use"), "-L", lib, "-lmx_b200",
+           "-Wl,--unresolved-symbols=ignore-in-shared-libs"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
+def mx_lib_path():
+    import microscaling_block_quantization_b200 as m
+    return m.LIB_PATH
+
+
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     import microscaling_block_quantization_b200 as m
     monkeypatch.setattr(m, "_lib", None)
