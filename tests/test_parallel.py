@@ -104,12 +104,14 @@ def _free_port():
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("case", sorted(CASES))
-def test_two_rank_bands_equal_the_whole_tensor(case):
+@pytest.mark.parametrize("case,world", [(c, 2) for c in sorted(CASES)] + [("nvfp4_row", 3), ("mxfp4_2d", 3)])
+def test_rank_bands_equal_the_whole_tensor(case, world):
+    """Two ranks, and three with uneven bands (96 rows of 1-row units; 160
+    rows of 32-row units: 64 / 64 / 32)."""
     ctx = mp.get_context("spawn")
     out = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, 2, port, case, out)) for r in range(2)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, case, out)) for r in range(world)]
     for p in procs:
         p.start()
     res = [out.get(timeout=120) for _ in procs]
