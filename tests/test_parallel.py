@@ -106,8 +106,8 @@ def _free_port():
 
 @pytest.mark.parametrize("case,world", [(c, 2) for c in sorted(CASES)] + [("nvfp4_row", 3), ("mxfp4_2d", 3)])
 def test_rank_bands_equal_the_whole_tensor(case, world):
-    """Two ranks, and three with uneven bands (96 rows of 1-row units; 160
-    rows of 32-row units: 64 / 64 / 32)."""
+    """Two ranks, and three (96 rows: 32 each; 160 rows in 32-row units:
+    uneven bands of 64 / 64 / 32)."""
     ctx = mp.get_context("spawn")
     out = ctx.Queue()
     port = _free_port()
