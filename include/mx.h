@@ -219,8 +219,11 @@ int mx_quantize(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t ro
  *   capture.  Every call shares the one array (zero at load; every call
  *   leaves its control words zero), so calls that overlap on the
  *   GPU -- on different streams, or from different threads -- race: order them
- *   on one stream.  Rotation (mx_hadamard_quantize) is not covered, nor
- *   MX_TS_AMAX (its amax word is in a caller's workspace): MX_ERR_UNSUPPORTED.
+ *   on one stream.  A call that returns MX_ERR_CUDA queues a reset of the
+ *   array's control words on `stream` before it returns.  Rotation
+ *   (cfg->hadamard != 0, the mx_hadamard_quantize entry) is not covered, nor
+ *   MX_TS_AMAX (its amax word is in a caller's workspace): MX_ERR_UNSUPPORTED,
+ *   checked on the host before anything is queued.
  */
 int mx_quantize_noalloc(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t rows,
                         int64_t cols, void *codes, uint8_t *scales, float *tensor_scale,

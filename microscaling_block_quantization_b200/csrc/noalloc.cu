@@ -51,8 +51,9 @@ extern "C" int mx_quantize_noalloc(const mx_config *cfg, const void *x, int32_t 
     mx_sizes s;
     int rc = mx_query_sizes(cfg, rows, cols, &s);
     if (rc != MX_OK) return rc;
-    // a given amax lives in a caller's workspace, which this entry has none of
-    if (cfg->tensor_scale == MX_TS_AMAX) return MX_ERR_UNSUPPORTED;
+    // a given amax lives in a caller's workspace, which this entry has none
+    // of; rotation (mx_hadamard_quantize) is a separate entry point
+    if (cfg->tensor_scale == MX_TS_AMAX || cfg->hadamard) return MX_ERR_UNSUPPORTED;
     if (s.workspace_bytes > kScratchBytes) return MX_ERR_WORKSPACE;
     void *scratch = nullptr;
     rc = scratch_for_current_device(&scratch);
@@ -60,6 +61,14 @@ extern "C" int mx_quantize_noalloc(const mx_config *cfg, const void *x, int32_t 
     // The scratch needs no clearing: its control words are zero at load and
     // every call leaves them zero, and every statistics record a call reads is
     // written earlier in the same call.
-    return mx_quantize(cfg, x, x_dtype, rows, cols, codes, scales, tensor_scale, macro_scales, offsets,
-                       stats, scratch, kScratchBytes, stream);
+    rc = mx_quantize(cfg, x, x_dtype, rows, cols, codes, scales, tensor_scale, macro_scales, offsets,
+                     stats, scratch, kScratchBytes, stream);
+    // A launch that failed after an earlier one of the same call was queued
+    // (the tensor-amax pass, an MSE round) can leave a control word set, and
+    // unlike a caller's workspace nobody else can clear this one: queue a
+    // reset of the 256-byte header behind whatever did run (a memset node,
+    // no allocation).
+    if (rc == MX_ERR_CUDA)
+        (void)cudaMemsetAsync(scratch, 0, mxk::kWsHeader, static_cast<cudaStream_t>(stream));
+    return rc;
 }

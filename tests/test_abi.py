@@ -130,6 +130,10 @@ def test_sharding_entry_points_checked_on_host(mx):
                           None, 0, None) == -5
     assert mx.mx_quantize_noalloc(amax_cfg, P(4096), 0, 64, 64, P(4096), P(4096), P(4096), None, None,
                                   None, None) == -2
+    # rotation is not covered by the no-alloc entry: unsupported, not invalid
+    for n in (16, 32):
+        assert mx.mx_quantize_noalloc(mx.Config(hadamard=n), P(4096), 0, 64, 64, P(4096), P(4096), None,
+                                      None, None, P(4096), None) == -2
     assert mx.mx_quantize(mx.Config(block=16, scale_fmt=mx.SCALE_UE4M3, rule=mx.RULE_NEAREST, tensor_scale=4),
                           P(4096), 0, 64, 64, P(4096), P(4096), P(4096), None, None, None, None, 0, None) == -1
     assert mx.mx_stats_finalize(None, None) == -1

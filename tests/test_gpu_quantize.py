@@ -61,13 +61,20 @@ def assert_stats(g, o, n):
     assert g[3] == o[3] and g[4] == o[4] and g[10] == o[10]
 
 
-def run_case(mx, orc, x_cpu, cfg, check_stats=True, given_ts=None):
+def run_case(mx, orc, x_cpu, cfg, check_stats=True, given_ts=None, want_rotated=None, bf16_out=False):
+    """Quantize on the GPU and with the oracle; compare every output.
+    want_rotated: ask the library for the rotated tensor y too (default: when
+    the config rotates).  Without it, a rotation with blocks of 16 or 32 runs
+    on the TMA-fed quantizer, with it on the lane-per-chunk kernel.
+    bf16_out: also compare the bf16 dequantized tensor."""
     rows, cols = x_cpu.shape
     x = x_cpu.cuda()
     ts_in = None
     if given_ts is not None:
         ts_in = torch.tensor([given_ts], dtype=torch.float32, device="cuda")
-    q = mx.quantize(x, cfg, stats=check_stats, tensor_scale=ts_in, rotated=bool(cfg.hadamard))
+    if want_rotated is None:
+        want_rotated = bool(cfg.hadamard)
+    q = mx.quantize(x, cfg, stats=check_stats, tensor_scale=ts_in, rotated=want_rotated)
     xh = mx.dequantize(q, torch.float32)
     torch.cuda.synchronize()
     oc = ocfg(orc, cfg)
@@ -80,7 +87,7 @@ def run_case(mx, orc, x_cpu, cfg, check_stats=True, given_ts=None):
         assert np.array_equal(q.macro.cpu().numpy(), r["macro"]), "macro scale codes"
     if cfg.asymmetric:
         assert np.array_equal(q.offsets.cpu().numpy().view(np.uint16), r["offsets"]), "offsets"
-    if cfg.hadamard:
+    if cfg.hadamard and want_rotated:
         assert_same_f32(q.rotated.cpu().numpy(), r["y"], "rotated tensor")
     oxh = orc.dequantize(oc, r["packed"], r["scales"], r["tensor_scale"], r["macro"],
                          r["offsets"], rows, cols, unrotate=False)
@@ -89,8 +96,14 @@ def run_case(mx, orc, x_cpu, cfg, check_stats=True, given_ts=None):
         oxu = orc.dequantize(oc, r["packed"], r["scales"], r["tensor_scale"], r["macro"],
                              r["offsets"], rows, cols, unrotate=True)
         assert_same_f32(xh.cpu().numpy(), oxu, "dequantized (rotated back)")
+        want_bf16 = oxu
     else:
         assert_same_f32(xh.cpu().numpy(), oxh, "dequantized")
+        want_bf16 = oxh
+    if bf16_out:
+        xb = mx.dequantize(q, torch.bfloat16)
+        wb = torch.from_numpy(np.ascontiguousarray(want_bf16, np.float32)).to(torch.bfloat16)
+        assert torch.equal(xb.cpu().view(torch.int16), wb.view(torch.int16)), "bf16 dequantized"
     if check_stats:
         ost, _ = orc.stats(r["y"], oxh)
         assert_stats(q.stats.cpu().numpy(), ost, rows * cols)

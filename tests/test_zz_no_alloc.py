@@ -50,7 +50,7 @@ def _same(mx, a, b):
     assert sa[3] == sb[3] and sa[4] == sb[4] and sa[10] == sb[10]
 
 
-@pytest.mark.parametrize("name", ["mxfp4", "nvfp4", "sr_fp32"])
+@pytest.mark.parametrize("name", ["mxfp4", "nvfp4", "sr_fp32", "nvfp4_mse"])
 def test_noalloc_matches_mx_quantize_twice(mx, name):
     if name == "mxfp4":
         cfg = mx.MXFP4
@@ -58,6 +58,12 @@ def test_noalloc_matches_mx_quantize_twice(mx, name):
     elif name == "nvfp4":
         cfg = mx.NVFP4
         x = inputs.normal(512, 4096, sigma=0.02, seed=2).cuda()
+    elif name == "nvfp4_mse":
+        # the heaviest scratch user: four global-step reductions through the
+        # records and the ticket, and the per-round tensor scales kept in the
+        # control words, which the call clears for the next one
+        cfg = mx.Config(block=16, scale_fmt=mx.SCALE_UE4M3, rule=mx.RULE_MSE, tensor_scale=mx.TS_COMPUTE)
+        x = inputs.normal(512, 2048, sigma=0.02, seed=3).cuda()
     else:
         cfg = mx.Config(round=mx.ROUND_STOCHASTIC, seed=9)
         x = inputs.gradient_like(256, 4096, seed=5).cuda()
@@ -66,3 +72,20 @@ def test_noalloc_matches_mx_quantize_twice(mx, name):
     second = _noalloc(mx, cfg, x)
     _same(mx, first, ref)
     _same(mx, second, ref)
+
+
+def test_noalloc_rejections_leave_the_array_usable(mx):
+    """The two configurations the no-alloc entry does not take -- a rotation,
+    and an amax handed in through a caller's workspace -- are refused with
+    MX_ERR_UNSUPPORTED before anything is queued, and a following call still
+    reproduces mx_quantize."""
+    x = inputs.normal(256, 1024, sigma=0.02, seed=2).cuda()
+    P = lambda t: C.c_void_p(t.data_ptr())
+    q = mx.alloc_outputs(mx.NVFP4, 256, 1024, x.device, stats=True)
+    stream = C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for cfg in (mx.Config(hadamard=32), mx.Config(hadamard=16, block=16),
+                mx.Config(block=16, scale_fmt=mx.SCALE_UE4M3, rule=mx.RULE_NEAREST, tensor_scale=mx.TS_AMAX)):
+        rc = mx.mx_quantize_noalloc(cfg, P(x), mx.DT_BF16, 256, 1024, P(q.codes), P(q.scales),
+                                    P(q.tensor_scale), None, None, P(q.stats), stream)
+        assert rc == -2, mx.mx_strerror(rc)
+    _same(mx, _noalloc(mx, mx.NVFP4, x), mx.quantize(x, mx.NVFP4))
