@@ -326,10 +326,15 @@ int mx_gemm(const mx_config *ca, const mx_config *cb, const void *Aq, const uint
 /*
  * mx_gemm_qsnr -- post-operation QSNR ([MXFP4-OAS] Sec.3 Eq. (2)):
  * 10 log10(||A B^T||_F^2 / ||A B^T - A^Q (B^Q)^T||_F^2) with A [M x K] and
- * B [N x K] bf16 (device).  Both products are formed tile by tile on the
- * tensor cores (bf16 with FP32 accumulation, and block-scaled FP4) and the
- * epilogue reduces the two sums without writing C.  stats: device, 3 doubles
- * [sum C_ref^2, sum (C_ref - C_q)^2, QSNR dB].  Shapes as mx_gemm.
+ * B [N x K] bf16 (device).  One persistent kernel forms both products of
+ * every 128 x 256 (N % 256 == 0, else 128 x 128) output tile on the tensor
+ * cores -- the block-scaled one (operand pairs as mx_gemm), then bf16 with
+ * FP32 accumulation -- and its epilogue reduces sum C_ref^2 and
+ * sum (C_ref - C_q)^2 (binary32 over 32 columns, then binary64) without
+ * writing C; a second launch adds the per-CTA records in a fixed order.
+ * stats: device, 3 doubles [sum C_ref^2, sum (C_ref - C_q)^2, QSNR dB].
+ * workspace: mx_gemm_workspace_bytes() bytes (a fixed 16,640: the per-CTA
+ * records, independent of the shape).  Shapes as mx_gemm.
  */
 int64_t mx_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 int mx_gemm_qsnr(const mx_config *ca, const mx_config *cb, const void *A, const void *B, int64_t M,

@@ -15,8 +15,10 @@
 //                32-element blocks) / kind::mxf4nvf4 (UE4M3, 16-element
 //                blocks) / kind::f16 (bf16), tcgen05.commit to free stages;
 //   warps 2..5   epilogue: tcgen05.ld of the accumulator lanes of their
-//                quadrant, per-tensor scales, and either the C store or the
-//                QSNR sums against a previously computed C_q.
+//                quadrant, per-tensor scales, the C store.
+// The persistent 128 x 256 kernel (k_gemm_p) and the fused QSNR(AB) kernel
+// (k_gemm_qsnr_f: both products of one output tile in turn, the error sums
+// reduced in the epilogue, C never written) follow below.
 // Every TMA load targets its own CTA only; every wait on an mbarrier is bounded and sets a
 // device status word instead of hanging.
 #include <cuda.h>
@@ -40,7 +42,7 @@ constexpr uint64_t kWaitNs = 2000000000ull;       // bound of one mbarrier wait:
 
 enum { KIND_BF16 = 0, KIND_MXF4 = 1, KIND_NVF4 = 2, KIND_MXF6 = 3 };
 constexpr uint32_t kFmtE2M1 = 5;     // E2M1 in the kind::mxf8f6f4 instruction descriptor
-enum { EPI_BF16 = 0, EPI_F32 = 1, EPI_QSNR = 2 };
+enum { EPI_BF16 = 0, EPI_F32 = 1 };
 
 // device status word of the bounded waits (read and cleared by mx_device_status)
 __device__ int g_status;
@@ -50,8 +52,8 @@ struct GParams {
     const uint8_t *sfa, *sfb;    // scale chunks (FP4 kinds)
     const float *tsA, *tsB;      // per-tensor scales or null
     void *C;                     // EPI_BF16 / EPI_F32 output, row-major M x N
-    const float *Cq;             // EPI_QSNR: the quantized product, fp32 M x N
-    double *partials;            // EPI_QSNR: per-CTA [sum C^2, sum (C - Cq)^2]
+    double *partials;            // QSNR(AB): per-CTA [sum C_ref^2, sum (C_ref - C_q)^2]
+    double *stats;               // QSNR(AB): [sum C_ref^2, sum (C_ref - C_q)^2, dB]
     uint32_t ab_fmt;             // KIND_MXF6: A / B element formats of the instruction descriptor
     uint32_t stage_tx;           // KIND_MXF6: bytes the TMA brings per stage (A, B and scales)
 };
@@ -225,7 +227,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *empty = full + kStages;
     uint64_t *accf = empty + kStages;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(accf + 1);
-    double *red = reinterpret_cast<double *>(tmem_holder + 4);   // 4 warps x 2 sums
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
@@ -320,7 +321,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         float scale = 1.0f;
         if (p.tsA) scale = __fmul_rn(scale, *p.tsA);
         if (p.tsB) scale = __fmul_rn(scale, *p.tsB);
-        double s_ref = 0.0, s_err = 0.0;
         if (ready) {
 #pragma unroll 1
             for (int ch = 0; ch < BN / 32; ++ch) {
@@ -338,51 +338,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[i + 2 * j + 1] * scale)) << 16);
                         *reinterpret_cast<uint4 *>(dst + i) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
-                } else if constexpr (EPI == EPI_F32) {
+                } else {
                     float *dst = static_cast<float *>(p.C) + (size_t)row * p.N + col;
 #pragma unroll
                     for (int i = 0; i < 32; i += 4)
                         *reinterpret_cast<float4 *>(dst + i) =
                             make_float4(v[i] * scale, v[i + 1] * scale, v[i + 2] * scale, v[i + 3] * scale);
-                } else {
-                    const float *cq = p.Cq + (size_t)row * p.N + col;
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        const float4 c4 = *reinterpret_cast<const float4 *>(cq + i);
-                        const float cr[4] = {v[i] * scale, v[i + 1] * scale, v[i + 2] * scale, v[i + 3] * scale};
-                        const float cqv[4] = {c4.x, c4.y, c4.z, c4.w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const double a = (double)cr[j], d = a - (double)cqv[j];
-                            s_ref += a * a;
-                            s_err += d * d;
-                        }
-                    }
                 }
-            }
-        }
-        if constexpr (EPI == EPI_QSNR) {
-            for (int o = 16; o > 0; o >>= 1) {
-                s_ref += __shfl_down_sync(0xffffffffu, s_ref, o);
-                s_err += __shfl_down_sync(0xffffffffu, s_err, o);
-            }
-            if (lane == 0) {
-                red[2 * (warp - 2)] = s_ref;
-                red[2 * (warp - 2) + 1] = s_err;
             }
         }
     }
     tc_fence_before();
     __syncthreads();
-    if constexpr (EPI == EPI_QSNR) {
-        if (threadIdx.x == 0) {
-            double a = 0.0, b = 0.0;
-            for (int w = 0; w < 4; ++w) { a += red[2 * w]; b += red[2 * w + 1]; }
-            double *o = p.partials + 2 * ((size_t)blockIdx.y * gridDim.x + blockIdx.x);
-            o[0] = a;
-            o[1] = b;
-        }
-    }
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(kTmemCols));
@@ -598,6 +565,267 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Fused QSNR(AB) ("Unveiling the Potential of Quantization with MXFP4", Sec.3
+// Eq. (2)): persistent, one CTA per SM, 128 x BNT output tiles.  For every
+// tile the MMA warp forms C_q = A^Q (B^Q)^T with the block-scaled kind into
+// the accumulator (BNT TMEM columns), the eight epilogue warps move it into
+// registers (BNT / 2 floats a thread, times the tensor scales) and hand the
+// columns back, the MMA warp then forms C_ref = A B^T with kind::f16 on the
+// bf16 operands into the same columns, and the epilogue reduces
+// sum C_ref^2 and sum (C_ref - C_q)^2 against the registers.  C is never
+// written.  The producer streams both phases through one shared-memory ring:
+// a block-scaled stage is 128 bytes of every row (plus the scale chunks), a
+// bf16 stage 64 elements (also 128 bytes) of every row.  Tiles are walked in
+// groups of kGroupM tile rows so that the A and B slices a wave of CTAs reads
+// stay in L2 (the bf16 operands are four times the FP4 ones).
+constexpr int kGroupM = 16;
+
+template <int KIND, int BNT>
+struct KindQ {
+    static constexpr int kChunks = KindP<KIND>::kChunks;          // scale chunks per stage and 128 rows
+    static constexpr int kBHalves = BNT / 128;                    // 128-row groups of B
+    static constexpr int kSfaBytes = kChunks * 512;
+    static constexpr int kSfbBytes = kBHalves * kChunks * 512;
+    static constexpr int kABytes = BM * 128, kBBytes = BNT * 128;
+    static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+    static constexpr int kSfCols = kChunks * 4 + kBHalves * kChunks * 4;
+    static constexpr int kSmem = 1024 + kStagesP * kStageBytes + 256;
+};
+
+// tile index -> (tile row, tile column): groups of kGroupM tile rows, walked
+// column by column inside a group
+__device__ __forceinline__ void qsnr_tile(int tile, int ntm, int ntn, int &mt, int &nt)
+{
+    const int per = kGroupM * ntn;
+    const int g = tile / per, r = tile - g * per;
+    const int gm = min(kGroupM, ntm - g * kGroupM);
+    mt = g * kGroupM + r % gm;
+    nt = r / gm;
+}
+
+template <int KIND, int BNT>
+__global__ void __launch_bounds__(kThreadsP, 1)
+    k_gemm_qsnr_f(const GParams p, const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const __grid_constant__ CUtensorMap tmAr, const __grid_constant__ CUtensorMap tmBr)
+{
+    using KT = KindQ<KIND, BNT>;
+    constexpr int HALF = BNT / 2;                 // columns per epilogue warp
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *sA = smem;
+    uint8_t *sB = sA + kStagesP * KT::kABytes;
+    uint8_t *sSFA = sB + kStagesP * KT::kBBytes;
+    uint8_t *sSFB = sSFA + kStagesP * KT::kSfaBytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sSFB + kStagesP * KT::kSfbBytes);
+    uint64_t *empty = full + kStagesP;
+    uint64_t *accf = empty + kStagesP;            // accumulator full (MMA -> epilogue), once per product
+    uint64_t *acce = accf + 1;                    // accumulator read out (epilogue -> MMA)
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(acce + 1);
+    double *red = reinterpret_cast<double *>(tmem_holder + 4);      // 8 warps x 2 sums
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntn = p.N / BNT, ntm = p.M / BM;
+    const int ntiles = ntn * ntm;
+    const int kq = p.K / (KIND == KIND_MXF6 ? 128 : 256);      // block-scaled stages per tile
+    const int kr = p.K / 64;                                     // bf16 stages per tile
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStagesP; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accf, 1);
+        mbar_init(acce, 8);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(saddr(tmem_holder)), "r"(kTmemColsP));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_holder;
+    const uint32_t tsf = tbase + BNT;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const int sf_chunks_row = (p.K / (KIND == KIND_NVF4 ? 16 : 32)) / 4;
+            const uint32_t tx_q = KIND == KIND_MXF6 ? p.stage_tx : (uint32_t)KT::kStageBytes;
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                int mt, nt;
+                qsnr_tile(tile, ntm, ntn, mt, nt);
+                const int m0 = mt * BM, n0 = nt * BNT;
+                for (int kt = 0; kt < kq + kr; ++kt, ++it) {
+                    const int s = it % kStagesP;
+                    if (it >= (uint32_t)kStagesP && !mbar_wait(&empty[s], ((it / kStagesP) - 1) & 1, 15)) { ok = false; break; }
+                    if (kt < kq) {
+                        mbar_expect_tx(&full[s], tx_q);
+                        tma_load_2d(sA + s * KT::kABytes, &tmA, &full[s], kt * 128, m0);
+                        tma_load_2d(sB + s * KT::kBBytes, &tmB, &full[s], kt * 128, n0);
+                        const size_t ca = ((size_t)(m0 / 128) * sf_chunks_row + (size_t)kt * KT::kChunks) * 512;
+                        bulk_load(sSFA + s * KT::kSfaBytes, p.sfa + ca, KT::kSfaBytes, &full[s]);
+#pragma unroll
+                        for (int hb = 0; hb < KT::kBHalves; ++hb) {
+                            const size_t cb = ((size_t)(n0 / 128 + hb) * sf_chunks_row + (size_t)kt * KT::kChunks) * 512;
+                            bulk_load(sSFB + s * KT::kSfbBytes + hb * KT::kChunks * 512, p.sfb + cb,
+                                      KT::kChunks * 512, &full[s]);
+                        }
+                    } else {
+                        const int kx = (kt - kq) * 64;                       // bf16 elements
+                        mbar_expect_tx(&full[s], (uint32_t)(KT::kABytes + KT::kBBytes));
+                        tma_load_2d(sA + s * KT::kABytes, &tmAr, &full[s], kx, m0);
+                        tma_load_2d(sB + s * KT::kBBytes, &tmBr, &full[s], kx, n0);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // block-scaled kind (N = BNT) and kind::f16 on bf16 (N = BNT)
+            uint32_t idq = KIND == KIND_MXF6 ? p.ab_fmt : (1u << 7) | (1u << 10);
+            if (KIND != KIND_NVF4) idq |= 1u << 23;
+            idq |= (uint32_t)(BNT >> 3) << 17;
+            idq |= (uint32_t)(BM >> 4) << 24;
+            const uint32_t idr = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BNT >> 3) << 17) |
+                                 ((uint32_t)(BM >> 4) << 24);
+            uint32_t it = 0, ph = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+                for (int part = 0; part < 2 && ok; ++part, ++ph) {
+                    // the epilogue has read the previous product out of the accumulator
+                    if (ph > 0 && !mbar_wait(acce, (ph - 1) & 1, 16)) { ok = false; break; }
+                    tc_fence_after();
+                    const int k0 = part == 0 ? 0 : kq, k1 = part == 0 ? kq : kq + kr;
+                    for (int kt = k0; kt < k1; ++kt, ++it) {
+                        const int s = it % kStagesP;
+                        if (!mbar_wait(&full[s], (it / kStagesP) & 1, 17)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t a0 = saddr(sA + s * KT::kABytes), b0 = saddr(sB + s * KT::kBBytes);
+                        const uint32_t acc0 = kt > k0 ? 1u : 0u;
+                        if (part == 1) {
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                mma<KIND_BF16>(tbase, desc_sw128(a0 + 32 * k), desc_sw128(b0 + 32 * k), idr, 0, 0,
+                                               (acc0 | (uint32_t)k) ? 1u : 0u);
+                        } else {
+                            const uint32_t sfa_t = tsf + s * KT::kSfCols;
+                            const uint32_t sfb_t = sfa_t + KT::kChunks * 4;
+#pragma unroll
+                            for (int c = 0; c < KT::kChunks; ++c) {
+                                asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                                             ::"r"(sfa_t + 4 * c), "l"(desc_sf(saddr(sSFA + s * KT::kSfaBytes + c * 512))));
+#pragma unroll
+                                for (int hb = 0; hb < KT::kBHalves; ++hb)
+                                    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                                                 ::"r"(sfb_t + 4 * KT::kBHalves * c + 4 * hb),
+                                                   "l"(desc_sf(saddr(sSFB + s * KT::kSfbBytes + hb * KT::kChunks * 512 + c * 512))));
+                            }
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                uint32_t idesc = idq, sfa, sfb;
+                                if constexpr (KIND == KIND_MXF4) {
+                                    const uint32_t id = (k & 1) * 2;
+                                    idesc |= (id << 29) | (id << 4);
+                                    sfa = sfa_t + 4 * (k >> 1);
+                                    sfb = sfb_t + 4 * KT::kBHalves * (k >> 1);
+                                } else if constexpr (KIND == KIND_MXF6) {
+                                    const uint32_t id = (uint32_t)k;
+                                    idesc |= (id << 29) | (id << 4);
+                                    sfa = sfa_t;
+                                    sfb = sfb_t;
+                                } else {
+                                    sfa = sfa_t + 4 * k;
+                                    sfb = sfb_t + 4 * KT::kBHalves * k;
+                                }
+                                mma<KIND>(tbase, desc_sw128(a0 + 32 * k), desc_sw128(b0 + 32 * k), idesc, sfa, sfb,
+                                          (acc0 | (uint32_t)k) ? 1u : 0u);
+                            }
+                        }
+                        tc_commit(&empty[s]);
+                    }
+                    if (ok) tc_commit(accf);
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // eight epilogue warps: TMEM lane quadrant q = warp % 4, column half h
+        const int q = warp & 3, h = (warp - 2) >> 2;
+        float scale = 1.0f;
+        if (p.tsA) scale = __fmul_rn(scale, *p.tsA);
+        if (p.tsB) scale = __fmul_rn(scale, *p.tsB);
+        const uint32_t tcol = tbase + ((uint32_t)(32 * q) << 16) + h * HALF;
+        double s_ref = 0.0, s_err = 0.0;
+        uint32_t ph = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            // C_q of this thread's row and column half, into registers
+            if (!mbar_wait(accf, ph & 1, 18)) break;
+            tc_fence_after();
+            float cq[HALF];
+#pragma unroll
+            for (int ch = 0; ch < HALF / 32; ++ch) tmem_ld32(tcol + ch * 32, cq + 32 * ch);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(acce)) : "memory");
+            ++ph;
+            // C_ref, 32 columns at a time, against the registers
+            if (!mbar_wait(accf, ph & 1, 19)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int ch = 0; ch < HALF / 32; ++ch) {
+                float v[32];
+                tmem_ld32(tcol + ch * 32, v);
+                if (ch == HALF / 32 - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(acce)) : "memory");
+                }
+                // 32 terms per chunk in binary32 (two chains), then binary64
+                float r0 = 0.f, r1 = 0.f, e0 = 0.f, e1 = 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const float d0 = __fmaf_rn(-cq[32 * ch + i], scale, v[i]);
+                    const float d1 = __fmaf_rn(-cq[32 * ch + i + 1], scale, v[i + 1]);
+                    r0 = __fmaf_rn(v[i], v[i], r0);
+                    r1 = __fmaf_rn(v[i + 1], v[i + 1], r1);
+                    e0 = __fmaf_rn(d0, d0, e0);
+                    e1 = __fmaf_rn(d1, d1, e1);
+                }
+                s_ref += (double)r0 + (double)r1;
+                s_err += (double)e0 + (double)e1;
+            }
+            ++ph;
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+            s_ref += __shfl_down_sync(0xffffffffu, s_ref, o);
+            s_err += __shfl_down_sync(0xffffffffu, s_err, o);
+        }
+        if (lane == 0) {
+            red[2 * (warp - 2)] = s_ref;
+            red[2 * (warp - 2) + 1] = s_err;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double a = 0.0, b = 0.0;
+        for (int w = 0; w < 8; ++w) { a += red[2 * w]; b += red[2 * w + 1]; }
+        p.partials[2 * blockIdx.x] = a;
+        p.partials[2 * blockIdx.x + 1] = b;
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(kTmemColsP));
+    }
+}
+
 // Sum the per-CTA records in a fixed order: [sum C_ref^2, sum err^2, QSNR dB].
 __global__ void k_gemm_qsnr_finalize(const double *partials, int n, double *out)
 {
@@ -734,6 +962,51 @@ int launch_p(const GParams &p, const void *A, const void *B, cudaStream_t st)
     return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
 }
 
+constexpr int kMaxQsnrCtas = 1024;     // per-CTA records of the fused QSNR(AB) kernel
+
+template <int KIND, int BNT>
+int launch_qsnr_f(const GParams &p, const void *Aq, const void *Bq, const void *A, const void *B,
+                  cudaStream_t st)
+{
+    using KT = KindQ<KIND, BNT>;
+    CUtensorMap ta, tb, tar, tbr;
+    GParams q = p;
+    int abits = 4, bbits = 4;
+    if (KIND == KIND_MXF6) {
+        const bool a4 = ((p.ab_fmt >> 7) & 7u) == kFmtE2M1, b4 = ((p.ab_fmt >> 10) & 7u) == kFmtE2M1;
+        abits = a4 ? -4 : -6;
+        bbits = b4 ? -4 : -6;
+        q.stage_tx = (uint32_t)((a4 ? KT::kABytes / 2 : KT::kABytes / 4 * 3) +
+                                (b4 ? KT::kBBytes / 2 : KT::kBBytes / 4 * 3) + KT::kSfaBytes + KT::kSfbBytes);
+    }
+    if (!make_map(&ta, Aq, p.M, p.K, abits, 128) || !make_map(&tb, Bq, p.N, p.K, bbits, BNT) ||
+        !make_map(&tar, A, p.M, p.K, 16, 128) || !make_map(&tbr, B, p.N, p.K, 16, BNT))
+        return MX_ERR_CUDA;
+    auto k = k_gemm_qsnr_f<KIND, BNT>;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, KT::kSmem) != cudaSuccess)
+            return MX_ERR_CUDA;
+        attr = true;
+    }
+    const int tiles = (p.M / BM) * (p.N / BNT);
+    int grid = mxk::device_sm_count();
+    if (grid > tiles) grid = tiles;
+    if (grid > kMaxQsnrCtas) grid = kMaxQsnrCtas;
+    k<<<grid, kThreadsP, KT::kSmem, st>>>(q, ta, tb, tar, tbr);
+    if (cudaGetLastError() != cudaSuccess) return MX_ERR_CUDA;
+    k_gemm_qsnr_finalize<<<1, 256, 0, st>>>(p.partials, grid, p.stats);
+    return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+}
+
+template <int KIND>
+int launch_qsnr_kind(const GParams &p, const void *Aq, const void *Bq, const void *A, const void *B,
+                     cudaStream_t st)
+{
+    return p.N % BNP == 0 ? launch_qsnr_f<KIND, BNP>(p, Aq, Bq, A, B, st)
+                          : launch_qsnr_f<KIND, BN>(p, Aq, Bq, A, B, st);
+}
+
 // MXFP4 (E2M1 + E8M0, block 32) or NVFP4 (E2M1 + UE4M3, block 16) operands
 // quantized along K in the tcgen05 scale layout; returns the kind or -1.
 int fp4_kind(const mx_config *a, const mx_config *b)
@@ -791,8 +1064,8 @@ int64_t mx_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)
 {
     (void)K;
     if (M <= 0 || N <= 0) return 0;
-    const int64_t tiles = (M / BM) * (N / BN);
-    return 256 + M * N * 4 + tiles * 16;
+    // one record of two binary64 sums per CTA of the fused kernel
+    return 256 + (int64_t)kMaxQsnrCtas * 16;
 }
 
 int mx_gemm(const mx_config *ca, const mx_config *cb, const void *Aq, const uint8_t *Asf,
@@ -847,32 +1120,39 @@ int mx_gemm_qsnr(const mx_config *ca, const mx_config *cb, const void *A, const 
                  const uint8_t *Bsf, const float *tsA, const float *tsB, double *stats,
                  void *workspace, int64_t workspace_bytes, void *stream)
 {
-    if (fp4_kind(ca, cb) < 0) return MX_ERR_UNSUPPORTED;
+    const int kind = fp4_kind(ca, cb);
+    if (kind < 0) return MX_ERR_UNSUPPORTED;
     if (!shapes_ok(M, N, K)) return MX_ERR_INVALID;
-    if (!A || !B || !stats) return MX_ERR_INVALID;
+    if (!A || !B || !stats || !Aq || !Bq || !Asf || !Bsf) return MX_ERR_INVALID;
     if (!workspace || workspace_bytes < mx_gemm_workspace_bytes(M, N, K)) return MX_ERR_WORKSPACE;
-    if (!aligned16(A) || !aligned16(B) || !aligned16(workspace) || ((uintptr_t)stats & 7u))
+    if (!aligned16(A) || !aligned16(B) || !aligned16(Aq) || !aligned16(Bq) || !aligned16(Asf) ||
+        !aligned16(Bsf) || !aligned16(workspace) || ((uintptr_t)stats & 7u))
         return MX_ERR_ALIGN;
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    float *cq = reinterpret_cast<float *>(ws + 256);
-    double *partials = reinterpret_cast<double *>(ws + 256 + M * N * 4);
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // 1) C_q = A^Q (B^Q)^T (block-scaled FP4 MMA), fp32
-    int rc = mx_gemm(ca, cb, Aq, Asf, Bq, Bsf, tsA, tsB, M, N, K, cq, MX_DT_FP32, stream);
-    if (rc != MX_OK) return rc;
-    // 2) C_ref = A B^T (bf16 MMA, FP32 accumulate) with the QSNR sums in the epilogue
     GParams p;
     memset(&p, 0, sizeof(p));
     p.M = (int)M;
     p.N = (int)N;
     p.K = (int)K;
-    p.Cq = cq;
-    p.partials = partials;
-    rc = launch<KIND_BF16, EPI_QSNR>(p, A, B, st);
-    if (rc != MX_OK) return rc;
-    const int tiles = (int)((M / BM) * (N / BN));
-    k_gemm_qsnr_finalize<<<1, 256, 0, st>>>(partials, tiles, stats);
-    return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+    p.sfa = Asf;
+    p.sfb = Bsf;
+    if (kind == KIND_NVF4) {
+        p.tsA = ca->tensor_scale != MX_TS_NONE ? tsA : nullptr;
+        p.tsB = cb->tensor_scale != MX_TS_NONE ? tsB : nullptr;
+    }
+    p.partials = reinterpret_cast<double *>(static_cast<uint8_t *>(workspace) + 256);
+    p.stats = stats;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // both products of every output tile in one persistent kernel, the sums
+    // reduced in its epilogue (C is not written), then the per-CTA records
+    // summed in a fixed order
+    if (kind == KIND_MXF6) {
+        if (N % BNP) return MX_ERR_UNSUPPORTED;
+        if (((uintptr_t)Aq & 31u) || ((uintptr_t)Bq & 31u)) return MX_ERR_ALIGN;
+        p.ab_fmt = fp6_formats(ca, cb);
+        return launch_qsnr_f<KIND_MXF6, BNP>(p, Aq, Bq, A, B, st);
+    }
+    if (kind == KIND_MXF4) return launch_qsnr_kind<KIND_MXF4>(p, Aq, Bq, A, B, st);
+    return launch_qsnr_kind<KIND_NVF4>(p, Aq, Bq, A, B, st);
 }
 
 int mx_device_status(void *stream, int32_t *status)

@@ -114,18 +114,62 @@ def test_gemm_rejects_canonical_scales(mx):
     assert e.value.code == -2
 
 
-@pytest.mark.parametrize("name", ["mxfp4", "nvfp4"])
-def test_gemm_qsnr_small(mx, orc, name):
-    M, N, K = 256, 256, 512
+def _qsnr_vs_oracle(mx, orc, name, M, N, K, blas=False):
     a = inputs.laplace_outlier_cols(M, K, seed=6, n_outlier_cols=2)
     w = inputs.normal(N, K, sigma=0.02, seed=7)
     cfg = configs(mx)[name]
     qa = mx.quantize(a.cuda(), cfg, stats=False)
     qw = mx.quantize(w.cuda(), cfg, stats=False)
     st = mx.gemm_qsnr(a.cuda(), w.cuda(), qa, qw).cpu().numpy()
+    assert mx.mx_device_status() == 0
     ah, _ = deq(orc, name, a)
     wh, _ = deq(orc, name, w)
-    o = orc.gemm_qsnr(orc.input_f32(a), orc.input_f32(w), ah, wh)
+    f = orc.gemm_qsnr_blas if blas else orc.gemm_qsnr
+    o = f(orc.input_f32(a), orc.input_f32(w), ah, wh)
+    assert abs(st[0] - o[0]) <= 1e-3 * o[0]
+    assert abs(st[1] - o[1]) <= 1e-3 * o[1]
+    assert abs(st[2] - o[2]) <= 1e-2
+    return st
+
+
+@pytest.mark.parametrize("name", ["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("shape", [(256, 256, 512), (384, 640, 768), (128, 128, 256)])
+def test_gemm_qsnr_small(mx, orc, name, shape):
+    """Both products formed tile by tile in one kernel, C never written:
+    tiles of 128 x 256 (N % 256 == 0) and 128 x 128 (N = 640), against the
+    oracle's binary64 sums."""
+    _qsnr_vs_oracle(mx, orc, name, *shape)
+
+
+@pytest.mark.parametrize("name", ["mxfp4", "nvfp4"])
+@pytest.mark.parametrize("shape", [(2176, 2560, 512), (2176, 1920, 256)])
+def test_gemm_qsnr_many_tiles_per_cta(mx, orc, name, shape):
+    """More output tiles than CTAs (each CTA walks several tiles, the
+    accumulator hand-over alternating between the two products), and a
+    last group of tile rows shorter than the others."""
+    _qsnr_vs_oracle(mx, orc, name, *shape, blas=True)
+
+
+def test_gemm_qsnr_workspace_does_not_grow_with_c(mx):
+    """The QSNR(AB) scratch is a fixed set of per-CTA records, not C."""
+    lib = mx.lib()
+    assert lib.mx_gemm_workspace_bytes(8192, 14336, 4096) == lib.mx_gemm_workspace_bytes(128, 128, 256)
+    assert lib.mx_gemm_workspace_bytes(8192, 14336, 4096) < 1 << 20
+
+
+@pytest.mark.parametrize("name", ["mxfp4", "nvfp4"])
+def test_gemm_qsnr_llama_shape(mx, orc, name):
+    """QSNR(AB) of the full 8192 x 4096 by 14336 x 4096 layer against the
+    oracle's binary64 BLAS sums over its dequantized operands."""
+    A, W = inputs.llama_linear()
+    cfg = configs(mx)[name]
+    qa = mx.quantize(A.cuda(), cfg, stats=False)
+    qw = mx.quantize(W.cuda(), cfg, stats=False)
+    st = mx.gemm_qsnr(A.cuda(), W.cuda(), qa, qw).cpu().numpy()
+    assert mx.mx_device_status() == 0
+    ah, _ = deq(orc, name, A)
+    wh, _ = deq(orc, name, W)
+    o = orc.gemm_qsnr_blas(orc.input_f32(A), orc.input_f32(W), ah, wh)
     assert abs(st[0] - o[0]) <= 1e-3 * o[0]
     assert abs(st[1] - o[1]) <= 1e-3 * o[1]
     assert abs(st[2] - o[2]) <= 1e-2
