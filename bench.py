@@ -35,6 +35,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 M_TOK, K_DIM, N_OUT = 8192, 4096, 14336
+R_PAIRS = 8          # A/W launch pairs per per-variant timing graph
 WORKLOAD = ("Llama-3-8B-shaped linear layer: A 8192x4096 bf16 Laplace(0,1) seed 6, "
             "W 14336x4096 bf16 N(0,0.02) seed 7 (W stored out x in, product A W^T)")
 METRIC = "MX quantize+pack GB/s (% of ~8 TB/s HBM); block-scaled FP4 GEMM TFLOPS"
@@ -263,17 +264,25 @@ def run_ours(args, rank, world, device):
         run_step()
     torch.cuda.synchronize(device)
 
-    # the step, and every launch of it, captured as CUDA graphs: the kernels
-    # run back to back with no host work between them
+    # the step captured as a CUDA graph: the kernels run back to back with no
+    # host work between them.  Per variant, a graph of R_PAIRS back-to-back
+    # pairs of its launches on A and on W (one stream, the step's launch
+    # configuration): consecutive launches read different tensors, 176 MiB
+    # apart, so no input comes from L2, and the time over the pairs is the
+    # steady-state launch duration without graph-launch gaps
     step_graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(step_graph):
         run_step()
-    call_graphs = []
-    for call in plan:
+    variants = list(dict.fromkeys(name for name, _, _, _ in plan))
+    pair_graphs = {}
+    for name in variants:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            run_call(*call)
-        call_graphs.append(g)
+            for _ in range(R_PAIRS):
+                for call in plan:
+                    if call[0] == name:
+                        run_call(*call)
+        pair_graphs[name] = g
     for _ in range(args.warmup):
         step_graph.replay()
     torch.cuda.synchronize(device)
@@ -306,11 +315,10 @@ def run_ours(args, rank, world, device):
     ms_per_step = elapsed_ms / args.steps
     value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
 
-    # per-launch device time: each launch's graph replayed K times between
-    # events (inputs larger than L2, the same launch configuration as the step)
+    # per-variant device time (A + W launches) from its pair graph
     rows = {}
-    for i, (name, t, cfg, kind) in enumerate(plan):
-        g = call_graphs[i]
+    for name in variants:
+        g = pair_graphs[name]
         g.replay()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -318,13 +326,10 @@ def run_ours(args, rank, world, device):
             g.replay()
         e1.record(stream)
         torch.cuda.synchronize(device)
-        r = rows.setdefault(name, {"bytes": 0, "ms": 0.0})
-        r["bytes"] += algo_bytes(cfg, *T[t].shape, kind)
-        r["ms"] += e0.elapsed_time(e1) / args.steps
-    for r in rows.values():
-        r["GB_per_s"] = round(r["bytes"] / (r["ms"] * 1e-3) / 1e9, 1)
-        r["us"] = round(r["ms"] * 1e3, 2)
-        del r["ms"]
+        nb = sum(algo_bytes(cfg, *T[t].shape, kind) for n, t, cfg, kind in plan if n == name)
+        ms = e0.elapsed_time(e1) / (args.steps * R_PAIRS)
+        rows[name] = {"bytes": nb, "GB_per_s": round(nb / (ms * 1e-3) / 1e9, 1), "us": round(ms * 1e3, 2)}
+    del pair_graphs
 
     pk, pk_src = peaks()
     # the dominant kernel of the step: k_quant_fast, all eight quantizer
@@ -348,6 +353,10 @@ def run_ours(args, rank, world, device):
                 "by_variant_frac": {n: round(rows[n]["GB_per_s"] / pk["hbm_gbs"], 4) for n in qnames}}
 
     extra = run_extra_rows(mx, A, device, args)
+    try:
+        extra["c2_block_size_sweep"] = run_c2_sweep(mx, device, args)
+    except Exception as e:        # reported, not fatal: the headline step stands on its own
+        extra["c2_block_size_sweep"] = {"unavailable": f"{type(e).__name__}: {e}"}
 
     # end to end through the public API with host buffers
     e2e = run_e2e(mx, A_cpu, W_cpu, plan, outs, device, args, step_bytes, world)
@@ -396,6 +405,57 @@ def run_extra_rows(mx, A, device, args):
         out[name] = {"GB_per_s": round(nb / (ms * 1e-3) / 1e9, 1), "us": round(ms * 1e3, 2),
                      "qsnr_db": round(float(q.stats[7].item()), 4), "bias": float(q.stats[8].item())}
     del G
+    return out
+
+
+def run_c2_sweep(mx, device, args):
+    """The block-size sweep of "Is Finer Better?": 4096 x 4096 weight-like
+    N(0, sigma) tensors, sigma in {0.002, 0.02, 0.2} (seeds 1, 2, 3), E2M1
+    with UE4M3 / UE5M3 nearest block scales, without and with the FP32 tensor
+    scale, blocks 8 ... 256.  Per configuration: the per-tensor MSE at each
+    sigma, and the quantize call's GB/s (tensor-amax pass included) with a
+    cold L2: each timed call follows a read of a 256 MiB buffer, and is timed
+    between event nodes of a graph on either side of it."""
+    from microscaling_block_quantization_b200 import inputs
+    sigmas = (0.002, 0.02, 0.2)
+    xs = [inputs.normal(4096, 4096, sigma=sg, seed=i + 1).to(device) for i, sg in enumerate(sigmas)]
+    evict = torch.ones(256 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    out = {}
+    for fmt, fname in ((mx.SCALE_UE4M3, "UE4M3"), (mx.SCALE_UE5M3, "UE5M3")):
+        for ts in (0, 1):
+            for B in (8, 16, 32, 64, 128, 256):
+                cfg = mx.Config(block=B, scale_fmt=fmt, rule=mx.RULE_NEAREST, tensor_scale=ts)
+                ws = mx.new_workspace(cfg, 4096, 4096, device)
+                qs = [mx.alloc_outputs(cfg, 4096, 4096, device, stats=True) for _ in xs]
+                for x, q in zip(xs, qs):
+                    mx.quantize(x, cfg, out=q, workspace=ws)
+                torch.cuda.synchronize(device)
+                rec = {"mse": {str(sg): float(q.stats[5].item()) for sg, q in zip(sigmas, qs)}}
+                evs = [(torch.cuda.Event(enable_timing=True, external=True),
+                        torch.cuda.Event(enable_timing=True, external=True)) for _ in xs]
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    for (ea, eb), x, q in zip(evs, xs, qs):
+                        evict.sum()
+                        ea.record()
+                        mx.quantize(x, cfg, out=q, workspace=ws)
+                        eb.record()
+                ms = 0.0
+                n = max(3, args.steps // 2)
+                for _ in range(n + 1):
+                    g.replay()
+                    torch.cuda.synchronize(device)
+                    if _ == 0:
+                        continue
+                    ms += sum(ea.elapsed_time(eb) for ea, eb in evs) / len(evs)
+                ms /= n
+                nb = algo_bytes(cfg, 4096, 4096, "q")
+                rec["GB_per_s"] = round(nb / (ms * 1e-3) / 1e9, 1)
+                rec["us"] = round(ms * 1e3, 2)
+                out[f"{fname}_ts{ts}_B{B}"] = rec
+                del g
+    del evict
     return out
 
 
@@ -573,15 +633,20 @@ def run_gemm(mx, A, W, device, args, world):
 
 
 # ------------------------------------------------------------ CPU oracle ---
-def oracle_sample(rows_a=512, rows_w=512):
-    """The oracle on a bounded sample of the step: the first rows of A and W
+_LAYER_CPU = {}
+
+
+def oracle_sample(rows_a=512, rows_w=512, row0=0):
+    """The oracle on a bounded sample of the step: rows row0.. of A and W
     through every launch of the step (same configs)."""
     import oracle as O
     import microscaling_block_quantization_b200 as mx
     from microscaling_block_quantization_b200 import inputs
 
-    A, W = inputs.llama_linear(M_TOK, K_DIM, N_OUT)
-    T = {"A": A[:rows_a], "W": W[:rows_w]}
+    if not _LAYER_CPU:
+        _LAYER_CPU["A"], _LAYER_CPU["W"] = inputs.llama_linear(M_TOK, K_DIM, N_OUT)
+    A, W = _LAYER_CPU["A"], _LAYER_CPU["W"]
+    T = {"A": A[row0:row0 + rows_a], "W": W[row0:row0 + rows_w]}
     plan = step_plan(mx)
 
     def ocfg(c):
@@ -608,7 +673,40 @@ def oracle_sample(rows_a=512, rows_w=512):
     return run, nbytes, f"first {rows_a} rows of A and {rows_w} rows of W through every launch of the step"
 
 
+def host_cpu():
+    """(logical cores, CPU model) of this host."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count() or 1, model
+
+
+def _oracle_band(band):
+    """One worker of the all-cores leg: the oracle, unchanged, on a band of
+    rows of A and W through every launch of the step (a spawned process)."""
+    from microscaling_block_quantization_b200 import inputs
+    lo, hi = band
+    if not _LAYER_CPU or _LAYER_CPU["A"].shape[0] < hi:
+        # the first hi rows of the layer (numpy's streams are drawn in row order)
+        _LAYER_CPU["A"], _LAYER_CPU["W"] = inputs.llama_linear(hi, K_DIM, hi)
+    run, nbytes, _ = oracle_sample(rows_a=hi - lo, rows_w=hi - lo, row0=lo)
+    run()
+    return nbytes
+
+
 def cpu_baseline(target_s=10.0):
+    """The oracle as it stands on the host cores: one thread on the first 512
+    rows of A and W, and all cores as independent processes, each running the
+    unchanged oracle on its own band of rows (the oracle has no threading of
+    its own; blocks are independent, so the bands need no exchange)."""
+    import multiprocessing as mp
+    cores, model = host_cpu()
     run, nbytes, sample = oracle_sample()
     t0 = time.perf_counter()
     run()
@@ -618,8 +716,26 @@ def cpu_baseline(target_s=10.0):
     for _ in range(reps):
         run()
     dt = (time.perf_counter() - t0) / reps
-    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{sample}; {reps} repetitions, {dt:.3f} s each, single-threaded scalar C"}
+    single = nbytes / dt / 1e9
+    out = {"value": round(single, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "sample": f"{sample}; {reps} repetitions, {dt:.3f} s each, single-threaded scalar C",
+           "host": {"logical_cores": cores, "cpu_model": model}}
+    # all cores: one spawned process per core, 256 rows of A and W each
+    rows = 256
+    bands = [(i * rows, (i + 1) * rows) for i in range(cores)]
+    try:
+        ctx = mp.get_context("spawn")
+        with ctx.Pool(cores) as pool:
+            pool.map(_oracle_band, bands[:cores])          # import and build once per worker
+            t0 = time.perf_counter()
+            total = sum(pool.map(_oracle_band, bands))
+            dt_all = time.perf_counter() - t0
+        out["all_cores"] = {"value": round(total / dt_all / 1e9, 4), "unit": "GB/s", "cores": cores,
+                            "sample": f"{cores} processes x (256 rows of A and of W through every launch of "
+                                      f"the step), {dt_all:.3f} s"}
+    except Exception as e:  # the single-thread figure stands on its own
+        out["all_cores"] = {"unavailable": f"{type(e).__name__}: {e}"}
+    return out
 
 
 def run_reference(args, rank, world):
@@ -627,6 +743,7 @@ def run_reference(args, rank, world):
     step a bounded sample of the workload."""
     if rank != 0:
         return None
+    cores, model = host_cpu()
     run, nbytes, sample = oracle_sample(rows_a=256, rows_w=256)
     for _ in range(args.warmup):
         run()
@@ -641,7 +758,7 @@ def run_reference(args, rank, world):
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "sample": sample},
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "host": {"logical_cores": cores, "cpu_model": model}},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -752,6 +869,11 @@ def main():
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "step": [f"{n}:{t}" for n, t, _, _ in step_plan(__import__("microscaling_block_quantization_b200"))],
                    "step_algorithmic_bytes": r["step_bytes"], "hbm_frac_of_8TBs": round(r["value"] / world / 8000, 4),
+                   "quantize_only_GB_per_s": r["roofline"]["achieved"],
+                   "quantize_only_note": "the step's 8 quantizer launches (no dequantizer): their algorithmic bytes "
+                                         "over their summed launch durations, one stream",
+                   "per_launch_timing": f"per variant a graph of {R_PAIRS} back-to-back A/W launch pairs, "
+                                        "replayed K times (no graph-launch gap between launches)",
                    "l2": "inputs larger than L2 (A+W 176 MiB > 126 MB); consecutive launches alternate tensors",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "streams": "one" if args.one_stream else

@@ -69,11 +69,95 @@ __device__ __forceinline__ void hadamard_groups(float y[32])
     }
 }
 
+// ---- bf16 inputs kept packed (two elements a 32-bit word) ------------------
+// The block statistic is taken on the packed words (halfwise maximum of
+// magnitudes, NaN-propagating), and each element is widened and scaled in one
+// mixed-precision multiply-add, y * c + (-0) with y and c bf16 and the result
+// rounded once to binary32 (exact for a power-of-two c; c = 1 widens; the
+// -0 addend keeps the sign of a zero product): no separate unpacking.
+
+// halfwise max(|a|, |b|), NaN-propagating (the result's sign bits are unused)
+__device__ __forceinline__ uint32_t bf2_absmax(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+// halfwise min(|a|, |b|)
+__device__ __forceinline__ uint32_t bf2_absmin(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("min.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// max |y| (NaN-propagating) of the 2N values in N words, as binary32 (a tree)
+template <int N>
+__device__ __forceinline__ float bf_absmax(const uint32_t *w)
+{
+    uint32_t m[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) m[i] = w[i];
+#pragma unroll
+    for (int st = 1; st < N; st *= 2)
+#pragma unroll
+        for (int i = 0; i + st < N; i += 2 * st) m[i] = bf2_absmax(m[i], m[i + st]);
+    return fmax_nan(fabsf(__uint_as_float(m[0] << 16)), fabsf(__uint_as_float(m[0] & 0xffff0000u)));
+}
+// min |y| of the 2N values in N words, as binary32
+template <int N>
+__device__ __forceinline__ float bf_absmin(const uint32_t *w)
+{
+    uint32_t m[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) m[i] = w[i];
+#pragma unroll
+    for (int st = 1; st < N; st *= 2)
+#pragma unroll
+        for (int i = 0; i + st < N; i += 2 * st) m[i] = bf2_absmin(m[i], m[i + st]);
+    return fminf(fabsf(__uint_as_float(m[0] << 16)), fabsf(__uint_as_float(m[0] & 0xffff0000u)));
+}
+
+// the eight bf16 values of four words times the bf16 value c (low 16 bits),
+// each product rounded once to binary32
+__device__ __forceinline__ void bf16x8_scale(const uint32_t *w, uint32_t c, float s[8])
+{
+    asm("{\n\t.reg .b16 a0, a1, a2, a3, a4, a5, a6, a7, k, kx;\n\t.reg .f32 z;\n\t"
+        "mov.b32 {a0, a1}, %8;\n\t"
+        "mov.b32 {a2, a3}, %9;\n\t"
+        "mov.b32 {a4, a5}, %10;\n\t"
+        "mov.b32 {a6, a7}, %11;\n\t"
+        "mov.b32 {k, kx}, %12;\n\t"
+        "mov.f32 z, 0f80000000;\n\t"
+        "fma.rn.f32.bf16 %0, a0, k, z;\n\t"
+        "fma.rn.f32.bf16 %1, a1, k, z;\n\t"
+        "fma.rn.f32.bf16 %2, a2, k, z;\n\t"
+        "fma.rn.f32.bf16 %3, a3, k, z;\n\t"
+        "fma.rn.f32.bf16 %4, a4, k, z;\n\t"
+        "fma.rn.f32.bf16 %5, a5, k, z;\n\t"
+        "fma.rn.f32.bf16 %6, a6, k, z;\n\t"
+        "fma.rn.f32.bf16 %7, a7, k, z;\n\t}"
+        : "=f"(s[0]), "=f"(s[1]), "=f"(s[2]), "=f"(s[3]), "=f"(s[4]), "=f"(s[5]), "=f"(s[6]), "=f"(s[7])
+        : "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(c));
+}
+
+// Lane t's chunk of 32 bf16 values as 16 words, out of the swizzled tile.
+__device__ __forceinline__ void ring_read_words(const uint8_t *stage, int t, uint32_t w[16])
+{
+    const uint8_t *row = stage + 64 * t;
+    const int sw = (t >> 1) & 3;                       // 64-byte swizzle
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(row + 16 * (k ^ sw));
+        w[4 * k] = u.x; w[4 * k + 1] = u.y; w[4 * k + 2] = u.z; w[4 * k + 3] = u.w;
+    }
+}
+
 // HADN: block rotation over groups of HADN (0: none, 16, 32) before
 // quantization; MBS: 1 x 128 macro scale over the
 // 4 lanes of a macro block (consecutive chunks of a tile are consecutive lanes).
 template <typename InT, int B, bool STATS, int HADN, bool MBS, bool NEAR>
-__global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) k_quant_fast(const QParams p, const __grid_constant__ CUtensorMap tm)
+__global__ void __launch_bounds__(kFastThreads, (HADN || MBS || (STATS && sizeof(InT) != 2)) ? 2 : 3) k_quant_fast(const QParams p, const __grid_constant__ CUtensorMap tm)
 {
     constexpr int NB = B <= 32 ? 32 / B : 1;
     constexpr int G = B <= 32 ? 1 : B / 32;
@@ -117,6 +201,8 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) 
         // rotation with power-of-two scales: the normaliser c = 1/sqrt(n) moves
         // into the scale, s = y_H * (c * 2^-k) = (y_H * c) * 2^-k exactly
         constexpr bool FOLD = HADN != 0 && !MBS && !NEAR;
+        // bf16 input with neither rotation nor macro scale: kept packed
+        constexpr bool PACKED = sizeof(InT) == 2 && HADN == 0 && !MBS;
         const float hc = HADN ? hadamard_scale(HADN) : 1.0f;
         const bool e8m0 = !NEAR && p.sd.fmt == S_E8M0;
         const float thr_m = e8m0_threshold(p.ed, p.sd);
@@ -125,8 +211,10 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) 
         uint32_t i = 0;
         for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
             if (!ring.acquire(i, kWaitFull)) break;
-            float y[32];
-            ring_read_chunk(ring.stage(i % RingCfg<InT>::kStages), t, static_cast<const InT *>(nullptr), y);
+            float y[PACKED ? 1 : 32];
+            uint32_t w[PACKED ? 16 : 1];
+            if constexpr (PACKED) ring_read_words(ring.stage(i % RingCfg<InT>::kStages), t, w);
+            else ring_read_chunk(ring.stage(i % RingCfg<InT>::kStages), t, static_cast<const InT *>(nullptr), y);
             ring.release(i);                  // the chunk is in registers: hand the slot back
             if constexpr (HADN != 0) hadamard_groups<HADN, !FOLD>(y);
             // macro-block scale: y' = y * (1 / S_M), x_hat = (q X) S_M
@@ -154,6 +242,92 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) 
             uint32_t scode[NB];
             // packed two-lane binary32 arithmetic (each lane rounded as a scalar op)
             int nzc = 0, ftzc = 0;
+            if constexpr (PACKED) {
+#pragma unroll
+                for (int k = 0; k < NB; ++k) {
+                    const uint32_t *wb = w + k * (L / 2);
+                    float a = bf_absmax<L / 2>(wb), mabs = 1.0f;
+                    if (STATS) mabs = bf_absmin<L / 2>(wb);
+                    int bad = !(a <= FLT_MAX);
+                    if (G > 1) {
+                        a = grp_max(bad ? 0.0f : a, G);
+                        bad = grp_or(bad, G);
+                    }
+                    const BlockScale bs = NEAR ? near_block_scale(p.sd, ns, bad ? 0.0f : a, bad)
+                                        : e8m0 ? e8m0_block_scale(bad ? 0.0f : a, bad, p.ed.emax, thr_m)
+                                               : block_scale(p.ed, p.sd, bad ? 0.0f : a, bad, sT);
+                    scode[k] = bs.code;
+                    float deqT = bs.nan ? __uint_as_float(0x7fc00000u) : bs.deq;
+                    float inv = bs.inv;
+                    // a flushed block: residuals are the inputs themselves
+                    if (bs.zero && !bs.nan) {
+                        inv = 1.0f;
+                        deqT = 1.0f;
+                    }
+                    // power-of-two rules: s = y 2^-k straight from the packed
+                    // words (exact); nearest scales: widen, then multiply
+                    const uint32_t kb = NEAR ? 0x3f80u : (__float_as_uint(inv) >> 16);
+                    const float2 inv2 = make_float2(inv, inv);
+                    float2 sx2 = make_float2(0.f, 0.f), re2[2] = {sx2, sx2}, rb2[2] = {sx2, sx2};
+                    int qz = 0;
+#pragma unroll
+                    for (int g = 0; g < L / 8; ++g) {
+                        float s8[8];
+                        bf16x8_scale(wb + 4 * g, kb, s8);
+                        if (NEAR && STATS) {
+#pragma unroll
+                            for (int e = 0; e < 8; e += 2) {
+                                const float2 yv = make_float2(s8[e], s8[e + 1]);
+                                sx2 = __ffma2_rn(yv, yv, sx2);
+                            }
+                        }
+                        if (NEAR) {
+#pragma unroll
+                            for (int e = 0; e < 8; e += 2) {
+                                const float2 v = __fmul2_rn(make_float2(s8[e], s8[e + 1]), inv2);
+                                s8[e] = v.x;
+                                s8[e + 1] = v.y;
+                            }
+                        }
+                        const uint32_t word = bs.zero ? 0u : cvt_e2m1x8(s8);
+                        words[(k * L) / 8 + g] = word;
+                        if (STATS) {
+                            uint32_t h[4];
+                            e2m1x8_halves(word, h);
+#pragma unroll
+                            for (int e = 0; e < 8; e += 2) {
+                                const float2 d = sub_f16x2_from(s8[e], s8[e + 1], h[e >> 1]);   // s - q
+                                const int u = (e >> 1) & 1;
+                                re2[u] = __ffma2_rn(d, d, re2[u]);
+                                rb2[u] = __fadd2_rn(rb2[u], d);
+                                if (!NEAR) {
+                                    // y = 2^k s exactly: sum s^2, scaled below
+                                    const float2 sv = make_float2(s8[e], s8[e + 1]);
+                                    sx2 = __ffma2_rn(sv, sv, sx2);
+                                }
+                            }
+                            qz += zero_codes8(word);
+                        }
+                    }
+                    if (STATS) {
+                        if (ok) {
+                            const double X = (double)deqT;
+                            // reference values y = R s: R = 1 (nearest: sums of y), 2^k, or 1 in a flushed block
+                            const double R = NEAR ? 1.0 : (bs.zero && !bs.nan) ? 1.0 : (double)bs.deq;
+                            acc.e2 += (double)((re2[0].x + re2[1].x) + (re2[0].y + re2[1].y)) * X * X;
+                            acc.e -= (double)((rb2[0].x + rb2[1].x) + (rb2[0].y + rb2[1].y)) * X;
+                            acc.x2 += (double)(sx2.x + sx2.y) * R * R;
+                        }
+                        int xz = 0;
+                        if (mabs == 0.0f)                  // rare: count exact zeros
+#pragma unroll
+                            for (int j = 0; j < L / 2; ++j)
+                                xz += ((wb[j] & 0x7fffu) == 0u) + ((wb[j] & 0x7fff0000u) == 0u);
+                        nzc += L - xz;
+                        if (!bs.nan) ftzc += qz - xz;
+                    }
+                }
+            } else {
 #pragma unroll
             for (int k = 0; k < NB; ++k) {
                 const int j0 = k * L;
@@ -238,6 +412,7 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || STATS) ? 2 : 3) 
                     nzc += L - xz;
                     if (!bs.nan) ftzc += qz - xz;
                 }
+            }
             }
             if (ok) {
                 reinterpret_cast<uint4 *>(p.codes)[c] = make_uint4(words[0], words[1], words[2], words[3]);
