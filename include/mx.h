@@ -343,6 +343,17 @@ int mx_gemm_qsnr(const mx_config *ca, const mx_config *cb, const void *A, const 
                  void *workspace, int64_t workspace_bytes, void *stream);
 
 /*
+ * mx_gemm_qsnr_finalize -- recomputes entry [2] (QSNR dB, [MXFP4-OAS] Sec.3
+ * Eq. (2)) of a 3-double mx_gemm_qsnr stats buffer (device) from its two sums
+ * [0] and [1]: after the sums of several row bands of A (each band's
+ * mx_gemm_qsnr against the same B) were added together across ranks, the
+ * buffer then holds the whole product's QSNR.  A zero reference gives NaN, a
+ * zero error +inf.  The pages have no multi-device procedure: this is how
+ * QSNR(AB) stays the one of the whole product when A is split by rows.
+ */
+int mx_gemm_qsnr_finalize(double *stats, void *stream);
+
+/*
  * mx_mbs_gemm_scales -- an MBS operand ([MXFP4-OAS] Sec.4 Macro Block
  * Scaling: E2M1 codes, E8M0 scale X per 1 x 32 block, E4M3 macro scale S_M per
  * 1 x 128, x_hat = q X S_M) as an operand of mx_gemm's NVFP4 kind.  The pages

@@ -115,12 +115,13 @@ def lib() -> C.CDLL:
         L.mx_device_status.argtypes = [P, C.POINTER(i32)]
         L.mx_tensor_amax.argtypes = [cfgp, P, i32, i64, i64, P, i64, P]
         L.mx_stats_finalize.argtypes = [P, P]
+        L.mx_gemm_qsnr_finalize.argtypes = [P, P]
         L.mx_strerror.argtypes = [C.c_int]
         L.mx_strerror.restype = C.c_char_p
         L.mx_version.restype = C.c_char_p
         for f in ("mx_query_sizes", "mx_quantize", "mx_quantize_noalloc", "mx_hadamard_quantize", "mx_dequantize",
                   "mx_qsnr", "mx_gemm", "mx_gemm_qsnr", "mx_mbs_gemm_scales", "mx_device_status",
-                  "mx_tensor_amax", "mx_stats_finalize"):
+                  "mx_tensor_amax", "mx_stats_finalize", "mx_gemm_qsnr_finalize"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -187,6 +188,10 @@ def mx_tensor_amax(cfg: Config, x, x_dtype, rows, cols, workspace, workspace_byt
 
 def mx_stats_finalize(stats, stream) -> int:
     return lib().mx_stats_finalize(stats, stream)
+
+
+def mx_gemm_qsnr_finalize(stats, stream) -> int:
+    return lib().mx_gemm_qsnr_finalize(stats, stream)
 
 
 def mx_quantize_noalloc(cfg: Config, x, x_dtype, rows, cols, codes, scales, tensor_scale, macro,
@@ -345,6 +350,13 @@ def stats_finalize(stats: torch.Tensor, stream=None) -> torch.Tensor:
     """Recompute MSE / R-MSE / QSNR / bias / flush share of a stats buffer from
     its sums and count, in place (``mx_stats_finalize``)."""
     _check("mx_stats_finalize", mx_stats_finalize(_p(stats), _stream(stream)))
+    return stats
+
+
+def gemm_qsnr_finalize(stats: torch.Tensor, stream=None) -> torch.Tensor:
+    """Recompute the dB entry of a QSNR(AB) stats buffer (float64[3] on the
+    device) from its two sums, in place (``mx_gemm_qsnr_finalize``)."""
+    _check("mx_gemm_qsnr_finalize", mx_gemm_qsnr_finalize(_p(stats), _stream(stream)))
     return stats
 
 

@@ -1155,6 +1155,15 @@ int mx_gemm_qsnr(const mx_config *ca, const mx_config *cb, const void *A, const 
     return launch_qsnr_kind<KIND_NVF4>(p, Aq, Bq, A, B, st);
 }
 
+int mx_gemm_qsnr_finalize(double *stats, void *stream)
+{
+    if (!stats) return MX_ERR_INVALID;
+    if ((uintptr_t)stats & 7u) return MX_ERR_ALIGN;
+    // one record: the buffer's own two sums, read before the three entries are written
+    k_gemm_qsnr_finalize<<<1, 256, 0, static_cast<cudaStream_t>(stream)>>>(stats, 1, stats);
+    return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+}
+
 int mx_device_status(void *stream, int32_t *status)
 {
     if (!status) return MX_ERR_INVALID;

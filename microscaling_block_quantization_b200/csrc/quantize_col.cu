@@ -596,6 +596,315 @@ __global__ void __launch_bounds__(kColThreads) k_amax_col(const QParams p)
     if (lane == 0 && m > 0.0f) atomicMax(p.amax_word, __float_as_uint(m));
 }
 
+// ---------------------------------------------------------------------------
+// bf16 input, E2M1 round-to-nearest-even, symmetric, no macro scale or
+// rotation: column-wise B x 1 blocks and 2D 32 x 32 tiles.  Every warp owns
+// two tile buffers of RB rows x 128 columns (RB = B, or 32 for 2D; 256 bytes a
+// row) and keeps the next tile's 16-byte cp.async copies in flight while it
+// works the current one; lane l works columns 4l .. 4l + 3 of the tile (an
+// 8-byte slot of every row).  The column statistics are taken on the packed
+// bf16x2 words (halfwise maximum and minimum of magnitudes), each element is
+// scaled in one mixed-precision multiply-add (y * 2^-k exactly; nearest
+// scales: widened, then multiplied), and the fidelity sums are formed on the
+// scaled values, s - q with q decoded by the conversion instruction, times
+// the block's scale once per block.
+constexpr int kColxWarps = 12;
+constexpr int kColxThreads = kColxWarps * 32;
+constexpr int kColxTileRows = 32;
+constexpr int kColxCols = 128;                              // columns of a tile
+constexpr int kColxBufBytes = kColxTileRows * kColxCols * 2;    // 8 KB
+
+__device__ __forceinline__ uint32_t bfx_absmax(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ uint32_t bfx_absmin(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("min.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+// |half h| of a bf16x2 word as binary32
+__device__ __forceinline__ float bfx_half_abs(uint32_t w, int h)
+{
+    return fabsf(__uint_as_float(h ? (w & 0xffff0000u) : (w << 16)));
+}
+// the two bf16 values of a word times the bf16 values k0 / k1 (low 16 bits),
+// each product rounded once to binary32
+__device__ __forceinline__ float2 bfx_scale2(uint32_t w, uint32_t k0, uint32_t k1)
+{
+    float a, b;
+    asm("{\n\t.reg .b16 y0, y1, c0, c1, cx;\n\t.reg .f32 z;\n\t"
+        "mov.b32 {y0, y1}, %2;\n\t"
+        "mov.b32 {c0, cx}, %3;\n\t"
+        "mov.b32 {c1, cx}, %4;\n\t"
+        "mov.f32 z, 0f80000000;\n\t"
+        "fma.rn.f32.bf16 %0, y0, c0, z;\n\t"
+        "fma.rn.f32.bf16 %1, y1, c1, z;\n\t}"
+        : "=f"(a), "=f"(b) : "r"(w), "r"(k0), "r"(k1));
+    return make_float2(a, b);
+}
+// four binary32 values -> four E2M1 nibbles (the first in bits 0..3)
+__device__ __forceinline__ uint32_t cvt_e2m1x4(const float v[4])
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1;\n\t.reg .b16 h;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "mov.b16 h, {b0, b1};\n\t"
+        "cvt.u32.u16 %0, h;\n\t}"
+        : "=r"(r) : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]));
+    return r;
+}
+
+template <int AXIS, bool STATS, bool NEAR>
+__global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
+{
+    constexpr int NS = (AXIS == AX_COL) ? 4 : 1;          // blocks a lane holds per tile
+    extern __shared__ uint4 smem[];
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int RB = (AXIS == AX_2D) ? 32 : p.block;
+    uint8_t *const bufs = reinterpret_cast<uint8_t *>(smem) + (size_t)w * 2 * kColxBufBytes;
+    const int64_t ngc = (p.cols + kColxCols - 1) / kColxCols;
+    const int64_t nitems = (p.rows / RB) * ngc;
+    const int64_t gw = (int64_t)blockIdx.x * kColxWarps + w, nw = (int64_t)gridDim.x * kColxWarps;
+    const float sT = launch_tensor_scale(p);
+    // nearest scales: s_b s_T and its reciprocal for every scale code, once per CTA
+    __shared__ float2 near_tab[NEAR ? 256 : 1];
+    if constexpr (NEAR)
+        for (int c = threadIdx.x; c < 256; c += blockDim.x) {
+            const float d = __fmul_rn(ue_value(p.sd, (uint32_t)c), sT);
+            near_tab[c] = c < p.sd.ue_nan_code ? make_float2(d, __fdiv_rn(1.0f, d))
+                                               : make_float2(__uint_as_float(0x7fc00000u), 0.0f);
+        }
+    __syncthreads();
+    NearScale ns;
+    ns.maxv = p.ed.maxv;
+    ns.r_max = __fdiv_rn(1.0f, p.ed.maxv);
+    ns.sT = sT;
+    ns.r_T = (sT >= 0x1p-125f && sT <= 0x1p125f) ? __fdiv_rn(1.0f, sT) : 0.0f;
+    {
+        const float ms = __fmul_rn(p.ed.maxv, sT);
+        ns.c = (ms >= 0x1p-125f && ms <= 0x1p125f) ? __fdiv_rn(1.0f, ms) : 0.0f;
+    }
+    ns.tab = near_tab;
+    const bool e8m0 = !NEAR && p.sd.fmt == S_E8M0;
+    const float thr_m = e8m0_threshold(p.ed, p.sd);
+    const uint8_t *const xb = static_cast<const uint8_t *>(p.x);
+    const int64_t pitch = p.cols * 2;                        // bytes per row
+    Acc acc = {0, 0, 0, 0, 0};
+
+    // the tile's RB rows x 256 bytes as 16-byte copies, RB / 2 per lane
+    auto issue = [&](int64_t item, uint8_t *buf) {
+        const int64_t rg = item / ngc, cg = item - rg * ngc;
+        for (int k = 0; k < RB / 2; ++k) {
+            const int f = k * 32 + lane, r = f >> 4, ch = f & 15;
+            const int64_t cb = cg * (kColxCols * 2) + ch * 16;
+            const bool in = cb < pitch;
+            const uint8_t *src = in ? xb + (rg * RB + r) * pitch + cb : xb;
+            cp_async16(buf + r * 256 + ch * 16, src, in);
+        }
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+    };
+
+    int cur = 0;
+    if (gw < nitems) issue(gw, bufs);
+    for (int64_t item = gw; item < nitems; item += nw, cur ^= 1) {
+        const uint2 *b = reinterpret_cast<const uint2 *>(bufs + cur * kColxBufBytes) + lane;
+        if (item + nw < nitems) {
+            // the other buffer was read in the previous iteration by every lane
+            __syncwarp();
+            issue(item + nw, bufs + (cur ^ 1) * kColxBufBytes);
+            asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+        }
+        __syncwarp();                    // every lane's copies of this tile have landed
+        const int64_t rg = item / ngc, cg = item - rg * ngc;
+        const int64_t c0 = cg * kColxCols + lane * 4;
+        const bool ok = c0 < p.cols;
+        const int64_t r0 = rg * RB;
+
+        // column statistics on the packed words (two chains per word)
+        uint32_t am[4] = {0u, 0u, 0u, 0u}, mn[4] = {0x7f807f80u, 0x7f807f80u, 0x7f807f80u, 0x7f807f80u};
+#pragma unroll 4
+        for (int r = 0; r < RB; r += 2) {
+            const uint2 u0 = b[r * 32], u1 = b[(r + 1) * 32];
+            am[0] = bfx_absmax(am[0], u0.x);
+            am[1] = bfx_absmax(am[1], u0.y);
+            am[2] = bfx_absmax(am[2], u1.x);
+            am[3] = bfx_absmax(am[3], u1.y);
+            if (STATS) {
+                mn[0] = bfx_absmin(mn[0], u0.x);
+                mn[1] = bfx_absmin(mn[1], u0.y);
+                mn[2] = bfx_absmin(mn[2], u1.x);
+                mn[3] = bfx_absmin(mn[3], u1.y);
+            }
+        }
+        float a[4], mabs[4];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const uint32_t m = bfx_absmax(am[i], am[2 + i]);
+            a[2 * i] = bfx_half_abs(m, 0);
+            a[2 * i + 1] = bfx_half_abs(m, 1);
+            const uint32_t n = bfx_absmin(mn[i], mn[2 + i]);
+            mabs[2 * i] = bfx_half_abs(n, 0);
+            mabs[2 * i + 1] = bfx_half_abs(n, 1);
+        }
+
+        // shared scales: one per column (column axis) or per 32 x 32 tile (8 lanes)
+        BlockScale bs[NS];
+        if constexpr (AXIS == AX_COL) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int bad = !(a[j] <= FLT_MAX);
+                bs[j] = NEAR ? near_block_scale(p.sd, ns, bad ? 0.0f : a[j], bad)
+                      : e8m0 ? e8m0_block_scale(bad ? 0.0f : a[j], bad, p.ed.emax, thr_m)
+                             : block_scale(p.ed, p.sd, bad ? 0.0f : a[j], bad, sT);
+            }
+        } else {
+            float m = fmax_nan(fmax_nan(a[0], a[1]), fmax_nan(a[2], a[3]));
+            int bad = !(m <= FLT_MAX);
+            m = grp_max(bad ? 0.0f : m, 8);
+            bad = grp_or(bad, 8);
+            bs[0] = NEAR ? near_block_scale(p.sd, ns, m, bad)
+                  : e8m0 ? e8m0_block_scale(m, bad, p.ed.emax, thr_m)
+                         : block_scale(p.ed, p.sd, m, bad, sT);
+        }
+        if (ok) {
+            if constexpr (AXIS == AX_COL) {
+                const uint32_t w0 = bs[0].code | (bs[1].code << 8) | (bs[2].code << 16) | (bs[3].code << 24);
+                *reinterpret_cast<uint32_t *>(p.scales + (r0 / RB) * p.cols + c0) = w0;
+            } else if ((lane & 7) == 0) {
+                p.scales[(r0 / 32) * (p.cols / 32) + c0 / 32] = (uint8_t)bs[0].code;
+            }
+        }
+
+        // per column: multiplier (bf16 bits for the power-of-two rules), the
+        // nibble mask of flushed blocks, dequantization and reference factors
+        uint32_t kb[4], zmask = 0xffffu;
+        float inv[4], X[4], R[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const BlockScale &s = bs[(AXIS == AX_COL) ? j : 0];
+            const bool flush = s.zero && !s.nan;
+            inv[j] = flush ? 1.0f : s.inv;
+            kb[j] = NEAR ? 0x3f80u : (__float_as_uint(inv[j]) >> 16);
+            if (s.zero) zmask &= ~(0xfu << (4 * j));
+            X[j] = s.nan ? __uint_as_float(0x7fc00000u) : flush ? 1.0f : s.deq;
+            R[j] = (NEAR || flush) ? 1.0f : s.deq;
+        }
+
+        float2 re2[2], rb2[2], sx2[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            re2[i] = make_float2(0.f, 0.f);
+            rb2[i] = re2[i];
+            sx2[i] = re2[i];
+        }
+        int qz = 0;
+        uint8_t *const codes = static_cast<uint8_t *>(p.codes) + (r0 * p.cols + c0) / 2;
+#pragma unroll 4
+        for (int r = 0; r < RB; ++r) {
+            const uint2 u = b[r * 32];
+            const uint32_t v[2] = {u.x, u.y};
+            float s4[4];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                float2 sv = bfx_scale2(v[i], kb[2 * i], kb[2 * i + 1]);
+                if (NEAR) {
+                    if (STATS) sx2[i] = __ffma2_rn(sv, sv, sx2[i]);       // reference y
+                    sv = __fmul2_rn(sv, make_float2(inv[2 * i], inv[2 * i + 1]));
+                }
+                s4[2 * i] = sv.x;
+                s4[2 * i + 1] = sv.y;
+            }
+            const uint32_t word = cvt_e2m1x4(s4) & zmask;
+            if (ok) *reinterpret_cast<uint16_t *>(codes + (int64_t)r * (p.cols / 2)) = (uint16_t)word;
+            if (STATS) {
+                uint32_t h0, h1;
+                asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
+                    "mov.b32 {c0, c1, c2, c3}, %2;\n\t"
+                    "cvt.rn.f16x2.e2m1x2 %0, c0;\n\t"
+                    "cvt.rn.f16x2.e2m1x2 %1, c1;\n\t}"
+                    : "=r"(h0), "=r"(h1) : "r"(word));
+                const uint32_t h[2] = {h0, h1};
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float2 d = sub_f16x2_from(s4[2 * i], s4[2 * i + 1], h[i]);   // s - q
+                    re2[i] = __ffma2_rn(d, d, re2[i]);
+                    rb2[i] = __fadd2_rn(rb2[i], d);
+                    if (!NEAR) {
+                        const float2 sv = make_float2(s4[2 * i], s4[2 * i + 1]);
+                        sx2[i] = __ffma2_rn(sv, sv, sx2[i]);                 // y = R s
+                    }
+                }
+                qz += 4 - __popc(((word & 0x7777u) + 0x7777u) & 0x8888u);
+            }
+        }
+        if (STATS && ok) {
+            // y - x_hat = X (s - q) per column; reference sums R^2 sum s^2 (or sum y^2)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = j >> 1;
+                const float e = (j & 1) ? re2[i].y : re2[i].x, bb = (j & 1) ? rb2[i].y : rb2[i].x;
+                const float sx = (j & 1) ? sx2[i].y : sx2[i].x;
+                const double Xd = (double)X[j], Rd = (double)R[j];
+                acc.e2 += (double)e * Xd * Xd;
+                acc.e -= (double)bb * Xd;
+                acc.x2 += (double)sx * Rd * Rd;
+            }
+            // exact zeros (rare), nonzero and flushed counts; NaN blocks
+            // (all codes zero) are not flushes
+            int xzt = 0, nanz = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                int xz = 0;
+                if (mabs[j] == 0.0f)
+                    for (int r = 0; r < RB; ++r) {
+                        const uint2 u = b[r * 32];
+                        const uint32_t vv = (j >> 1) ? u.y : u.x;
+                        xz += ((vv >> (16 * (j & 1))) & 0x7fffu) == 0u;
+                    }
+                xzt += xz;
+                nanz += bs[(AXIS == AX_COL) ? j : 0].nan ? RB : xz;
+            }
+            acc.nz += (double)(4 * RB - xzt);
+            acc.ftz += (double)(qz - nanz);
+        }
+    }
+    finish_launch(p, acc);
+}
+
+template <int AXIS, bool STATS, bool NEAR>
+int launch_colx_k(const QParams &p, cudaStream_t st, int *grid_out)
+{
+    auto k = k_quant_colx<AXIS, STATS, NEAR>;
+    const size_t smem = (size_t)kColxWarps * 2 * kColxBufBytes;
+    const int occ = cached_occupancy(reinterpret_cast<const void *>(k), kColxThreads, smem);
+    const int RB = (AXIS == AX_2D) ? 32 : p.block;
+    const int64_t items = (p.rows / RB) * ((p.cols + kColxCols - 1) / kColxCols);
+    int64_t g = (int64_t)device_sm_count() * occ;
+    const int64_t need = (items + kColxWarps - 1) / kColxWarps;
+    if (need < g) g = need;
+    if (g < 1) g = 1;
+    if (g > kMaxPartials) g = kMaxPartials;
+    k<<<(unsigned)g, kColxThreads, smem, st>>>(p);
+    if (grid_out) *grid_out = (int)g;
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+template <int AXIS>
+int launch_colx(const QParams &p, cudaStream_t st, int *grid_out)
+{
+    const bool near = p.sd.fmt != S_E8M0 && p.sd.rule == R_NEAREST;
+    if (p.partials)
+        return near ? launch_colx_k<AXIS, true, true>(p, st, grid_out) : launch_colx_k<AXIS, true, false>(p, st, grid_out);
+    return near ? launch_colx_k<AXIS, false, true>(p, st, grid_out) : launch_colx_k<AXIS, false, false>(p, st, grid_out);
+}
+
 template <typename K>
 int launch_k(K kernel, const QParams &p, int64_t work_warps, size_t smem, cudaStream_t st,
              int *grid_out)
@@ -628,6 +937,8 @@ int launch_axis(const QParams &p, int fast, cudaStream_t st, int *grid_out)
         return launch_col_k<InT, 4, AXIS, false, true>(p, st, grid_out);
     }
     if constexpr (sizeof(InT) == 2) {
+        // E2M1 nearest-even without a macro scale: the double-buffered kernel
+        if (fast && !p.mbs && p.ed.elem == 0) return launch_colx<AXIS>(p, st, grid_out);
         if (p.ed.code_bits == 4) {
             if (fast) return launch_col_k<InT, 8, AXIS, true, false>(p, st, grid_out);
             return launch_col_k<InT, 8, AXIS, false, false>(p, st, grid_out);

@@ -46,14 +46,16 @@ __device__ __forceinline__ void butterfly_stage2(float y[32])
         }
 }
 
-template <int N, bool SCALE = true>
+template <int N, bool SCALE = true, bool STAGE1 = true>
 __device__ __forceinline__ void hadamard_groups(float y[32])
 {
+    if constexpr (STAGE1) {
 #pragma unroll
-    for (int j = 0; j < 32; j += 2) {
-        const float a = y[j], b = y[j + 1];
-        y[j] = __fadd_rn(a, b);
-        y[j + 1] = __fsub_rn(a, b);
+        for (int j = 0; j < 32; j += 2) {
+            const float a = y[j], b = y[j + 1];
+            y[j] = __fadd_rn(a, b);
+            y[j + 1] = __fsub_rn(a, b);
+        }
     }
     butterfly_stage2<2>(y);
     butterfly_stage2<4>(y);
@@ -141,6 +143,38 @@ __device__ __forceinline__ void bf16x8_scale(const uint32_t *w, uint32_t c, floa
         : "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(c));
 }
 
+// First butterfly stage of the rotation straight from four bf16 words: for
+// the pair (a, b) of each word, b + a and a - b rounded once to binary32
+// (a widened exactly, then b * (+1 / -1) + a in one mixed-precision
+// multiply-add each) -- the values of the binary32 additions on the widened
+// pair.
+__device__ __forceinline__ void bf16x8_stage1(const uint32_t *w, float y[8])
+{
+    asm("{\n\t.reg .b16 a0, b0, a1, b1, a2, b2, a3, b3, p1, m1;\n\t"
+        ".reg .f32 z, t0, t1, t2, t3;\n\t"
+        "mov.b32 {a0, b0}, %8;\n\t"
+        "mov.b32 {a1, b1}, %9;\n\t"
+        "mov.b32 {a2, b2}, %10;\n\t"
+        "mov.b32 {a3, b3}, %11;\n\t"
+        "mov.b16 p1, 0x3F80;\n\t"
+        "mov.b16 m1, 0xBF80;\n\t"
+        "mov.f32 z, 0f80000000;\n\t"
+        "fma.rn.f32.bf16 t0, a0, p1, z;\n\t"
+        "fma.rn.f32.bf16 t1, a1, p1, z;\n\t"
+        "fma.rn.f32.bf16 t2, a2, p1, z;\n\t"
+        "fma.rn.f32.bf16 t3, a3, p1, z;\n\t"
+        "fma.rn.f32.bf16 %0, b0, p1, t0;\n\t"
+        "fma.rn.f32.bf16 %1, b0, m1, t0;\n\t"
+        "fma.rn.f32.bf16 %2, b1, p1, t1;\n\t"
+        "fma.rn.f32.bf16 %3, b1, m1, t1;\n\t"
+        "fma.rn.f32.bf16 %4, b2, p1, t2;\n\t"
+        "fma.rn.f32.bf16 %5, b2, m1, t2;\n\t"
+        "fma.rn.f32.bf16 %6, b3, p1, t3;\n\t"
+        "fma.rn.f32.bf16 %7, b3, m1, t3;\n\t}"
+        : "=f"(y[0]), "=f"(y[1]), "=f"(y[2]), "=f"(y[3]), "=f"(y[4]), "=f"(y[5]), "=f"(y[6]), "=f"(y[7])
+        : "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]));
+}
+
 // Lane t's chunk of 32 bf16 values as 16 words, out of the swizzled tile.
 __device__ __forceinline__ void ring_read_words(const uint8_t *stage, int t, uint32_t w[16])
 {
@@ -157,7 +191,7 @@ __device__ __forceinline__ void ring_read_words(const uint8_t *stage, int t, uin
 // quantization; MBS: 1 x 128 macro scale over the
 // 4 lanes of a macro block (consecutive chunks of a tile are consecutive lanes).
 template <typename InT, int B, bool STATS, int HADN, bool MBS, bool NEAR>
-__global__ void __launch_bounds__(kFastThreads, (HADN || MBS || (STATS && sizeof(InT) != 2)) ? 2 : 3) k_quant_fast(const QParams p, const __grid_constant__ CUtensorMap tm)
+__global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && sizeof(InT) != 2)) ? 2 : 3) k_quant_fast(const QParams p, const __grid_constant__ CUtensorMap tm)
 {
     constexpr int NB = B <= 32 ? 32 / B : 1;
     constexpr int G = B <= 32 ? 1 : B / 32;
@@ -201,8 +235,9 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || (STATS && sizeof
         // rotation with power-of-two scales: the normaliser c = 1/sqrt(n) moves
         // into the scale, s = y_H * (c * 2^-k) = (y_H * c) * 2^-k exactly
         constexpr bool FOLD = HADN != 0 && !MBS && !NEAR;
-        // bf16 input with neither rotation nor macro scale: kept packed
-        constexpr bool PACKED = sizeof(InT) == 2 && HADN == 0 && !MBS;
+        // bf16 input without rotation: kept packed
+        constexpr bool PACKED = sizeof(InT) == 2 && HADN == 0;
+        constexpr bool ROT16 = sizeof(InT) == 2 && HADN != 0;
         const float hc = HADN ? hadamard_scale(HADN) : 1.0f;
         const bool e8m0 = !NEAR && p.sd.fmt == S_E8M0;
         const float thr_m = e8m0_threshold(p.ed, p.sd);
@@ -212,14 +247,21 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || (STATS && sizeof
         for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
             if (!ring.acquire(i, kWaitFull)) break;
             float y[PACKED ? 1 : 32];
-            uint32_t w[PACKED ? 16 : 1];
-            if constexpr (PACKED) ring_read_words(ring.stage(i % RingCfg<InT>::kStages), t, w);
+            uint32_t w[PACKED || ROT16 ? 16 : 1];
+            if constexpr (PACKED || ROT16) ring_read_words(ring.stage(i % RingCfg<InT>::kStages), t, w);
             else ring_read_chunk(ring.stage(i % RingCfg<InT>::kStages), t, static_cast<const InT *>(nullptr), y);
             ring.release(i);                  // the chunk is in registers: hand the slot back
-            if constexpr (HADN != 0) hadamard_groups<HADN, !FOLD>(y);
+            if constexpr (ROT16) {
+                // bf16 rotation: the first butterfly stage widens the pairs
+#pragma unroll
+                for (int g = 0; g < 4; ++g) bf16x8_stage1(w + 4 * g, y + 8 * g);
+                hadamard_groups<HADN, !FOLD, false>(y);
+            } else if constexpr (HADN != 0) {
+                hadamard_groups<HADN, !FOLD>(y);
+            }
             // macro-block scale: y' = y * (1 / S_M), x_hat = (q X) S_M
             float sm = 1.0f;
-            if constexpr (MBS) {
+            if constexpr (MBS && !PACKED) {
                 const float m = absmax_nan<32>(y);
                 int mbad = !(m <= FLT_MAX);
                 float mm = grp_max(mbad ? 0.0f : m, 4);
@@ -243,48 +285,87 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || (STATS && sizeof
             // packed two-lane binary32 arithmetic (each lane rounded as a scalar op)
             int nzc = 0, ftzc = 0;
             if constexpr (PACKED) {
+                // block statistics of the packed words
+                float a[NB], mn[NB];
+                int bad[NB];
+#pragma unroll
+                for (int k = 0; k < NB; ++k) {
+                    a[k] = bf_absmax<L / 2>(w + k * (L / 2));
+                    mn[k] = STATS ? bf_absmin<L / 2>(w + k * (L / 2)) : 1.0f;
+                    bad[k] = !(a[k] <= FLT_MAX);
+                    if (G > 1) {
+                        a[k] = grp_max(bad[k] ? 0.0f : a[k], G);
+                        bad[k] = grp_or(bad[k], G);
+                    }
+                }
+                // macro-block scale over the 4 lanes of a 1 x 128 block; the
+                // block rule then sees y' = RN(y / S_M), whose block max and
+                // min are RN(max |y| / S_M) and RN(min |y| / S_M) (rounding is
+                // monotone)
+                float sm = 1.0f, invm = 1.0f;
+                if constexpr (MBS) {
+                    float m = a[0];
+                    int mbad = bad[0];
+#pragma unroll
+                    for (int k = 1; k < NB; ++k) {
+                        m = fmax_nan(m, a[k]);
+                        mbad |= bad[k];
+                    }
+                    const float mm = grp_max(mbad ? 0.0f : m, 4);
+                    mbad = grp_or(mbad, 4);
+                    const uint32_t mcode = macro_code(p.ed, mm, mbad);
+                    sm = e4m3_value(mcode);
+                    invm = __fdiv_rn(1.0f, sm);
+                    if ((t & 3) == 0 && ok) p.macro[c >> 2] = (uint8_t)mcode;
+#pragma unroll
+                    for (int k = 0; k < NB; ++k) {
+                        a[k] = __fmul_rn(a[k], invm);
+                        mn[k] = __fmul_rn(mn[k], invm);
+                    }
+                }
 #pragma unroll
                 for (int k = 0; k < NB; ++k) {
                     const uint32_t *wb = w + k * (L / 2);
-                    float a = bf_absmax<L / 2>(wb), mabs = 1.0f;
-                    if (STATS) mabs = bf_absmin<L / 2>(wb);
-                    int bad = !(a <= FLT_MAX);
-                    if (G > 1) {
-                        a = grp_max(bad ? 0.0f : a, G);
-                        bad = grp_or(bad, G);
-                    }
-                    const BlockScale bs = NEAR ? near_block_scale(p.sd, ns, bad ? 0.0f : a, bad)
-                                        : e8m0 ? e8m0_block_scale(bad ? 0.0f : a, bad, p.ed.emax, thr_m)
-                                               : block_scale(p.ed, p.sd, bad ? 0.0f : a, bad, sT);
+                    const BlockScale bs = NEAR ? near_block_scale(p.sd, ns, bad[k] ? 0.0f : a[k], bad[k])
+                                        : e8m0 ? e8m0_block_scale(bad[k] ? 0.0f : a[k], bad[k], p.ed.emax, thr_m)
+                                               : block_scale(p.ed, p.sd, bad[k] ? 0.0f : a[k], bad[k], sT);
                     scode[k] = bs.code;
                     float deqT = bs.nan ? __uint_as_float(0x7fc00000u) : bs.deq;
-                    float inv = bs.inv;
+                    if (MBS) deqT = __fmul_rn(deqT, sm);       // X S_M, exact (E4M3 times a power of two)
+                    float inv = bs.inv, im = invm;
                     // a flushed block: residuals are the inputs themselves
-                    if (bs.zero && !bs.nan) {
+                    const bool flush = bs.zero && !bs.nan;
+                    if (flush) {
                         inv = 1.0f;
+                        im = 1.0f;
                         deqT = 1.0f;
                     }
                     // power-of-two rules: s = y 2^-k straight from the packed
-                    // words (exact); nearest scales: widen, then multiply
-                    const uint32_t kb = NEAR ? 0x3f80u : (__float_as_uint(inv) >> 16);
-                    const float2 inv2 = make_float2(inv, inv);
+                    // words (exact); nearest scales and MBS: widen, then
+                    // multiply (MBS: by 1 / S_M, then by 2^-k, as the rule is
+                    // defined on y')
+                    constexpr bool WIDEN = NEAR || MBS;
+                    const uint32_t kb = WIDEN ? 0x3f80u : (__float_as_uint(inv) >> 16);
+                    const float2 inv2 = make_float2(inv, inv), im2 = make_float2(im, im);
                     float2 sx2 = make_float2(0.f, 0.f), re2[2] = {sx2, sx2}, rb2[2] = {sx2, sx2};
                     int qz = 0;
 #pragma unroll
                     for (int g = 0; g < L / 8; ++g) {
                         float s8[8];
                         bf16x8_scale(wb + 4 * g, kb, s8);
-                        if (NEAR && STATS) {
+                        if (WIDEN && STATS) {
 #pragma unroll
                             for (int e = 0; e < 8; e += 2) {
                                 const float2 yv = make_float2(s8[e], s8[e + 1]);
                                 sx2 = __ffma2_rn(yv, yv, sx2);
                             }
                         }
-                        if (NEAR) {
+                        if (WIDEN) {
 #pragma unroll
                             for (int e = 0; e < 8; e += 2) {
-                                const float2 v = __fmul2_rn(make_float2(s8[e], s8[e + 1]), inv2);
+                                float2 v = make_float2(s8[e], s8[e + 1]);
+                                if (MBS) v = __fmul2_rn(v, im2);
+                                v = __fmul2_rn(v, inv2);
                                 s8[e] = v.x;
                                 s8[e + 1] = v.y;
                             }
@@ -300,7 +381,7 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || (STATS && sizeof
                                 const int u = (e >> 1) & 1;
                                 re2[u] = __ffma2_rn(d, d, re2[u]);
                                 rb2[u] = __fadd2_rn(rb2[u], d);
-                                if (!NEAR) {
+                                if (!WIDEN) {
                                     // y = 2^k s exactly: sum s^2, scaled below
                                     const float2 sv = make_float2(s8[e], s8[e + 1]);
                                     sx2 = __ffma2_rn(sv, sv, sx2);
@@ -311,15 +392,16 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || MBS || (STATS && sizeof
                     }
                     if (STATS) {
                         if (ok) {
+                            // y - x_hat = deqT (s - q); reference sums of y (R = 1)
+                            // or of s with y = 2^k s (R = 2^k; 1 in a flushed block)
                             const double X = (double)deqT;
-                            // reference values y = R s: R = 1 (nearest: sums of y), 2^k, or 1 in a flushed block
-                            const double R = NEAR ? 1.0 : (bs.zero && !bs.nan) ? 1.0 : (double)bs.deq;
+                            const double R = (WIDEN || flush) ? 1.0 : (double)bs.deq;
                             acc.e2 += (double)((re2[0].x + re2[1].x) + (re2[0].y + re2[1].y)) * X * X;
                             acc.e -= (double)((rb2[0].x + rb2[1].x) + (rb2[0].y + rb2[1].y)) * X;
                             acc.x2 += (double)(sx2.x + sx2.y) * R * R;
                         }
                         int xz = 0;
-                        if (mabs == 0.0f)                  // rare: count exact zeros
+                        if (mn[k] == 0.0f)                 // rare: count exact zeros
 #pragma unroll
                             for (int j = 0; j < L / 2; ++j)
                                 xz += ((wb[j] & 0x7fffu) == 0u) + ((wb[j] & 0x7fff0000u) == 0u);

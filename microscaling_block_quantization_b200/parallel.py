@@ -23,6 +23,11 @@ are properties of the whole tensor, and each costs one small exchange:
 Bands follow the block geometry along rows so that no block straddles ranks:
 column blocks of B rows, 2D blocks of 32 rows, 128 rows for the tcgen05 scale
 layout and for column-axis macro blocks.
+
+QSNR(AB) of a product split by the rows of A (Sec.3 Eq. (2) of the first
+page): each rank holds a band of A's rows (bf16 and quantized) and the whole
+B (bf16 and quantized); both sums of Eq. (2) add over the bands, so one sum
+reduction of two numbers gives the whole product's QSNR.
 """
 from __future__ import annotations
 
@@ -32,8 +37,8 @@ import math
 import torch
 import torch.distributed as dist
 
-from . import (AXIS_2D, AXIS_COL, TS_AMAX, TS_COMPUTE, Config, Quantized, new_workspace, quantize,
-               stats_finalize, tensor_amax)
+from . import (AXIS_2D, AXIS_COL, TS_AMAX, TS_COMPUTE, Config, Quantized, gemm_qsnr, gemm_qsnr_finalize,
+               new_workspace, quantize, stats_finalize, tensor_amax)
 
 # entries of a stats buffer that add over bands: the five sums and the count
 SUM_ENTRIES = (0, 1, 2, 3, 4, 10)
@@ -105,3 +110,25 @@ def quantize_sharded(x_band: torch.Tensor, cfg: Config, *, stats: bool = True, g
         reduce_stats(q.stats, group)
         stats_finalize(q.stats, stream=stream)
     return q
+
+
+def reduce_qsnr_sums(stats: torch.Tensor, group=None) -> None:
+    """Sum of the ranks' [sum C_ref^2, sum (C_ref - C_q)^2], in place (the dB
+    entry is left for ``gemm_qsnr_finalize``)."""
+    dist.all_reduce(stats[:2], op=dist.ReduceOp.SUM, group=group)
+
+
+def gemm_qsnr_sharded(A_band: torch.Tensor, B: torch.Tensor, qa_band: Quantized, qb: Quantized, *,
+                      group=None, stream=None) -> torch.Tensor:
+    """QSNR(AB) of a product whose A is split by rows over the ranks: this
+    rank's band of A (bf16 rows and their quantized form, rows in units of
+    128) against the replicated B; returns the whole product's float64[3]
+    [sum C_ref^2, sum (C_ref - C_q)^2, dB].  An empty band contributes zeros.
+    Every rank of `group` must call it (one collective)."""
+    if A_band.shape[0] == 0:
+        st = torch.zeros(3, dtype=torch.float64, device=B.device)
+    else:
+        st = gemm_qsnr(A_band, B, qa_band, qb, stream=stream)
+    reduce_qsnr_sums(st, group)
+    gemm_qsnr_finalize(st, stream=stream)
+    return st

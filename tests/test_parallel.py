@@ -132,3 +132,54 @@ def test_rank_bands_equal_the_whole_tensor(case, world):
             assert st[i] == pytest.approx(want_stats[i], rel=1e-12, abs=1e-300)
         for i in (3, 4, 9, 10):
             assert st[i] == want_stats[i]
+
+
+def _qsnr_rank(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        M, N, K = 384, 128, 256
+        a = inputs.laplace_outlier_cols(M, K, seed=6, n_outlier_cols=2)
+        w = inputs.normal(N, K, sigma=0.02, seed=7)
+        r0, r1 = parallel.row_band(M, world, rank, parallel.row_align(mx.Config(sf_layout=1)))
+        st = np.zeros(3)
+        if r1 > r0:
+            oc = orc.Cfg()
+            ra, rw = orc.quantize(oc, a[r0:r1]), orc.quantize(oc, w)
+            ah = orc.dequantize(oc, ra["packed"], ra["scales"], None, None, None, r1 - r0, K)
+            wh = orc.dequantize(oc, rw["packed"], rw["scales"], None, None, None, N, K)
+            st = orc.gemm_qsnr(orc.input_f32(a[r0:r1]), orc.input_f32(w), ah, wh)
+        t = torch.from_numpy(np.asarray(st, np.float64).copy())
+        parallel.reduce_qsnr_sums(t)
+        out.put((rank, t.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_qsnr_ab_row_bands_add_up(world):
+    """QSNR(AB) with A split by rows (bands of 128: with four ranks over 384
+    rows one band is empty): the two sums of Eq. (2) reduced over the ranks
+    are the whole product's."""
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_qsnr_rank, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [out.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    M, N, K = 384, 128, 256
+    a = inputs.laplace_outlier_cols(M, K, seed=6, n_outlier_cols=2)
+    w = inputs.normal(N, K, sigma=0.02, seed=7)
+    oc = orc.Cfg()
+    ra, rw = orc.quantize(oc, a), orc.quantize(oc, w)
+    ah = orc.dequantize(oc, ra["packed"], ra["scales"], None, None, None, M, K)
+    wh = orc.dequantize(oc, rw["packed"], rw["scales"], None, None, None, N, K)
+    whole = orc.gemm_qsnr(orc.input_f32(a), orc.input_f32(w), ah, wh)
+    for _, st in res:
+        assert st[0] == pytest.approx(whole[0], rel=1e-12)
+        assert st[1] == pytest.approx(whole[1], rel=1e-12)
