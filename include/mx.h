@@ -380,11 +380,28 @@ int mx_mbs_gemm_scales(const mx_config *cfg, const uint8_t *scales, const uint8_
                        int64_t rows, int64_t cols, uint8_t *sf16, float *tensor_scale,
                        void *workspace, int64_t workspace_bytes, void *stream);
 
+/*
+ * mx_tensor_peak -- tensor-core ceiling probe for the roofline of mx_gemm (the
+ * pages have no counterpart; it measures the device, not the method).  One
+ * CTA per SM issues `iters` stages of four 128 x 256 x K block-scaled MMAs of
+ * a kind -- 1: kind::mxf4 (K = 64), 2: kind::mxf4nvf4 (K = 64), 3:
+ * kind::mxf8f6f4 (K = 32) -- on operands held in shared memory (zero codes,
+ * unit scales), with no global memory traffic; sf_copies 1 adds the
+ * per-stage scale copies into tensor memory that mx_gemm's stages make (into
+ * one slot of columns), 2 the same copies rotating over four slots as
+ * mx_gemm's stages do.
+ * *flops (host) receives the launch's flop count: time the launch on
+ * `stream` (CUDA events) for the throughput.  1 <= iters <= 2^22.
+ * Asynchronous like the other calls.
+ */
+int mx_tensor_peak(int32_t kind, int64_t iters, int32_t sf_copies, double *flops, void *stream);
+
 /* Status words of the bounded in-kernel waits: reads and clears them
  * (synchronises `stream`).  *status = 0 when no wait gave up, else the code of
  * the first wait that did: 1-3 and 11-14 the GEMM pipelines (128 x 128 and
- * persistent 128 x 256 tiles), 21-22 the E2M1 nearest-even quantizer's TMA
- * ring, 31-32 the other element types' ring.  A
+ * persistent 128 x 256 tiles), 15-19 the fused QSNR(AB) kernel, 20 the
+ * tensor-core probe, 21-22 the E2M1 nearest-even quantizer's TMA ring, 31-32
+ * the other element types' ring.  A
  * kernel whose wait gave up has left its loop early, so its outputs are
  * incomplete; the library has no counterpart on the pages. */
 int mx_device_status(void *stream, int32_t *status);

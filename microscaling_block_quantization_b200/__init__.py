@@ -116,12 +116,13 @@ def lib() -> C.CDLL:
         L.mx_tensor_amax.argtypes = [cfgp, P, i32, i64, i64, P, i64, P]
         L.mx_stats_finalize.argtypes = [P, P]
         L.mx_gemm_qsnr_finalize.argtypes = [P, P]
+        L.mx_tensor_peak.argtypes = [i32, i64, i32, C.POINTER(C.c_double), P]
         L.mx_strerror.argtypes = [C.c_int]
         L.mx_strerror.restype = C.c_char_p
         L.mx_version.restype = C.c_char_p
         for f in ("mx_query_sizes", "mx_quantize", "mx_quantize_noalloc", "mx_hadamard_quantize", "mx_dequantize",
                   "mx_qsnr", "mx_gemm", "mx_gemm_qsnr", "mx_mbs_gemm_scales", "mx_device_status",
-                  "mx_tensor_amax", "mx_stats_finalize", "mx_gemm_qsnr_finalize"):
+                  "mx_tensor_amax", "mx_stats_finalize", "mx_gemm_qsnr_finalize", "mx_tensor_peak"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -351,6 +352,15 @@ def stats_finalize(stats: torch.Tensor, stream=None) -> torch.Tensor:
     its sums and count, in place (``mx_stats_finalize``)."""
     _check("mx_stats_finalize", mx_stats_finalize(_p(stats), _stream(stream)))
     return stats
+
+
+def tensor_peak(kind: int, iters: int, sf_copies: int = 0, stream=None) -> float:
+    """Launch the tensor-core ceiling probe (``mx_tensor_peak``; kind 1
+    kind::mxf4, 2 kind::mxf4nvf4, 3 kind::mxf8f6f4) on ``stream`` and return
+    the launch's flop count; the caller times the launch."""
+    f = C.c_double(0.0)
+    _check("mx_tensor_peak", lib().mx_tensor_peak(kind, iters, int(sf_copies), C.byref(f), _stream(stream)))
+    return f.value
 
 
 def gemm_qsnr_finalize(stats: torch.Tensor, stream=None) -> torch.Tensor:

@@ -826,6 +826,111 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core ceiling probe: every CTA (one per SM) issues `iters` stages of
+// four 128 x 256 x K MMAs of a kind on operands resident in its shared memory
+// (all-zero codes, unit scales), accumulating into tensor memory, with no
+// global traffic; with `sf_copies` each stage first copies its scale chunks
+// into tensor memory as the GEMM's stages do.  The launch time over the
+// flops gives the kind's tensor throughput on this device.  Waits bounded.
+template <int KIND>
+__global__ void __launch_bounds__(128, 1) k_tc_peak(int64_t iters, int sf_copies)
+{
+    using KT = KindP<KIND>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *sA = smem, *sB = sA + KT::kABytes, *sSFA = sB + KT::kBBytes, *sSFB = sSFA + KT::kSfaBytes;
+    uint64_t *done = reinterpret_cast<uint64_t *>(sSFB + KT::kSfbBytes);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(done + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // zero codes; unit scales (E8M0 127, UE4M3 0x38)
+    const uint32_t one = KIND == KIND_NVF4 ? 0x38383838u : 0x7f7f7f7fu;
+    for (int i = threadIdx.x; i < (KT::kABytes + KT::kBBytes) / 4; i += blockDim.x)
+        reinterpret_cast<uint32_t *>(sA)[i] = 0u;
+    for (int i = threadIdx.x; i < (KT::kSfaBytes + KT::kSfbBytes) / 4; i += blockDim.x)
+        reinterpret_cast<uint32_t *>(sSFA)[i] = one;
+    if (threadIdx.x == 0) {
+        mbar_init(done, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(saddr(tmem_holder)), "r"(kTmemColsP));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_holder, tsf = tbase + BNP;
+    if (warp == 0 && lane == 0) {
+        const uint32_t idesc0 = idesc_p<KIND>((3u << 7) | (3u << 10));
+        const uint32_t a0 = saddr(sA), b0 = saddr(sB);
+        for (int64_t it = 0; it < iters; ++it) {
+            // sf_copies 2: the copies rotate over four slots of scale columns,
+            // as the GEMM's stages do; 1: one slot
+            const uint32_t sfa_t = tsf + (sf_copies == 2 ? (uint32_t)(it & 3) * KT::kSfCols : 0u);
+            if (sf_copies || it == 0) {
+#pragma unroll
+                for (int c = 0; c < KT::kChunks; ++c) {
+                    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                                 ::"r"(sfa_t + 4 * c), "l"(desc_sf(saddr(sSFA + c * 512))));
+                    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                                 ::"r"(sfa_t + KT::kChunks * 4 + 8 * c), "l"(desc_sf(saddr(sSFB + c * 512))));
+                    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                                 ::"r"(sfa_t + KT::kChunks * 4 + 8 * c + 4),
+                                   "l"(desc_sf(saddr(sSFB + KT::kChunks * 512 + c * 512))));
+                }
+            }
+            const uint32_t sfb_t = sfa_t + KT::kChunks * 4;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                uint32_t idesc = idesc0, sfa, sfb;
+                if constexpr (KIND == KIND_MXF4) {
+                    const uint32_t id = (k & 1) * 2;
+                    idesc |= (id << 29) | (id << 4);
+                    sfa = sfa_t + 4 * (k >> 1);
+                    sfb = sfb_t + 8 * (k >> 1);
+                } else if constexpr (KIND == KIND_MXF6) {
+                    const uint32_t id = (uint32_t)k;
+                    idesc |= (id << 29) | (id << 4);
+                    sfa = sfa_t;
+                    sfb = sfb_t;
+                } else {
+                    sfa = sfa_t + 4 * k;
+                    sfb = sfb_t + 8 * k;
+                }
+                mma<KIND>(tbase, desc_sw128(a0 + 32 * k), desc_sw128(b0 + 32 * k), idesc, sfa, sfb,
+                          (it > 0 || k > 0) ? 1u : 0u);
+            }
+        }
+        tc_commit(done);
+        mbar_wait(done, 0, 20);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(kTmemColsP));
+    }
+}
+
+template <int KIND>
+int launch_tc_peak(int64_t iters, int sf_copies, cudaStream_t st)
+{
+    using KT = KindP<KIND>;
+    const int smem = 1024 + KT::kABytes + KT::kBBytes + KT::kSfaBytes + KT::kSfbBytes + 64;
+    auto k = k_tc_peak<KIND>;
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return MX_ERR_CUDA;
+        attr = true;
+    }
+    k<<<mxk::device_sm_count(), 128, smem, st>>>(iters, sf_copies);
+    return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+}
+
 // Sum the per-CTA records in a fixed order: [sum C_ref^2, sum err^2, QSNR dB].
 __global__ void k_gemm_qsnr_finalize(const double *partials, int n, double *out)
 {
@@ -1162,6 +1267,23 @@ int mx_gemm_qsnr_finalize(double *stats, void *stream)
     // one record: the buffer's own two sums, read before the three entries are written
     k_gemm_qsnr_finalize<<<1, 256, 0, static_cast<cudaStream_t>(stream)>>>(stats, 1, stats);
     return cudaGetLastError() == cudaSuccess ? MX_OK : MX_ERR_CUDA;
+}
+
+int mx_tensor_peak(int32_t kind, int64_t iters, int32_t sf_copies, double *flops, void *stream)
+{
+    // at most 2^22 stages: well under a second at any clock (the bounded
+    // waits give up after two)
+    if (iters <= 0 || iters > (INT64_C(1) << 22) || !flops || (kind < KIND_MXF4 || kind > KIND_MXF6))
+        return MX_ERR_INVALID;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // flops of the launch: CTAs x stages x four MMAs of 128 x 256 x K
+    const double k_mma = kind == KIND_MXF6 ? 32.0 : 64.0;
+    *flops = (double)mxk::device_sm_count() * (double)iters * 4.0 * 2.0 * BM * BNP * k_mma;
+    switch (kind) {
+    case KIND_MXF4: return launch_tc_peak<KIND_MXF4>(iters, sf_copies, st);
+    case KIND_NVF4: return launch_tc_peak<KIND_NVF4>(iters, sf_copies, st);
+    default: return launch_tc_peak<KIND_MXF6>(iters, sf_copies, st);
+    }
 }
 
 int mx_device_status(void *stream, int32_t *status)
