@@ -53,8 +53,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-case", default=None,
                     help="run one kernel alone (for ncu captures): quant_mxfp4_row, quant_nvfp4_row, "
-                         "quant_mxfp4_col, quant_mxfp4_2d, quant_had32_row, dequant_mxfp4_row, "
-                         "gemm_mxfp4, gemm_nvfp4")
+                         "quant_mxfp4_col, quant_mxfp4_2d, quant_had32_row, quant_mbs_oas_row, "
+                         "dequant_mxfp4_row, gemm_mxfp4, gemm_nvfp4, gemm_qsnr_mxfp4, gemm_qsnr_nvfp4")
     ap.add_argument("--rows", type=int, default=16384)
     ap.add_argument("--cols", type=int, default=8192)
     ap.add_argument("--reps", type=int, default=3)
@@ -419,7 +419,7 @@ def run_c2_sweep(mx, device, args):
     from microscaling_block_quantization_b200 import inputs
     sigmas = (0.002, 0.02, 0.2)
     xs = [inputs.normal(4096, 4096, sigma=sg, seed=i + 1).to(device) for i, sg in enumerate(sigmas)]
-    evict = torch.ones(256 << 20, dtype=torch.uint8, device=device)
+    evict = torch.ones(64 << 20, dtype=torch.float32, device=device)    # 256 MiB, read to evict L2
     stream = torch.cuda.current_stream(device)
     out = {}
     for fmt, fname in ((mx.SCALE_UE4M3, "UE4M3"), (mx.SCALE_UE5M3, "UE5M3")):
@@ -806,6 +806,8 @@ def kernel_case(args):
     res = {"case": case, "stats": not args.no_stats}
     if case.startswith("gemm"):
         M, N, K = M_TOK, N_OUT, K_DIM
+        qsnr = case.startswith("gemm_qsnr")
+        case = case.replace("gemm_qsnr", "gemm")
         cfg = {"gemm_mxfp4": mx.Config(sf_layout=1),
                "gemm_nvfp4": mx.Config(block=16, scale_fmt=1, rule=3, tensor_scale=1, sf_layout=1),
                "gemm_mxfp6": mx.Config(elem=mx.E2M3, sf_layout=1),
@@ -815,8 +817,14 @@ def kernel_case(args):
         w = (torch.randn(N, K, generator=g, device=dev) * 0.02).to(torch.bfloat16)
         qa, qw = mx.quantize(a, cfg, stats=False), mx.quantize(w, cfg_w, stats=False)
         c = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        run = lambda: mx.gemm(qa, qw, out=c)
-        work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
+        if qsnr:
+            # QSNR(AB): the block-scaled and the bf16 product, C not written
+            a16, w16 = a.to(torch.bfloat16), w.to(torch.bfloat16)
+            run = lambda: mx.gemm_qsnr(a16, w16, qa, qw)
+            work, unit = 4.0 * M * N * K / 1e12, "TFLOP/s (both products)"
+        else:
+            run = lambda: mx.gemm(qa, qw, out=c)
+            work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
     else:
         R, Cc = args.rows, args.cols
         x = torch.randn(R, Cc, generator=g, device=dev)
