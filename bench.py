@@ -920,7 +920,8 @@ def main():
                    "streams": "one" if args.one_stream else
                               "two: MXFP4 / rotated / MBS quantizers on one stream, NVFP4 (tensor-amax pass + "
                               "quantizer) and the dequantizers (after their codes) on a second, each with its "
-                              "own workspace; per-row figures are sequential single-launch replays"},
+                              "own workspace; per-variant figures come from one-stream graphs of back-to-back "
+                              "A/W launch pairs"},
         "roofline": r["roofline"],
         "cpu_baseline": cpu,
         "e2e": r["e2e"],
