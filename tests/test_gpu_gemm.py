@@ -102,8 +102,21 @@ def test_gemm_tiles_and_stage_ring(mx, orc, name, shape):
 
 
 @pytest.mark.parametrize("name", ["mxfp4", "nvfp4"])
-def test_gemm_bf16_output(mx, orc, name):
-    check_gemm(mx, orc, name, 256, 256, 512, out_dtype=torch.bfloat16)
+@pytest.mark.parametrize("shape", [(256, 256, 512), (384, 768, 512), (1280, 4096, 256)])
+def test_gemm_bf16_output(mx, orc, name, shape):
+    """bf16 C written by the epilogue's tensor stores (128 x 256 tiles; more
+    tiles than CTAs in the last shape): against the oracle, and bit for bit
+    the round-to-nearest-even of the binary32 C."""
+    check_gemm(mx, orc, name, *shape, out_dtype=torch.bfloat16)
+    M, N, K = shape
+    a = inputs.laplace_outlier_cols(M, K, seed=6, n_outlier_cols=2).cuda()
+    w = inputs.normal(N, K, sigma=0.02, seed=7).cuda()
+    cfg = configs(mx)[name]
+    qa, qw = mx.quantize(a, cfg, stats=False), mx.quantize(w, cfg, stats=False)
+    c16 = mx.gemm(qa, qw, out_dtype=torch.bfloat16)
+    c32 = mx.gemm(qa, qw, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(c16.view(torch.int16), c32.to(torch.bfloat16).view(torch.int16))
 
 
 def test_gemm_rejects_canonical_scales(mx):
