@@ -309,6 +309,24 @@ __device__ __forceinline__ uint32_t macro_code(const ElemDesc &ed, float amax, i
     return e4m3_encode_pos(__fdiv_rn(m, __fdiv_rn(ed.maxv, (float)(1 << ed.emax))));
 }
 
+// Same code as macro_code() without an IEEE division per call: d = max_elem /
+// 2^emax (exact) and r_d = RN(1/d) are the launch's; m / d goes through
+// div_by_recip (correctly rounded).  m is in [1, 2) and d in [1, 2), so the
+// quotient lies in (1/2, 2), inside E4M3's normal range, where the hardware
+// conversion rounds to nearest-even like e4m3_encode_pos().
+__device__ __forceinline__ uint32_t macro_code_recip(float d, float r_d, float amax, int bad)
+{
+    if (bad) return 0x7fu;
+    if (amax == 0.0f) return 0x38u;                 // E4M3 1.0
+    int e;
+    float m;
+    frexp_exact(amax, e, m);
+    const float x = div_by_recip(m, d, r_d);
+    uint16_t h;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(0.0f), "f"(x));
+    return h & 0xffu;
+}
+
 // ------------------------------------------------------------ rotation -----
 // Butterfly stages of the Sylvester-ordered fast Walsh-Hadamard transform on
 // a row chunk of 8 elements held by consecutive lanes (stride 8 and 16 are

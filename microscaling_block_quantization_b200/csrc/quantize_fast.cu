@@ -213,6 +213,15 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
             near_tab[c] = c < p.sd.ue_nan_code ? make_float2(d, __fdiv_rn(1.0f, d))
                                                : make_float2(__uint_as_float(0x7fc00000u), 0.0f);
         }
+    // macro scales: {S_M, RN(1 / S_M)} for every E4M3 code, once per CTA
+    __shared__ float2 macro_tab[MBS ? 128 : 1];
+    if constexpr (MBS)
+        for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+            const float v = e4m3_value((uint32_t)c);
+            macro_tab[c] = make_float2(v, __fdiv_rn(1.0f, v));
+        }
+    const float md = MBS ? __fmul_rn(p.ed.maxv, exp2i(-p.ed.emax)) : 1.0f;   // max_elem / 2^emax, exact
+    const float r_md = MBS ? __fdiv_rn(1.0f, md) : 1.0f;
     __syncthreads();
     NearScale ns;
     ns.maxv = p.ed.maxv;
@@ -266,9 +275,10 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
                 int mbad = !(m <= FLT_MAX);
                 float mm = grp_max(mbad ? 0.0f : m, 4);
                 mbad = grp_or(mbad, 4);
-                const uint32_t mcode = macro_code(p.ed, mm, mbad);
-                sm = e4m3_value(mcode);
-                const float invm = __fdiv_rn(1.0f, sm);
+                const uint32_t mcode = macro_code_recip(md, r_md, mm, mbad);
+                const float2 mt = macro_tab[mcode];
+                sm = mt.x;
+                const float invm = mt.y;
                 if ((t & 3) == 0 && tile * kConsumers + t < nch) p.macro[(tile * kConsumers + t) >> 2] = (uint8_t)mcode;
                 const float2 invm2 = make_float2(invm, invm);
 #pragma unroll
@@ -313,9 +323,10 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
                     }
                     const float mm = grp_max(mbad ? 0.0f : m, 4);
                     mbad = grp_or(mbad, 4);
-                    const uint32_t mcode = macro_code(p.ed, mm, mbad);
-                    sm = e4m3_value(mcode);
-                    invm = __fdiv_rn(1.0f, sm);
+                    const uint32_t mcode = macro_code_recip(md, r_md, mm, mbad);
+                    const float2 mt = macro_tab[mcode];
+                    sm = mt.x;
+                    invm = mt.y;
                     if ((t & 3) == 0 && ok) p.macro[c >> 2] = (uint8_t)mcode;
 #pragma unroll
                     for (int k = 0; k < NB; ++k) {
