@@ -184,25 +184,28 @@ __device__ __forceinline__ double warp_sum(double v)
     return v;
 }
 
-// CTA reduction in a fixed order; thread 0 writes the CTA's record.
+// CTA reduction in a fixed order (lanes, then the warps' sums as one more
+// warp reduction); thread 0 writes the CTA's record.
 static __device__ __forceinline__ void write_partials(double *partials, const Acc &a)
 {
-    __shared__ double sh[32][5];
+    __shared__ double sh[5][32];
     double v[5] = {a.x2, a.e2, a.e, a.ftz, a.nz};
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
 #pragma unroll
     for (int i = 0; i < 5; ++i) v[i] = warp_sum(v[i]);
     if (lane == 0)
 #pragma unroll
-        for (int i = 0; i < 5; ++i) sh[w][i] = v[i];
+        for (int i = 0; i < 5; ++i) sh[i][w] = v[i];
     __syncthreads();
-    if (threadIdx.x == 0) {
-        double s[5] = {0, 0, 0, 0, 0};
-        for (int k = 0; k < (int)(blockDim.x >> 5); ++k)
-            for (int i = 0; i < 5; ++i) s[i] += sh[k][i];
+    if (w == 0) {
+        const int nw = (int)(blockDim.x >> 5);
         double *o = partials + (int64_t)blockIdx.x * kPartialDoubles;
-        for (int i = 0; i < 5; ++i) o[i] = s[i];
-        o[5] = o[6] = o[7] = 0.0;
+#pragma unroll
+        for (int i = 0; i < 5; ++i) {
+            const double t = warp_sum(lane < nw ? sh[i][lane] : 0.0);
+            if (lane == 0) o[i] = t;
+        }
+        if (lane == 0) o[5] = o[6] = o[7] = 0.0;
     }
 }
 
@@ -248,35 +251,47 @@ __device__ __forceinline__ void finish_launch(const QParams &p, const Acc &a)
 {
     if (p.partials) write_partials(p.partials, a);
     if (!p.ticket) return;
+    // thread 0 wrote the record; its release-acquire ticket orders the record
+    // before the last CTA's reads of it (the barrier below extends that
+    // order to the other threads of the last CTA)
     __shared__ unsigned s_last;
     if (threadIdx.x == 0) {
-        __threadfence();
-        s_last = atomicAdd(p.ticket, 1u) == gridDim.x - 1;
+        unsigned prev;
+        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(prev) : "l"(p.ticket) : "memory");
+        s_last = prev == gridDim.x - 1;
     }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
     if (p.partials) {
-        // every thread of the last CTA takes a strided share of the records,
-        // then warps, then the CTA (a fixed order for a given launch shape)
-        __shared__ double red[32][5];
+        // every thread of the last CTA takes a strided share of the records
+        // (two in flight), then warps, then the warps' sums (a fixed order
+        // for a given launch shape)
+        __shared__ double red[5][32];
         double s[5] = {0, 0, 0, 0, 0};
-        for (unsigned i = threadIdx.x; i < gridDim.x; i += blockDim.x)
+        for (unsigned i0 = threadIdx.x; i0 < gridDim.x; i0 += 2 * blockDim.x) {
+            const unsigned i1 = i0 + blockDim.x;
+            double r0[5], r1[5];
 #pragma unroll
-            for (int k = 0; k < 5; ++k) s[k] += __ldcg(p.partials + (size_t)i * kPartialDoubles + k);
+            for (int k = 0; k < 5; ++k) r0[k] = __ldcg(p.partials + (size_t)i0 * kPartialDoubles + k);
+#pragma unroll
+            for (int k = 0; k < 5; ++k)
+                r1[k] = i1 < gridDim.x ? __ldcg(p.partials + (size_t)i1 * kPartialDoubles + k) : 0.0;
+#pragma unroll
+            for (int k = 0; k < 5; ++k) s[k] += r0[k] + r1[k];
+        }
 #pragma unroll
         for (int k = 0; k < 5; ++k) s[k] = warp_sum(s[k]);
-        const int w = threadIdx.x >> 5;
-        if ((threadIdx.x & 31) == 0)
+        const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        if (lane == 0)
 #pragma unroll
-            for (int k = 0; k < 5; ++k) red[w][k] = s[k];
+            for (int k = 0; k < 5; ++k) red[k][w] = s[k];
         __syncthreads();
-        if (threadIdx.x == 0) {
-            double t[5] = {0, 0, 0, 0, 0};
-            for (int v = 0; v < (int)(blockDim.x >> 5); ++v)
+        if (w == 0) {
+            const int nw = (int)(blockDim.x >> 5);
+            double t[5];
 #pragma unroll
-                for (int k = 0; k < 5; ++k) t[k] += red[v][k];
-            store_stats(p.stats, t, p.count);
+            for (int k = 0; k < 5; ++k) t[k] = warp_sum(lane < nw ? red[k][lane] : 0.0);
+            if (lane == 0) store_stats(p.stats, t, p.count);
         }
     }
     if (threadIdx.x == 0) {

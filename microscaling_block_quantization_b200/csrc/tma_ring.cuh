@@ -83,16 +83,20 @@ struct Ring {
     __device__ __forceinline__ void produce(const CUtensorMap *tm, uint32_t ntiles, int where) const
     {
         constexpr uint32_t S = RingCfg<InT>::kStages;
+        // the quantizer reads each input line once: mark it first to evict,
+        // so that it does not displace lines other launches still need
+        uint64_t pol;
+        asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
         uint32_t i = 0;
         for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
             const uint32_t s = i % S;
             if (i >= S && !ring_wait(&empty[s], ((i / S) - 1) & 1, where)) break;
             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
                          ::"r"(ring_saddr(&full[s])), "r"(RingCfg<InT>::kTileBytes) : "memory");
-            asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-                         " [%0], [%1, {%3, %4}], [%2];"
+            asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+                         " [%0], [%1, {%3, %4}], [%2], %5;"
                          ::"r"(ring_saddr(stage(s))), "l"((uint64_t)tm), "r"(ring_saddr(&full[s])),
-                           "r"(0), "r"((int)(tile * kRingConsumers))
+                           "r"(0), "r"((int)(tile * kRingConsumers)), "l"(pol)
                          : "memory");
         }
     }
