@@ -35,7 +35,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 M_TOK, K_DIM, N_OUT = 8192, 4096, 14336
-R_PAIRS = 8          # A/W launch pairs per per-variant timing graph
+R_PAIRS = 8          # repeats of a variant's A+W call per per-variant timing graph
 WORKLOAD = ("Llama-3-8B-shaped linear layer: A 8192x4096 bf16 Laplace(0,1) seed 6, "
             "W 14336x4096 bf16 N(0,0.02) seed 7 (W stored out x in, product A W^T)")
 METRIC = "MX quantize+pack GB/s (% of ~8 TB/s HBM); block-scaled FP4 GEMM TFLOPS"
@@ -87,6 +87,23 @@ def step_plan(mx):
     ]
 
 
+def step_calls(plan):
+    """The step's calls: each quantizer variant as one grouped call over its
+    tensors (A and W share the launch), each dequantizer one call per tensor.
+    (name, tensors, config, kind), in plan order."""
+    calls, seen = [], {}
+    for name, t, cfg, kind in plan:
+        if kind == "q":
+            if name in seen:
+                seen[name][1].append(t)
+                continue
+            seen[name] = (name, [t], cfg, kind)
+            calls.append(seen[name])
+        else:
+            calls.append((name, [t], cfg, kind))
+    return [(n, tuple(ts), c, k) for n, ts, c, k in calls]
+
+
 def algo_bytes(cfg, rows, cols, kind, in_bytes=2):
     n = rows * cols
     code = n if cfg.elem in (2, 3) else n // 2
@@ -98,12 +115,13 @@ def algo_bytes(cfg, rows, cols, kind, in_bytes=2):
     return code + nb + macro + offs + 2 * n       # dequantize to bf16
 
 
-def launches_per_call(cfg, kind):
+def launches_per_call(cfg, kind, ntensors=1):
     if kind == "d":
-        return 1
-    k = 1                                  # quantize (its last CTA sums the statistics)
+        return ntensors                    # one dequantizer launch per tensor
+    groups = (ntensors + 3) // 4           # a grouped launch takes up to 4 tensors
+    k = groups                             # quantize (the last CTA of each tensor sums its statistics)
     if cfg.tensor_scale == 1:
-        k += 1                             # tensor-amax pre-pass
+        k += groups                        # tensor-amax pre-pass
     return k
 
 
@@ -207,17 +225,19 @@ def run_ours(args, rank, world, device):
             outs[key] = torch.empty(x.shape, dtype=torch.bfloat16, device=device)
             outs[(key, "src")] = src
 
-    # each stream owns a workspace: concurrent calls must not share control words
-    ws_main = mx.new_workspace(mx.MXFP4, *A.shape, device)
-    ws_side = mx.new_workspace(mx.MXFP4, *A.shape, device)
+    calls = step_calls(plan)
+    # each stream owns a workspace per tensor: concurrent calls, and the
+    # tensors of one grouped call, must not share control words
+    wss = {(sd, t): mx.new_workspace(mx.MXFP4, *A.shape, device) for sd in ("main", "side") for t in T}
 
-    def run_call(name, t, cfg, kind, stream=None, ws=None):
+    def run_call(name, ts, cfg, kind, stream=None, wsk="main"):
         # stream=None: the current stream, i.e. the capture stream inside a graph
-        key = (name, t)
         if kind == "q":
-            mx.quantize(T[t], cfg, out=outs[key], stream=stream, workspace=ws_main if ws is None else ws)
+            mx.quantize_group([T[t] for t in ts], cfg, outs=[outs[(name, t)] for t in ts], stream=stream,
+                              workspaces=[wss[(wsk, t)] for t in ts])
         else:
-            mx.dequantize(outs[(key, "src")], out=outs[key], stream=stream)
+            for t in ts:
+                mx.dequantize(outs[((name, t), "src")], out=outs[(name, t)], stream=stream)
 
     # The step's launches are independent problems except that each
     # dequantizer reads the MXFP4 codes of its tensor.  They are captured on
@@ -231,33 +251,32 @@ def run_ours(args, rank, world, device):
 
     def run_step():
         if args.one_stream:
-            for call in plan:
+            for call in calls:
                 run_call(*call)
             return
         main = torch.cuda.current_stream(device)
         fork = torch.cuda.Event()
         fork.record(main)
         side.wait_event(fork)
-        codes_ready = {}
-        for call in plan:
-            name, t, cfg, kind = call
+        codes_ready = None
+        for call in calls:
+            name, ts, cfg, kind = call
             if name in SIDE:
                 if kind == "d":
-                    side.wait_event(codes_ready[t])
+                    side.wait_event(codes_ready)
                 with torch.cuda.stream(side):
-                    run_call(*call, stream=side, ws=ws_side)
+                    run_call(*call, stream=side, wsk="side")
             else:
                 run_call(*call)
                 if name == "mxfp4_row":
-                    ev = torch.cuda.Event()
-                    ev.record(main)
-                    codes_ready[t] = ev
+                    codes_ready = torch.cuda.Event()
+                    codes_ready.record(main)
         join = torch.cuda.Event()
         join.record(side)
         main.wait_event(join)
 
     step_bytes = sum(algo_bytes(cfg, *T[t].shape, kind) for _, t, cfg, kind in plan)
-    launches = sum(launches_per_call(cfg, kind) for _, _, cfg, kind in plan)
+    launches = sum(launches_per_call(cfg, kind, len(ts)) for _, ts, cfg, kind in calls)
 
     # eager warm-up (caches kernel attributes)
     for _ in range(max(1, args.warmup)):
@@ -266,10 +285,11 @@ def run_ours(args, rank, world, device):
 
     # the step captured as a CUDA graph: the kernels run back to back with no
     # host work between them.  Per variant, a graph of R_PAIRS back-to-back
-    # pairs of its launches on A and on W (one stream, the step's launch
-    # configuration): consecutive launches read different tensors, 176 MiB
-    # apart, so no input comes from L2, and the time over the pairs is the
-    # steady-state launch duration without graph-launch gaps
+    # repeats of its call on A and W (one stream, the step's launch
+    # configuration: one grouped quantizer launch over both tensors); the two
+    # tensors together (176 MiB) are larger than L2, so no input comes from
+    # L2, and the time over the repeats is the steady-state call duration
+    # without graph-launch gaps
     step_graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(step_graph):
         run_step()
@@ -279,7 +299,7 @@ def run_ours(args, rank, world, device):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for _ in range(R_PAIRS):
-                for call in plan:
+                for call in calls:
                     if call[0] == name:
                         run_call(*call)
         pair_graphs[name] = g
@@ -332,17 +352,18 @@ def run_ours(args, rank, world, device):
     del pair_graphs
 
     pk, pk_src = peaks()
-    # the dominant kernel of the step: k_quant_fast, all eight quantizer
-    # launches (NVFP4's per-call time includes its tensor-amax pre-pass)
+    # the dominant kernel of the step: k_quant_fast, the four grouped
+    # quantizer launches over A and W (NVFP4's per-call time includes its
+    # tensor-amax pre-pass)
     qnames = ["mxfp4_row", "nvfp4_row", "had32_mxfp4", "mbs_oas_mxfp4"]
     qbytes = sum(rows[n]["bytes"] for n in qnames)
     qus = sum(rows[n]["us"] for n in qnames)
     achieved = round(qbytes / (qus * 1e-6) / 1e9, 1)
     traffic = traffic_record("mxfp4_row_W")
     roofline = {"bound": "hbm",
-                "kernel": "k_quant_fast (TMA-fed E2M1 quantizer, statistics summed by its last CTA): the step's "
-                          "8 quantizer launches, MXFP4 / NVFP4 (with its tensor-amax pre-pass) / rotation-32 / "
-                          "MBS+OAS on A and W",
+                "kernel": "k_quant_fast (TMA-fed E2M1 quantizer, statistics summed by the last CTA of each "
+                          "tensor): the step's 4 grouped launches, MXFP4 / NVFP4 (with its tensor-amax "
+                          "pre-pass) / rotation-32 / MBS+OAS, each over A and W",
                 "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk_src,
                 "traffic": traffic,
@@ -359,7 +380,7 @@ def run_ours(args, rank, world, device):
         extra["c2_block_size_sweep"] = {"unavailable": f"{type(e).__name__}: {e}"}
 
     # end to end through the public API with host buffers
-    e2e = run_e2e(mx, A_cpu, W_cpu, plan, outs, device, args, step_bytes, world)
+    e2e = run_e2e(mx, A_cpu, W_cpu, plan, calls, wss, device, args, step_bytes, world)
 
     # fidelity of the step (sanity: the stats the kernels produced)
     fid = {f"{name}_{t}_qsnr_db": round(float(outs[(name, t)].stats[7].item()), 4)
@@ -464,63 +485,63 @@ def run_c2_sweep(mx, device, args):
     return out
 
 
-def run_e2e(mx, A_cpu, W_cpu, plan, outs, device, args, step_bytes, world):
+def run_e2e(mx, A_cpu, W_cpu, plan, calls, wss, device, args, step_bytes, world):
     """Same step through the public API, inputs copied from pinned host memory
     and the codes, scales and stats read back, inside the timed region.  The
-    copies run on their own streams: A's results go back to the host while W
-    comes in and is quantized (PCIe is full duplex), and the next step's
-    inputs come in while the previous step's results go out.  Events order
-    every reuse of a device buffer."""
+    copies run on their own streams, and the device inputs and outputs are
+    double-buffered: step i+1's inputs come in and its calls run while step
+    i's results go out (PCIe is full duplex).  Events order every reuse of a
+    device buffer."""
     compute = torch.cuda.current_stream(device)
     h2d, d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
-    hA = A_cpu.pin_memory()
-    hW = W_cpu.pin_memory()
-    dA = torch.empty_like(hA, device=device)
-    dW = torch.empty_like(hW, device=device)
-    T = {"A": dA, "W": dW}
-    back = {"A": [], "W": []}
-    for name, t, cfg, kind in plan:
-        if kind == "q":
-            o = outs[(name, t)]
-            for d in (o.codes, o.scales, o.stats):
-                back[t].append((d, torch.empty(d.shape, dtype=d.dtype).pin_memory()))
-    h2d_bytes = hA.numel() * 2 + hW.numel() * 2
-    d2h_bytes = sum(d.numel() * d.element_size() for t in back for d, _ in back[t])
-    host = {"A": hA, "W": hW}
-    # per tensor: inputs landed, launches done, results read back
-    ev = {(k, t): None for k in ("in", "done", "out") for t in ("A", "W")}
+    host = {"A": A_cpu.pin_memory(), "W": W_cpu.pin_memory()}
+    bufs = []
+    for _ in range(2):
+        T = {t: torch.empty_like(h, device=device) for t, h in host.items()}
+        o = {(name, t): mx.alloc_outputs(cfg, *T[t].shape, device, stats=True)
+             for name, t, cfg, kind in plan if kind == "q"}
+        back = [(d, torch.empty(d.shape, dtype=d.dtype).pin_memory())
+                for q in o.values() for d in (q.codes, q.scales, q.stats)]
+        deq = {(name, t): torch.empty(T[t].shape, dtype=torch.bfloat16, device=device)
+               for name, t, cfg, kind in plan if kind == "d"}
+        bufs.append({"T": T, "outs": o, "back": back, "deq": deq, "in": None, "done": None, "out": None})
+    h2d_bytes = sum(h.numel() * h.element_size() for h in host.values())
+    d2h_bytes = sum(d.numel() * d.element_size() for d, _ in bufs[0]["back"])
+    it = [0]
 
     def one():
-        for t in ("A", "W"):
-            if ev[("done", t)] is not None:
-                h2d.wait_event(ev[("done", t)])          # the previous step has read T[t]
-            with torch.cuda.stream(h2d):
-                T[t].copy_(host[t], non_blocking=True)
-            ev[("in", t)] = torch.cuda.Event()
-            ev[("in", t)].record(h2d)
-        for t in ("A", "W"):
-            compute.wait_event(ev[("in", t)])
-            if ev[("out", t)] is not None:
-                compute.wait_event(ev[("out", t)])       # the previous results are on the host
-            for name, tt, cfg, kind in plan:
-                if tt != t:
-                    continue
-                if kind == "q":
-                    mx.quantize(T[t], cfg, out=outs[(name, t)], stream=compute)
-                else:
-                    mx.dequantize(outs[("mxfp4_row", t)], out=outs[(name, t)], stream=compute)
-            ev[("done", t)] = torch.cuda.Event()
-            ev[("done", t)].record(compute)
-            d2h.wait_event(ev[("done", t)])
-            with torch.cuda.stream(d2h):
-                for d, h in back[t]:
-                    h.copy_(d, non_blocking=True)
-            ev[("out", t)] = torch.cuda.Event()
-            ev[("out", t)].record(d2h)
+        b = bufs[it[0] % 2]
+        it[0] += 1
+        if b["done"] is not None:
+            h2d.wait_event(b["done"])                    # this buffer's previous step has read its inputs
+        with torch.cuda.stream(h2d):
+            for t, h in host.items():
+                b["T"][t].copy_(h, non_blocking=True)
+        b["in"] = torch.cuda.Event()
+        b["in"].record(h2d)
+        compute.wait_event(b["in"])
+        if b["out"] is not None:
+            compute.wait_event(b["out"])                 # this buffer's previous results are on the host
+        for name, ts, cfg, kind in calls:
+            if kind == "q":
+                mx.quantize_group([b["T"][t] for t in ts], cfg, outs=[b["outs"][(name, t)] for t in ts],
+                                  stream=compute, workspaces=[wss[("main", t)] for t in ts])
+            else:
+                for t in ts:
+                    mx.dequantize(b["outs"][("mxfp4_row", t)], out=b["deq"][(name, t)], stream=compute)
+        b["done"] = torch.cuda.Event()
+        b["done"].record(compute)
+        d2h.wait_event(b["done"])
+        with torch.cuda.stream(d2h):
+            for d, h in b["back"]:
+                h.copy_(d, non_blocking=True)
+        b["out"] = torch.cuda.Event()
+        b["out"].record(d2h)
 
     def drain():
-        for t in ("A", "W"):
-            compute.wait_event(ev[("out", t)])
+        for b in bufs:
+            if b["out"] is not None:
+                compute.wait_event(b["out"])
 
     steps = max(3, args.steps // 4)
     for _ in range(2):
@@ -545,7 +566,8 @@ def run_e2e(mx, A_cpu, W_cpu, plan, outs, device, args, step_bytes, world):
     return {"value": round(world * step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes, "ms_per_step": round(ms, 3),
             "steps": steps,
-            "overlap": "copy-in, compute and copy-out on three streams (A's results out while W comes in)"}
+            "overlap": "copy-in, compute and copy-out on three streams with double-buffered device inputs and "
+                       "outputs (a step's results go out while the next step's inputs come in and its calls run)"}
 
 
 def tensor_ceilings(mx, device, iters=100000):
@@ -916,17 +938,18 @@ def main():
         "config": {"workload": WORKLOAD, "step": [f"{n}:{t}" for n, t, _, _ in step_plan(__import__("microscaling_block_quantization_b200"))],
                    "step_algorithmic_bytes": r["step_bytes"], "hbm_frac_of_8TBs": round(r["value"] / world / 8000, 4),
                    "quantize_only_GB_per_s": r["roofline"]["achieved"],
-                   "quantize_only_note": "the step's 8 quantizer launches (no dequantizer): their algorithmic bytes "
-                                         "over their summed launch durations, one stream",
-                   "per_launch_timing": f"per variant a graph of {R_PAIRS} back-to-back A/W launch pairs, "
-                                        "replayed K times (no graph-launch gap between launches)",
-                   "l2": "inputs larger than L2 (A+W 176 MiB > 126 MB); consecutive launches alternate tensors",
+                   "quantize_only_note": "the step's 4 grouped quantizer calls on A and W (no dequantizer): their "
+                                         "algorithmic bytes over their summed call durations, one stream",
+                   "per_launch_timing": f"per variant a graph of {R_PAIRS} back-to-back calls over A and W "
+                                        "(one grouped quantizer launch each), replayed K times (no graph-launch "
+                                        "gap between launches)",
+                   "l2": "inputs larger than L2 (A+W 176 MiB > 126 MB) read once per call",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "streams": "one" if args.one_stream else
                               "two: MXFP4 / rotated / MBS quantizers on one stream, NVFP4 (tensor-amax pass + "
                               "quantizer) and the dequantizers (after their codes) on a second, each with its "
-                              "own workspace; per-variant figures come from one-stream graphs of back-to-back "
-                              "A/W launch pairs"},
+                              "own workspaces; per-variant figures come from one-stream graphs of back-to-back "
+                              "A+W calls"},
         "roofline": r["roofline"],
         "cpu_baseline": cpu,
         "e2e": r["e2e"],

@@ -244,6 +244,41 @@ int mx_hadamard_quantize(const mx_config *cfg, const void *x, int32_t x_dtype, i
                          uint8_t *macro_scales, uint16_t *offsets, double *stats,
                          float *rotated, void *workspace, int64_t workspace_bytes, void *stream);
 
+/* One tensor of mx_quantize_group: mx_quantize's per-tensor arguments. */
+typedef struct {
+    const void *x;            /* device input, rows x cols, row-major */
+    int64_t rows, cols;
+    void *codes;              /* device out, as mx_quantize */
+    uint8_t *scales;          /* device out, as mx_quantize */
+    float *tensor_scale;      /* device, as mx_quantize (this tensor's own s_T) */
+    uint8_t *macro_scales;    /* device out or NULL, as mx_quantize */
+    uint16_t *offsets;        /* device out or NULL, as mx_quantize */
+    double *stats;            /* device out or NULL: this tensor's statistics */
+    void *workspace;          /* device scratch of this tensor, as mx_quantize */
+    int64_t workspace_bytes;
+} mx_quantize_item;
+
+/*
+ * mx_quantize_group -- mx_quantize of n tensors that share one configuration
+ * and input dtype (for instance the activation and the weight of a layer, or
+ * the weights of several layers), each with its own outputs, tensor scale and
+ * statistics: the results are those of n mx_quantize calls (mx_hadamard_quantize
+ * without `rotated` when cfg->hadamard), bit for bit ([MXFP4-OAS] Sec.2: every
+ * block, and every tensor, is quantized on its own).  Shapes may differ.
+ *   For row-axis E2M1 round-to-nearest-even symmetric configurations (not the
+ *   MSE rule; with a rotation or a macro scale, blocks of 16 or 32) the
+ *   tensors share one quantizer launch, up to 4 tensors a launch, the CTAs
+ *   split among the tensors in proportion to their sizes; with a computed
+ *   tensor scale one tensor-amax launch comes before it.  Other
+ *   configurations run as n calls in order.
+ *   Items that need a workspace (stats != NULL, MX_TS_COMPUTE, MX_TS_AMAX)
+ *   must each have their own (MX_ERR_INVALID when two overlap).  Every item is
+ *   checked before anything is queued; a failing item fails the call with
+ *   that item's error.  n >= 1.
+ */
+int mx_quantize_group(const mx_config *cfg, int32_t x_dtype, const mx_quantize_item *items, int32_t n,
+                      void *stream);
+
 /*
  * mx_tensor_amax -- the tensor-amax pre-pass alone, for a tensor split by rows
  * over several devices (one process per GPU): amax_T = max |x| (of the rotated

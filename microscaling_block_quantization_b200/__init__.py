@@ -48,6 +48,13 @@ class mx_config(C.Structure):
                 ("seed", C.c_uint64)]
 
 
+class mx_quantize_item(C.Structure):
+    _fields_ = [("x", C.c_void_p), ("rows", C.c_int64), ("cols", C.c_int64), ("codes", C.c_void_p),
+                ("scales", C.c_void_p), ("tensor_scale", C.c_void_p), ("macro_scales", C.c_void_p),
+                ("offsets", C.c_void_p), ("stats", C.c_void_p), ("workspace", C.c_void_p),
+                ("workspace_bytes", C.c_int64)]
+
+
 class mx_sizes(C.Structure):
     _fields_ = [("codes_bytes", C.c_int64), ("n_scales", C.c_int64), ("n_macro", C.c_int64),
                 ("n_offsets", C.c_int64), ("workspace_bytes", C.c_int64), ("n_blocks", C.c_int64)]
@@ -103,6 +110,7 @@ def lib() -> C.CDLL:
         L.mx_quantize.argtypes = [cfgp, P, i32, i64, i64, P, P, P, P, P, P, P, i64, P]
         L.mx_hadamard_quantize.argtypes = [cfgp, P, i32, i64, i64, P, P, P, P, P, P, P, P, i64, P]
         L.mx_quantize_noalloc.argtypes = [cfgp, P, i32, i64, i64, P, P, P, P, P, P, P]
+        L.mx_quantize_group.argtypes = [cfgp, i32, C.POINTER(mx_quantize_item), i32, P]
         L.mx_dequantize.argtypes = [cfgp, P, P, P, P, P, i64, i64, P, i32, P]
         L.mx_qsnr_workspace_bytes.argtypes = [i64, i64]
         L.mx_qsnr_workspace_bytes.restype = i64
@@ -120,7 +128,8 @@ def lib() -> C.CDLL:
         L.mx_strerror.argtypes = [C.c_int]
         L.mx_strerror.restype = C.c_char_p
         L.mx_version.restype = C.c_char_p
-        for f in ("mx_query_sizes", "mx_quantize", "mx_quantize_noalloc", "mx_hadamard_quantize", "mx_dequantize",
+        for f in ("mx_query_sizes", "mx_quantize", "mx_quantize_group", "mx_quantize_noalloc",
+                  "mx_hadamard_quantize", "mx_dequantize",
                   "mx_qsnr", "mx_gemm", "mx_gemm_qsnr", "mx_mbs_gemm_scales", "mx_device_status",
                   "mx_tensor_amax", "mx_stats_finalize", "mx_gemm_qsnr_finalize", "mx_tensor_peak"):
             getattr(L, f).restype = C.c_int
@@ -180,6 +189,12 @@ def mx_quantize(cfg: Config, x, x_dtype, rows, cols, codes, scales, tensor_scale
     c = cfg.c()
     return lib().mx_quantize(C.byref(c), x, x_dtype, rows, cols, codes, scales, tensor_scale,
                              macro, offsets, stats, workspace, workspace_bytes, stream)
+
+
+def mx_quantize_group(cfg: Config, x_dtype, items, n, stream) -> int:
+    """``items``: a ctypes array of ``mx_quantize_item``."""
+    c = cfg.c()
+    return lib().mx_quantize_group(C.byref(c), x_dtype, items, n, stream)
 
 
 def mx_tensor_amax(cfg: Config, x, x_dtype, rows, cols, workspace, workspace_bytes, stream) -> int:
@@ -334,6 +349,45 @@ def quantize(x: torch.Tensor, cfg: Config = MXFP4, *, stats: bool = True,
                          ws.numel(), st)
         _check("mx_quantize", rc)
     return q
+
+
+def quantize_group(xs, cfg: Config = MXFP4, *, stats: bool = True, outs=None, stream=None,
+                   workspaces=None) -> list:
+    """Block-quantize several 2-D CUDA tensors of one dtype with one
+    configuration (``mx_quantize_group``): the same results as one
+    ``quantize`` per tensor, with the tensors sharing launches.  ``outs`` /
+    ``workspaces``: optional lists with one entry per tensor (each tensor that
+    needs scratch gets its own; by default one scratch per position and
+    device)."""
+    xs = list(xs)
+    if not xs:
+        return []
+    for i, x in enumerate(xs):
+        _cuda2d(x, f"xs[{i}]")
+    dt = _dtype_code(xs[0])
+    if any(_dtype_code(x) != dt for x in xs):
+        raise TypeError("every tensor of a group has the same dtype")
+    qs = list(outs) if outs is not None else [alloc_outputs(cfg, *x.shape, x.device, stats) for x in xs]
+    items = (mx_quantize_item * len(xs))()
+    keep = []
+    for i, (x, q) in enumerate(zip(xs, qs)):
+        rows, cols = x.shape
+        if workspaces is not None:
+            ws = workspaces[i]
+        else:
+            nbytes = query_sizes(cfg, rows, cols).workspace_bytes
+            w = _default_ws.setdefault(str(x.device) if i == 0 else f"{x.device}#{i}", Workspace())
+            ws = w.get(nbytes, x.device)
+        keep.append(ws)
+        items[i] = mx_quantize_item(x.data_ptr(), rows, cols, q.codes.data_ptr(), q.scales.data_ptr(),
+                                    q.tensor_scale.data_ptr(), _ptr_or_none(q.macro), _ptr_or_none(q.offsets),
+                                    _ptr_or_none(q.stats), ws.data_ptr(), ws.numel())
+    _check("mx_quantize_group", mx_quantize_group(cfg, dt, items, len(xs), _stream(stream)))
+    return qs
+
+
+def _ptr_or_none(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
 
 
 def tensor_amax(x: torch.Tensor, cfg: Config, workspace: torch.Tensor, stream=None) -> None:

@@ -6,6 +6,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <new>
+
 #include "mx.h"
 #include "mx_internal.h"
 
@@ -165,11 +167,15 @@ int64_t codes_bytes_of(const mx_config *c, int64_t rows, int64_t cols)
 
 int cuda_ok(cudaError_t e) { return e == cudaSuccess ? MX_OK : MX_ERR_CUDA; }
 
-int quantize_impl(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t rows, int64_t cols,
-                  void *codes, uint8_t *scales, float *tensor_scale, uint8_t *macro_scales,
-                  uint16_t *offsets, double *stats, float *rotated, void *workspace,
-                  int64_t workspace_bytes, void *stream, bool want_had, bool amax_only = false)
+// Validation and launch parameters of one tensor of a quantize call.  *empty:
+// nothing to launch (the caller still writes the statistics of an empty
+// tensor).
+int prepare_quantize(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t rows, int64_t cols,
+                     void *codes, uint8_t *scales, float *tensor_scale, uint8_t *macro_scales,
+                     uint16_t *offsets, double *stats, float *rotated, void *workspace,
+                     int64_t workspace_bytes, bool want_had, bool amax_only, QParams &p, bool &empty)
 {
+    empty = false;
     int rc = check_config(cfg, rows, cols, want_had);
     if (rc != MX_OK) return rc;
     if (x_dtype != MX_DT_BF16 && x_dtype != MX_DT_FP32) return MX_ERR_INVALID;
@@ -181,11 +187,9 @@ int quantize_impl(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t 
     const bool need_ws = stats != nullptr || cfg->tensor_scale == MX_TS_COMPUTE ||
                          cfg->tensor_scale == MX_TS_AMAX || amax_only;
     if (need_ws && (!workspace || workspace_bytes < kWorkspaceBytes)) return MX_ERR_WORKSPACE;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t n = rows * cols;
     if (n == 0) {
-        if (amax_only) return MX_OK;
-        if (stats) return launch_finalize_stats(nullptr, 0, 0.0, stats, st) ? MX_ERR_CUDA : MX_OK;
+        empty = true;
         return MX_OK;
     }
     if (!x || (!amax_only && (!codes || !scales))) return MX_ERR_INVALID;
@@ -195,7 +199,6 @@ int quantize_impl(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t 
         (stats && ((uintptr_t)stats & 7u)) || (tensor_scale && ((uintptr_t)tensor_scale & 3u)))
         return MX_ERR_ALIGN;
 
-    QParams p;
     memset(&p, 0, sizeof(p));
     p.x = x;
     p.rows = rows;
@@ -221,28 +224,62 @@ int quantize_impl(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t 
     p.sf_gemm = cfg->sf_layout;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     p.amax_word = ws ? reinterpret_cast<unsigned int *>(ws) : nullptr;
-    double *partials = ws ? reinterpret_cast<double *>(ws + kWsHeader) : nullptr;
+    p.partials = (stats && ws) ? reinterpret_cast<double *>(ws + kWsHeader) : nullptr;
+    p.stats = stats;
+    p.count = (double)n;
+    p.ticket = need_ws ? reinterpret_cast<unsigned int *>(ws + kWsTicket) : nullptr;
+    return MX_OK;
+}
+
+// the element path of the fast (TMA ring) quantizer: E2M1, RTNE, symmetric,
+// not the MSE rule
+bool fast_elements(const mx_config *cfg)
+{
+    return cfg->elem == MX_E2M1 && cfg->round == MX_ROUND_RTNE && !cfg->asymmetric && cfg->rule != MX_RULE_MSE;
+}
+
+int quantize_impl(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t rows, int64_t cols,
+                  void *codes, uint8_t *scales, float *tensor_scale, uint8_t *macro_scales,
+                  uint16_t *offsets, double *stats, float *rotated, void *workspace,
+                  int64_t workspace_bytes, void *stream, bool want_had, bool amax_only = false)
+{
+    QParams p;
+    bool empty;
+    const int rc = prepare_quantize(cfg, x, x_dtype, rows, cols, codes, scales, tensor_scale, macro_scales,
+                                    offsets, stats, rotated, workspace, workspace_bytes, want_had, amax_only,
+                                    p, empty);
+    if (rc != MX_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (empty) {
+        if (amax_only) return MX_OK;
+        if (stats) return launch_finalize_stats(nullptr, 0, 0.0, stats, st) ? MX_ERR_CUDA : MX_OK;
+        return MX_OK;
+    }
     const int in_fp32 = x_dtype == MX_DT_FP32;
 
     // the tensor-amax pre-pass; the quantizer derives s_T from its word
     if ((cfg->tensor_scale == MX_TS_COMPUTE || amax_only) && launch_tensor_amax(p, cfg->axis, in_fp32, st))
         return MX_ERR_CUDA;
     if (amax_only) return MX_OK;
-    p.partials = stats ? partials : nullptr;
-    p.stats = stats;
-    p.count = (double)n;
-    p.ticket = need_ws ? reinterpret_cast<unsigned int *>(ws + kWsTicket) : nullptr;
-    const int fast = cfg->elem == MX_E2M1 && cfg->round == MX_ROUND_RTNE && !cfg->asymmetric &&
-                     cfg->rule != MX_RULE_MSE;
     if (cfg->rule == MX_RULE_MSE && cfg->scale_fmt != MX_SCALE_E8M0) {
         // (a computed tensor scale: the global-step passes reduce through the
         // workspace records and ticket, which need_ws has required)
+        uint8_t *ws = static_cast<uint8_t *>(workspace);
         float *chain = ws ? reinterpret_cast<float *>(ws + kWsMseChain) : nullptr;
+        double *partials = ws ? reinterpret_cast<double *>(ws + kWsHeader) : nullptr;
         return launch_quantize_mse(p, partials, chain, in_fp32, st) ? MX_ERR_CUDA : MX_OK;
     }
     int grid = 0;
-    if (launch_quantize(p, cfg->axis, in_fp32, fast, st, &grid)) return MX_ERR_CUDA;
+    if (launch_quantize(p, cfg->axis, in_fp32, fast_elements(cfg), st, &grid)) return MX_ERR_CUDA;
     return MX_OK;
+}
+
+// the configurations launch_quantize sends to the fast quantizer (without a
+// rotated output)
+bool groupable(const mx_config *cfg)
+{
+    return cfg->axis == MX_AXIS_ROW && fast_elements(cfg) &&
+           ((!cfg->macro_block && !cfg->hadamard) || cfg->block == 16 || cfg->block == 32);
 }
 
 }  // namespace
@@ -296,6 +333,70 @@ int mx_hadamard_quantize(const mx_config *cfg, const void *x, int32_t x_dtype, i
 {
     return quantize_impl(cfg, x, x_dtype, rows, cols, codes, scales, tensor_scale, macro_scales,
                          offsets, stats, rotated, workspace, workspace_bytes, stream, true);
+}
+
+int mx_quantize_group(const mx_config *cfg, int32_t x_dtype, const mx_quantize_item *items, int32_t n,
+                      void *stream)
+{
+    if (!cfg || !items || n < 1) return MX_ERR_INVALID;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    QParams *ps = new (std::nothrow) QParams[n];
+    bool *empty = new (std::nothrow) bool[n];
+    int rc = (ps && empty) ? MX_OK : MX_ERR_INVALID;
+    // every item is checked before anything is queued
+    for (int i = 0; i < n && rc == MX_OK; ++i) {
+        const mx_quantize_item &it = items[i];
+        rc = prepare_quantize(cfg, it.x, x_dtype, it.rows, it.cols, it.codes, it.scales, it.tensor_scale,
+                              it.macro_scales, it.offsets, it.stats, nullptr, it.workspace, it.workspace_bytes,
+                              cfg->hadamard != 0, false, ps[i], empty[i]);
+    }
+    // items that use their workspace must not share one
+    const bool uses_ws = cfg->tensor_scale == MX_TS_COMPUTE || cfg->tensor_scale == MX_TS_AMAX;
+    for (int i = 0; i < n && rc == MX_OK; ++i)
+        for (int j = i + 1; j < n && rc == MX_OK; ++j) {
+            const bool wi = items[i].stats || uses_ws, wj = items[j].stats || uses_ws;
+            if (!wi || !wj || !items[i].workspace || !items[j].workspace) continue;
+            const uintptr_t a0 = (uintptr_t)items[i].workspace, b0 = (uintptr_t)items[j].workspace;
+            if (a0 < b0 + (uintptr_t)kWorkspaceBytes && b0 < a0 + (uintptr_t)kWorkspaceBytes) rc = MX_ERR_INVALID;
+        }
+    const int in_fp32 = x_dtype == MX_DT_FP32;
+    if (rc == MX_OK && !groupable(cfg)) {
+        // other configurations: one call per tensor, in order
+        for (int i = 0; i < n && rc == MX_OK; ++i) {
+            const mx_quantize_item &it = items[i];
+            rc = quantize_impl(cfg, it.x, x_dtype, it.rows, it.cols, it.codes, it.scales, it.tensor_scale,
+                               it.macro_scales, it.offsets, it.stats, nullptr, it.workspace, it.workspace_bytes,
+                               stream, cfg->hadamard != 0);
+        }
+    } else if (rc == MX_OK) {
+        // empty tensors: their statistics; the others in launches of up to
+        // kFastGroupMax tensors (with the tensor-amax pre-pass of each launch's
+        // tensors before it)
+        QParams chunk[kFastGroupMax];
+        int m = 0;
+        for (int i = 0; i <= n && rc == MX_OK; ++i) {
+            if (i < n && empty[i]) {
+                if (items[i].stats && launch_finalize_stats(nullptr, 0, 0.0, items[i].stats, st)) rc = MX_ERR_CUDA;
+                continue;
+            }
+            if (i < n) chunk[m++] = ps[i];
+            if (m == kFastGroupMax || (i == n && m > 0)) {
+                if (cfg->tensor_scale == MX_TS_COMPUTE) {
+                    if (cfg->hadamard) {
+                        for (int k = 0; k < m && rc == MX_OK; ++k)
+                            if (launch_tensor_amax(chunk[k], cfg->axis, in_fp32, st)) rc = MX_ERR_CUDA;
+                    } else if (launch_tensor_amax_group(chunk, m, in_fp32, st)) {
+                        rc = MX_ERR_CUDA;
+                    }
+                }
+                if (rc == MX_OK && launch_quantize_fast_group(chunk, m, in_fp32, st)) rc = MX_ERR_CUDA;
+                m = 0;
+            }
+        }
+    }
+    delete[] ps;
+    delete[] empty;
+    return rc;
 }
 
 int mx_tensor_amax(const mx_config *cfg, const void *x, int32_t x_dtype, int64_t rows, int64_t cols,

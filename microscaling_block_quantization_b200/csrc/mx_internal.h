@@ -10,6 +10,8 @@ namespace mxk {
 // Upper bound on the CTAs of a reducing launch: each CTA writes one partial
 // record of kPartialDoubles doubles into the caller's workspace.
 constexpr int kMaxPartials = 4096;
+// tensors of one grouped quantizer launch
+constexpr int kFastGroupMax = 4;
 constexpr int kPartialDoubles = 8;
 // workspace: [0, 256) control words, then the partials.  Control words: the
 // tensor-amax accumulator at byte 0, the launch ticket at byte 64.  Both are
@@ -123,6 +125,11 @@ int launch_amax_col(const QParams &p, int in_fp32, cudaStream_t st);
 // E2M1 round-to-nearest-even, symmetric, row axis, no macro scale, rotation
 // or rotated output: the TMA-fed persistent quantizer.
 int launch_quantize_fast(const QParams &p, int in_fp32, cudaStream_t st, int *grid_out);
+// one launch over ps[0..n) (n <= kFastGroupMax, one configuration, every tensor
+// non-empty and eligible for launch_quantize_fast)
+int launch_quantize_fast_group(const QParams *ps, int n, int in_fp32, cudaStream_t st);
+// the tensor-amax pre-pass of ps[0..n) without rotation, one launch
+int launch_tensor_amax_group(const QParams *ps, int n, int in_fp32, cudaStream_t st);
 // Other element types / rounding modes / offsets, row axis, blocks of 32, no
 // macro scale, rotation or rotated output: the TMA-fed persistent quantizer.
 int launch_quantize_gen(const QParams &p, int in_fp32, cudaStream_t st, int *grid_out);

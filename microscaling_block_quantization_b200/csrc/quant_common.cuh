@@ -186,7 +186,7 @@ __device__ __forceinline__ double warp_sum(double v)
 
 // CTA reduction in a fixed order (lanes, then the warps' sums as one more
 // warp reduction); thread 0 writes the CTA's record.
-static __device__ __forceinline__ void write_partials(double *partials, const Acc &a)
+static __device__ __forceinline__ void write_partials(double *partials, const Acc &a, uint32_t rec)
 {
     __shared__ double sh[5][32];
     double v[5] = {a.x2, a.e2, a.e, a.ftz, a.nz};
@@ -199,7 +199,7 @@ static __device__ __forceinline__ void write_partials(double *partials, const Ac
     __syncthreads();
     if (w == 0) {
         const int nw = (int)(blockDim.x >> 5);
-        double *o = partials + (int64_t)blockIdx.x * kPartialDoubles;
+        double *o = partials + (int64_t)rec * kPartialDoubles;
 #pragma unroll
         for (int i = 0; i < 5; ++i) {
             const double t = warp_sum(lane < nw ? sh[i][lane] : 0.0);
@@ -211,14 +211,18 @@ static __device__ __forceinline__ void write_partials(double *partials, const Ac
 
 // Tensor scale of a launch: given, or s_T = amax / (max_elem * scale_max)
 // from the tensor-amax word of the pre-pass (amax = 0 -> 1); CTA 0 stores it.
-__device__ __forceinline__ float launch_tensor_scale(const QParams &p)
+__device__ __forceinline__ float launch_tensor_scale(const QParams &p, bool first_cta)
 {
     if (p.ts_mode == TS_NONE) return 1.0f;
     if (p.ts_mode == TS_GIVEN) return *p.tensor_scale;
     const float amax = __uint_as_float(__ldcg(p.amax_word));
     const float ts = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, __fmul_rn(p.ed.maxv, p.sd.ue_maxv));
-    if (blockIdx.x == 0 && threadIdx.x == 0) *p.tensor_scale = ts;
+    if (first_cta && threadIdx.x == 0) *p.tensor_scale = ts;
     return ts;
+}
+__device__ __forceinline__ float launch_tensor_scale(const QParams &p)
+{
+    return launch_tensor_scale(p, blockIdx.x == 0);
 }
 
 // The derived statistics of the summed records: MSE, R-MSE, QSNR Eq. (1),
@@ -247,9 +251,9 @@ __device__ __forceinline__ void store_stats(double *stats, const double s[5], do
 // CTA's record of the fidelity sums; then the last CTA to finish sums all
 // records in a fixed order into the statistics, and clears the tensor-amax
 // word and the ticket.
-__device__ __forceinline__ void finish_launch(const QParams &p, const Acc &a)
+__device__ __forceinline__ void finish_launch(const QParams &p, const Acc &a, uint32_t cta, uint32_t ncta)
 {
-    if (p.partials) write_partials(p.partials, a);
+    if (p.partials) write_partials(p.partials, a, cta);
     if (!p.ticket) return;
     // thread 0 wrote the record; its release-acquire ticket orders the record
     // before the last CTA's reads of it (the barrier below extends that
@@ -258,7 +262,7 @@ __device__ __forceinline__ void finish_launch(const QParams &p, const Acc &a)
     if (threadIdx.x == 0) {
         unsigned prev;
         asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(prev) : "l"(p.ticket) : "memory");
-        s_last = prev == gridDim.x - 1;
+        s_last = prev == ncta - 1;
     }
     __syncthreads();
     if (!s_last) return;
@@ -268,14 +272,14 @@ __device__ __forceinline__ void finish_launch(const QParams &p, const Acc &a)
         // for a given launch shape)
         __shared__ double red[5][32];
         double s[5] = {0, 0, 0, 0, 0};
-        for (unsigned i0 = threadIdx.x; i0 < gridDim.x; i0 += 2 * blockDim.x) {
+        for (unsigned i0 = threadIdx.x; i0 < ncta; i0 += 2 * blockDim.x) {
             const unsigned i1 = i0 + blockDim.x;
             double r0[5], r1[5];
 #pragma unroll
             for (int k = 0; k < 5; ++k) r0[k] = __ldcg(p.partials + (size_t)i0 * kPartialDoubles + k);
 #pragma unroll
             for (int k = 0; k < 5; ++k)
-                r1[k] = i1 < gridDim.x ? __ldcg(p.partials + (size_t)i1 * kPartialDoubles + k) : 0.0;
+                r1[k] = i1 < ncta ? __ldcg(p.partials + (size_t)i1 * kPartialDoubles + k) : 0.0;
 #pragma unroll
             for (int k = 0; k < 5; ++k) s[k] += r0[k] + r1[k];
         }
@@ -298,6 +302,10 @@ __device__ __forceinline__ void finish_launch(const QParams &p, const Acc &a)
         if (p.ts_mode == TS_COMPUTE) *p.amax_word = 0u;
         *p.ticket = 0u;
     }
+}
+__device__ __forceinline__ void finish_launch(const QParams &p, const Acc &a)
+{
+    finish_launch(p, a, blockIdx.x, gridDim.x);
 }
 
 // x_hat of one element from its grid value q (the dequantization rule).

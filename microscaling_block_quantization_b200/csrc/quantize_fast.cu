@@ -10,6 +10,8 @@
 // reads of its own chunk are bank-conflict free), each consumer lane
 // quantizes one chunk per tile: all of HBM's latency is covered by the ring,
 // and the registers hold no load buffers.  Every mbarrier wait is bounded.
+#include <string.h>
+
 #include "tma_ring.cuh"
 
 namespace mxk {
@@ -187,11 +189,22 @@ __device__ __forceinline__ void ring_read_words(const uint8_t *stage, int t, uin
     }
 }
 
+// A launch over up to kFastGroupMax tensors of one configuration: the CTAs
+// are split among the tensors (cta0 prefix), every CTA works on one tensor
+// with that tensor's tensor map and outputs; p[0] also carries the shared
+// configuration.
+struct FastGroup {
+    CUtensorMap tm[kFastGroupMax];
+    QParams p[kFastGroupMax];
+    uint32_t cta0[kFastGroupMax + 1];
+    int n;
+};
+
 // HADN: block rotation over groups of HADN (0: none, 16, 32) before
 // quantization; MBS: 1 x 128 macro scale over the
 // 4 lanes of a macro block (consecutive chunks of a tile are consecutive lanes).
 template <typename InT, int B, bool STATS, int HADN, bool MBS, bool NEAR>
-__global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && sizeof(InT) != 2)) ? 2 : 3) k_quant_fast(const QParams p, const __grid_constant__ CUtensorMap tm)
+__global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && sizeof(InT) != 2)) ? 2 : 3) k_quant_fast(const __grid_constant__ FastGroup g)
 {
     constexpr int NB = B <= 32 ? 32 / B : 1;
     constexpr int G = B <= 32 ? 1 : B / 32;
@@ -199,18 +212,24 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
     extern __shared__ uint8_t smem_raw[];
     const Ring<InT> ring(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // this CTA's tensor, and its place among the tensor's CTAs
+    int item = 0;
+    while (item + 1 < g.n && blockIdx.x >= g.cta0[item + 1]) ++item;
+    const QParams &pc = g.p[0];
+    const QParams &p = g.p[item];
+    const uint32_t cta = blockIdx.x - g.cta0[item], ncta = g.cta0[item + 1] - g.cta0[item];
     const uint32_t nch = (uint32_t)(p.rows * p.cols / 32);
     const uint32_t ntiles = (nch + kConsumers - 1) / kConsumers;
     pdl_trigger();
     if (threadIdx.x == 0) ring.init();
     pdl_wait();
-    const float sT = launch_tensor_scale(p);
+    const float sT = launch_tensor_scale(p, cta == 0);
     // nearest scales: s_b s_T and its reciprocal for every scale code, once per CTA
     __shared__ float2 near_tab[NEAR ? 256 : 1];
     if constexpr (NEAR)
         for (int c = threadIdx.x; c < 256; c += blockDim.x) {
-            const float d = __fmul_rn(ue_value(p.sd, (uint32_t)c), sT);
-            near_tab[c] = c < p.sd.ue_nan_code ? make_float2(d, __fdiv_rn(1.0f, d))
+            const float d = __fmul_rn(ue_value(pc.sd, (uint32_t)c), sT);
+            near_tab[c] = c < pc.sd.ue_nan_code ? make_float2(d, __fdiv_rn(1.0f, d))
                                                : make_float2(__uint_as_float(0x7fc00000u), 0.0f);
         }
     // macro scales: {S_M, RN(1 / S_M)} for every E4M3 code, once per CTA
@@ -220,17 +239,17 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
             const float v = e4m3_value((uint32_t)c);
             macro_tab[c] = make_float2(v, __fdiv_rn(1.0f, v));
         }
-    const float md = MBS ? __fmul_rn(p.ed.maxv, exp2i(-p.ed.emax)) : 1.0f;   // max_elem / 2^emax, exact
+    const float md = MBS ? __fmul_rn(pc.ed.maxv, exp2i(-pc.ed.emax)) : 1.0f;   // max_elem / 2^emax, exact
     const float r_md = MBS ? __fdiv_rn(1.0f, md) : 1.0f;
     __syncthreads();
     NearScale ns;
-    ns.maxv = p.ed.maxv;
-    ns.r_max = __fdiv_rn(1.0f, p.ed.maxv);
+    ns.maxv = pc.ed.maxv;
+    ns.r_max = __fdiv_rn(1.0f, pc.ed.maxv);
     ns.sT = sT;
     ns.r_T = (sT >= 0x1p-125f && sT <= 0x1p125f) ? __fdiv_rn(1.0f, sT) : 0.0f;
     {
         // the UE4M3 shortcut's constant, when max_elem s_T and its reciprocal are normal
-        const float ms = __fmul_rn(p.ed.maxv, sT);
+        const float ms = __fmul_rn(pc.ed.maxv, sT);
         ns.c = (ms >= 0x1p-125f && ms <= 0x1p125f) ? __fdiv_rn(1.0f, ms) : 0.0f;
     }
     ns.tab = near_tab;
@@ -238,7 +257,7 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
     Acc acc = {0, 0, 0, 0, 0};
     if (warp == kConsumers / 32) {
         // producer: one lane streams the CTA's tiles through the ring
-        if (lane == 0) ring.produce(&tm, ntiles, kWaitEmpty);
+        if (lane == 0) ring.produce(&g.tm[item], ntiles, kWaitEmpty, cta, ncta);
         __syncwarp();
     } else {
         // rotation with power-of-two scales: the normaliser c = 1/sqrt(n) moves
@@ -248,12 +267,12 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
         constexpr bool PACKED = sizeof(InT) == 2 && HADN == 0;
         constexpr bool ROT16 = sizeof(InT) == 2 && HADN != 0;
         const float hc = HADN ? hadamard_scale(HADN) : 1.0f;
-        const bool e8m0 = !NEAR && p.sd.fmt == S_E8M0;
-        const float thr_m = e8m0_threshold(p.ed, p.sd);
+        const bool e8m0 = !NEAR && pc.sd.fmt == S_E8M0;
+        const float thr_m = e8m0_threshold(pc.ed, pc.sd);
         const uint32_t S = (uint32_t)(p.cols / B);
         const int t = threadIdx.x;
         uint32_t i = 0;
-        for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+        for (uint32_t tile = cta; tile < ntiles; tile += ncta, ++i) {
             if (!ring.acquire(i, kWaitFull)) break;
             float y[PACKED ? 1 : 32];
             uint32_t w[PACKED || ROT16 ? 16 : 1];
@@ -337,9 +356,9 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
 #pragma unroll
                 for (int k = 0; k < NB; ++k) {
                     const uint32_t *wb = w + k * (L / 2);
-                    const BlockScale bs = NEAR ? near_block_scale(p.sd, ns, bad[k] ? 0.0f : a[k], bad[k])
-                                        : e8m0 ? e8m0_block_scale(bad[k] ? 0.0f : a[k], bad[k], p.ed.emax, thr_m)
-                                               : block_scale(p.ed, p.sd, bad[k] ? 0.0f : a[k], bad[k], sT);
+                    const BlockScale bs = NEAR ? near_block_scale(pc.sd, ns, bad[k] ? 0.0f : a[k], bad[k])
+                                        : e8m0 ? e8m0_block_scale(bad[k] ? 0.0f : a[k], bad[k], pc.ed.emax, thr_m)
+                                               : block_scale(pc.ed, pc.sd, bad[k] ? 0.0f : a[k], bad[k], sT);
                     scode[k] = bs.code;
                     float deqT = bs.nan ? __uint_as_float(0x7fc00000u) : bs.deq;
                     if (MBS) deqT = __fmul_rn(deqT, sm);       // X S_M, exact (E4M3 times a power of two)
@@ -432,9 +451,9 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
                     bad = grp_or(bad, G);
                 }
                 if (FOLD) a = __fmul_rn(a, hc);            // max |y_H c| = RN(max |y_H| c)
-                const BlockScale bs = NEAR ? near_block_scale(p.sd, ns, bad ? 0.0f : a, bad)
-                                    : e8m0 ? e8m0_block_scale(bad ? 0.0f : a, bad, p.ed.emax, thr_m)
-                                           : block_scale(p.ed, p.sd, bad ? 0.0f : a, bad, sT);
+                const BlockScale bs = NEAR ? near_block_scale(pc.sd, ns, bad ? 0.0f : a, bad)
+                                    : e8m0 ? e8m0_block_scale(bad ? 0.0f : a, bad, pc.ed.emax, thr_m)
+                                           : block_scale(pc.ed, pc.sd, bad ? 0.0f : a, bad, sT);
                 scode[k] = bs.code;
                 float deqT = bs.nan ? __uint_as_float(0x7fc00000u) : bs.deq;     // nearest: s_b s_T
                 if (MBS) deqT = __fmul_rn(deqT, sm);       // X * S_M is exact (power of two times E4M3)
@@ -511,7 +530,7 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
                 reinterpret_cast<uint4 *>(p.codes)[c] = make_uint4(words[0], words[1], words[2], words[3]);
                 if (G == 1 || (lane & (G - 1)) == 0) {
                     const uint32_t b0 = (G == 1) ? c * NB : c / G;
-                    if (p.sf_gemm) {
+                    if (pc.sf_gemm) {
                         const uint32_t r = b0 / S, j = b0 - r * S;
 #pragma unroll
                         for (int k = 0; k < NB; ++k) p.scales[sf_chunk_index(r, j + k, S)] = (uint8_t)scode[k];
@@ -532,62 +551,97 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
             }
         }
     }
-    finish_launch(p, acc);
+    finish_launch(p, acc, cta, ncta);
+}
+
+// CTAs of a grouped launch: one per tensor, then one at a time to the tensor
+// with the most tiles per CTA (as long as it has more tiles than CTAs)
+void split_ctas(const uint64_t *tiles, int n, uint64_t total, uint32_t *cta0)
+{
+    uint64_t c[kFastGroupMax], sum = 0;
+    for (int i = 0; i < n; ++i) {
+        c[i] = 1;
+        sum += tiles[i];
+    }
+    if (total > sum) total = sum;
+    for (uint64_t k = n; k < total; ++k) {
+        int best = -1;
+        for (int i = 0; i < n; ++i)
+            if (c[i] < tiles[i] && (best < 0 || tiles[i] * c[best] > tiles[best] * c[i])) best = i;
+        if (best < 0) break;
+        ++c[best];
+    }
+    cta0[0] = 0;
+    for (int i = 0; i < n; ++i) cta0[i + 1] = cta0[i] + (uint32_t)c[i];
 }
 
 template <typename InT, int B, bool STATS, int HADN, bool MBS, bool NEAR>
-int launch_fast_b(const QParams &p, cudaStream_t st, int *grid_out)
+int launch_fast_b(const QParams *ps, int n, cudaStream_t st)
 {
-    const uint64_t nch = (uint64_t)(p.rows * p.cols / 32);
-    CUtensorMap tm;
-    if (ring_map<InT>(&tm, p.x, nch) != 0) return -1;
+    FastGroup g;
+    memset(&g, 0, sizeof(g));
+    uint64_t tiles[kFastGroupMax];
+    for (int i = 0; i < n; ++i) {
+        const uint64_t nch = (uint64_t)(ps[i].rows * ps[i].cols / 32);
+        if (ring_map<InT>(&g.tm[i], ps[i].x, nch) != 0) return -1;
+        g.p[i] = ps[i];
+        tiles[i] = (nch + kConsumers - 1) / kConsumers;
+    }
+    g.n = n;
     auto k = k_quant_fast<InT, B, STATS, HADN, MBS, NEAR>;
-    const unsigned g = ring_grid(reinterpret_cast<const void *>(k), RingCfg<InT>::kSmem, nch);
-    const cudaError_t e = launch_pdl(k, g, kFastThreads, RingCfg<InT>::kSmem, st, p, tm);
-    *grid_out = (int)g;
+    const int occ = cached_occupancy(reinterpret_cast<const void *>(k), kFastThreads, RingCfg<InT>::kSmem);
+    uint64_t total = (uint64_t)device_sm_count() * occ;
+    if (total > (uint64_t)kMaxPartials) total = kMaxPartials;
+    if (total < (uint64_t)n) total = n;
+    split_ctas(tiles, n, total, g.cta0);
+    const cudaError_t e = launch_pdl(k, g.cta0[n], kFastThreads, RingCfg<InT>::kSmem, st, g);
     return e == cudaSuccess ? 0 : -1;
 }
 
 // statistics on / off; nearest (UE4M3 / UE5M3) or power-of-two scales (the
 // macro scale comes only with E8M0)
 template <typename InT, int B, int HADN, bool MBS>
-int launch_fast_s(const QParams &p, cudaStream_t st, int *grid_out)
+int launch_fast_s(const QParams *ps, int n, cudaStream_t st)
 {
+    const QParams &p = ps[0];
     const bool near = p.sd.fmt != S_E8M0 && p.sd.rule == R_NEAREST;
+    bool stats = false;
+    for (int i = 0; i < n; ++i) stats = stats || ps[i].partials != nullptr;
     if (MBS || !near)
-        return p.partials ? launch_fast_b<InT, B, true, HADN, MBS, false>(p, st, grid_out)
-                          : launch_fast_b<InT, B, false, HADN, MBS, false>(p, st, grid_out);
-    return p.partials ? launch_fast_b<InT, B, true, HADN, false, true>(p, st, grid_out)
-                      : launch_fast_b<InT, B, false, HADN, false, true>(p, st, grid_out);
+        return stats ? launch_fast_b<InT, B, true, HADN, MBS, false>(ps, n, st)
+                     : launch_fast_b<InT, B, false, HADN, MBS, false>(ps, n, st);
+    return stats ? launch_fast_b<InT, B, true, HADN, false, true>(ps, n, st)
+                 : launch_fast_b<InT, B, false, HADN, false, true>(ps, n, st);
 }
 
 template <typename InT, int B>
-int launch_fast_rot(const QParams &p, cudaStream_t st, int *grid_out)
+int launch_fast_rot(const QParams *ps, int n, cudaStream_t st)
 {
-    const bool m = p.mbs != 0;
-    switch (p.had) {
-    case 0: return launch_fast_s<InT, B, 0, true>(p, st, grid_out);
-    case 16: return m ? launch_fast_s<InT, B, 16, true>(p, st, grid_out) : launch_fast_s<InT, B, 16, false>(p, st, grid_out);
-    case 32: return m ? launch_fast_s<InT, B, 32, true>(p, st, grid_out) : launch_fast_s<InT, B, 32, false>(p, st, grid_out);
+    const bool m = ps[0].mbs != 0;
+    switch (ps[0].had) {
+    case 0: return launch_fast_s<InT, B, 0, true>(ps, n, st);
+    case 16: return m ? launch_fast_s<InT, B, 16, true>(ps, n, st) : launch_fast_s<InT, B, 16, false>(ps, n, st);
+    case 32: return m ? launch_fast_s<InT, B, 32, true>(ps, n, st) : launch_fast_s<InT, B, 32, false>(ps, n, st);
     default: return -1;
     }
 }
 
 template <typename InT>
-int launch_fast_t(const QParams &p, cudaStream_t st, int *grid_out)
+int launch_fast_t(const QParams *ps, int n, cudaStream_t st)
 {
+    const QParams &p = ps[0];
     if (p.had || p.mbs) {
         // rotation and / or macro scale: blocks of 16 and 32
-        if (p.block == 32) return launch_fast_rot<InT, 32>(p, st, grid_out);
-        return launch_fast_rot<InT, 16>(p, st, grid_out);
+        if (p.block == 32) return launch_fast_rot<InT, 32>(ps, n, st);
+        return launch_fast_rot<InT, 16>(ps, n, st);
     }
     switch (p.block) {
-    case 8: return launch_fast_s<InT, 8, 0, false>(p, st, grid_out);
-    case 16: return launch_fast_s<InT, 16, 0, false>(p, st, grid_out);
-    case 32: return launch_fast_s<InT, 32, 0, false>(p, st, grid_out);
-    case 64: return launch_fast_s<InT, 64, 0, false>(p, st, grid_out);
-    case 128: return launch_fast_s<InT, 128, 0, false>(p, st, grid_out);
-    case 256: return launch_fast_s<InT, 256, 0, false>(p, st, grid_out);
+    case 8: return launch_fast_s<InT, 8, 0, false>(ps, n, st);
+    case 16: return launch_fast_s<InT, 16, 0, false>(ps, n, st);
+    case 32: return launch_fast_s<InT, 32, 0, false>(ps, n, st);
+    case 64: return launch_fast_s<InT, 64, 0, false>(ps, n, st);
+    case 128: return launch_fast_s<InT, 128, 0, false>(ps, n, st);
+    case 256: return launch_fast_s<InT, 256, 0, false>(ps, n, st);
     default: return -1;
     }
 }
@@ -595,10 +649,18 @@ int launch_fast_t(const QParams &p, cudaStream_t st, int *grid_out)
 }  // namespace
 
 // E2M1 / RTNE / symmetric, row axis, no rotated output; rotation and macro
-// scale only with blocks of 16 or 32.
+// scale only with blocks of 16 or 32.  ps[0..n) share the configuration
+// (n <= kFastGroupMax, every tensor non-empty).
+int launch_quantize_fast_group(const QParams *ps, int n, int in_fp32, cudaStream_t st)
+{
+    if (n < 1 || n > kFastGroupMax) return -1;
+    return in_fp32 ? launch_fast_t<float>(ps, n, st) : launch_fast_t<__nv_bfloat16>(ps, n, st);
+}
+
 int launch_quantize_fast(const QParams &p, int in_fp32, cudaStream_t st, int *grid_out)
 {
-    return in_fp32 ? launch_fast_t<float>(p, st, grid_out) : launch_fast_t<__nv_bfloat16>(p, st, grid_out);
+    if (grid_out) *grid_out = 0;
+    return launch_quantize_fast_group(&p, 1, in_fp32, st);
 }
 
 int take_status_fast(cudaStream_t st, int *v) { return take_ring_status(st, v); }

@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kRingThreads, 2) k_quant_gen(const QParams p, 
     Acc acc = {0, 0, 0, 0, 0};
     const bool stats = p.partials != nullptr;
     if (warp == kRingConsumers / 32) {
-        if (lane == 0) ring.produce(&tm, ntiles, kWaitEmpty);
+        if (lane == 0) ring.produce(&tm, ntiles, kWaitEmpty, blockIdx.x, gridDim.x);
     } else {
         const float sT = launch_tensor_scale(p);
         const bool nearest = p.sd.fmt != S_E8M0 && p.sd.rule == R_NEAREST;

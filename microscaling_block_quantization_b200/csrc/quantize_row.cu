@@ -11,6 +11,7 @@
 // rotation fused with quantization); fmread summary of Yang et al. (rounding
 // modes, asymmetric scaling, row / column / 2D blocks).
 #include <mutex>
+#include <string.h>
 
 #include "quant_common.cuh"
 
@@ -293,23 +294,36 @@ __global__ void __launch_bounds__(kThreads) k_amax_row(const QParams p)
     if (lane == 0 && m > 0.0f) atomicMax(p.amax_word, __float_as_uint(m));
 }
 
-// Tensor absmax without rotation (any block axis): consecutive lanes read
-// consecutive 16-byte vectors, four in flight per thread, NaN skipped.  The
-// tensor is walked from its end towards its start, so that the quantizer's
-// forward walk that follows first meets the lines this pass touched last
-// (still in L2 when the tensor is not much larger than L2).
+// Tensor absmax without rotation (any block axis), of up to kFastGroupMax
+// tensors in one launch (the CTAs split among them in proportion to their
+// sizes): consecutive lanes read consecutive 16-byte vectors, four in flight
+// per thread, NaN skipped.  Each tensor is walked from its end towards its
+// start, so that the quantizer's forward walk that follows first meets the
+// lines this pass touched last (still in L2 when the tensor is not much
+// larger than L2).
+struct AmaxGroup {
+    const void *x[kFastGroupMax];
+    uint64_t nv[kFastGroupMax];             // 16-byte vectors
+    unsigned int *word[kFastGroupMax];
+    uint32_t cta0[kFastGroupMax + 1];
+    int n;
+};
+
 template <typename InT>
-__global__ void __launch_bounds__(kThreads) k_amax_vec(const QParams p)
+__global__ void __launch_bounds__(kThreads) k_amax_vec(const __grid_constant__ AmaxGroup g)
 {
     constexpr int U = 4;
-    const uint4 *x = static_cast<const uint4 *>(p.x);
-    const uint64_t nv = (uint64_t)(p.rows * p.cols) * sizeof(InT) / 16;
-    const uint64_t T = (uint64_t)gridDim.x * blockDim.x;
+    int item = 0;
+    while (item + 1 < g.n && blockIdx.x >= g.cta0[item + 1]) ++item;
+    const uint4 *x = static_cast<const uint4 *>(g.x[item]);
+    const uint64_t nv = g.nv[item];
+    const uint64_t cta = blockIdx.x - g.cta0[item];
+    const uint64_t T = (uint64_t)(g.cta0[item + 1] - g.cta0[item]) * blockDim.x;
     pdl_trigger();
     pdl_wait();
     float m = 0.0f;
     __nv_bfloat162 m2 = __float2bfloat162_rn(0.0f);
-    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv; i += U * T) {
+    for (uint64_t i = cta * blockDim.x + threadIdx.x; i < nv; i += U * T) {
         uint4 u[U];
 #pragma unroll
         for (int k = 0; k < U; ++k) {
@@ -334,7 +348,42 @@ __global__ void __launch_bounds__(kThreads) k_amax_vec(const QParams p)
         m = fmaxf(f.x, f.y);
     }
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-    if ((threadIdx.x & 31) == 0 && m > 0.0f) atomicMax(p.amax_word, __float_as_uint(m));
+    if ((threadIdx.x & 31) == 0 && m > 0.0f) atomicMax(g.word[item], __float_as_uint(m));
+}
+
+template <typename InT>
+int launch_amax_vec(const QParams *ps, int n, cudaStream_t st)
+{
+    AmaxGroup g;
+    memset(&g, 0, sizeof(g));
+    uint64_t warps[kFastGroupMax], sum = 0;
+    for (int i = 0; i < n; ++i) {
+        g.x[i] = ps[i].x;
+        g.nv[i] = (uint64_t)(ps[i].rows * ps[i].cols) * sizeof(InT) / 16;
+        g.word[i] = ps[i].amax_word;
+        warps[i] = (g.nv[i] / 4 + 31) / 32;
+        sum += warps[i];
+    }
+    g.n = n;
+    // the one-tensor grid for the sum of the tensors, then a share of it per
+    // tensor in proportion to its vectors (at least one CTA each)
+    const int total = grid_for(k_amax_vec<InT>, (int64_t)sum);
+    g.cta0[0] = 0;
+    uint64_t given = 0, acc = 0;
+    for (int i = 0; i < n; ++i) {
+        acc += warps[i];
+        uint64_t upto = sum ? (uint64_t)total * acc / sum : (uint64_t)i + 1;
+        if (upto < given + 1) upto = given + 1;
+        g.cta0[i + 1] = (uint32_t)upto;
+        given = upto;
+    }
+    return launch_pdl(k_amax_vec<InT>, g.cta0[n], kThreads, 0, st, g) == cudaSuccess ? 0 : -1;
+}
+
+int launch_tensor_amax_group(const QParams *ps, int n, int in_fp32, cudaStream_t st)
+{
+    if (n < 1 || n > kFastGroupMax) return -1;
+    return in_fp32 ? launch_amax_vec<float>(ps, n, st) : launch_amax_vec<__nv_bfloat16>(ps, n, st);
 }
 
 // Sum the per-CTA records in a fixed order and derive MSE, R-MSE, QSNR (Eq. (1)),
@@ -443,14 +492,7 @@ int launch_tensor_amax(const QParams &p, int axis, int in_fp32, cudaStream_t st)
     if (axis == AX_COL && p.had) {
         if (launch_amax_col(p, in_fp32, st)) return -1;
     } else if (!p.had) {
-        const int64_t warps = (p.rows * p.cols / 8 / 4 + 31) / 32;
-        if (in_fp32) {
-            const int g = grid_for(k_amax_vec<float>, warps);
-            e = launch_pdl(k_amax_vec<float>, g, kThreads, 0, st, p);
-        } else {
-            const int g = grid_for(k_amax_vec<__nv_bfloat16>, warps);
-            e = launch_pdl(k_amax_vec<__nv_bfloat16>, g, kThreads, 0, st, p);
-        }
+        if (launch_tensor_amax_group(&p, 1, in_fp32, st)) return -1;
     } else {
         const int64_t tiles = (p.rows * p.cols / 32 + 31) / 32;
         if (in_fp32) {

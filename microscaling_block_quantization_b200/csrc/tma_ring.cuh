@@ -79,8 +79,9 @@ struct Ring {
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    // producer lane: the CTA's tiles blockIdx.x, blockIdx.x + gridDim.x, ...
-    __device__ __forceinline__ void produce(const CUtensorMap *tm, uint32_t ntiles, int where) const
+    // producer lane: the CTA's tiles first, first + stride, ...
+    __device__ __forceinline__ void produce(const CUtensorMap *tm, uint32_t ntiles, int where, uint32_t first,
+                                            uint32_t stride) const
     {
         constexpr uint32_t S = RingCfg<InT>::kStages;
         // the quantizer reads each input line once: mark it first to evict,
@@ -88,7 +89,7 @@ struct Ring {
         uint64_t pol;
         asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
         uint32_t i = 0;
-        for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+        for (uint32_t tile = first; tile < ntiles; tile += stride, ++i) {
             const uint32_t s = i % S;
             if (i >= S && !ring_wait(&empty[s], ((i / S) - 1) & 1, where)) break;
             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"

@@ -140,6 +140,33 @@ def test_sharding_entry_points_checked_on_host(mx):
     assert mx.mx_stats_finalize(P(4100), None) == -3
 
 
+def test_group_checked_on_host(mx):
+    """mx_quantize_group checks every item before anything is queued: an
+    invalid item fails the whole call with that item's error, and two items
+    whose statistics would share one workspace are rejected."""
+    P = C.c_void_p
+    WS = 1 << 20
+
+    def item(x=4096, rows=64, cols=64, stats=None, ws=None, wsb=0):
+        return mx.mx_quantize_item(x, rows, cols, 4096, 4096, 4096, None, None, stats, ws, wsb)
+
+    def call(cfg, *its):
+        arr = (mx.mx_quantize_item * max(len(its), 1))(*its)
+        return mx.mx_quantize_group(cfg, 0, arr, len(its), None)
+
+    assert mx.lib().mx_quantize_group(None, 0, None, 1, None) == -1
+    assert mx.mx_quantize_group(mx.MXFP4, 0, None, 1, None) == -1
+    assert call(mx.MXFP4) == -1                                         # no items
+    assert call(mx.MXFP4, item(), item(cols=48)) == -1                  # cols % 32
+    assert call(mx.MXFP4, item(), item(x=4100)) == -3                   # misaligned input
+    assert call(mx.MXFP4, item(), item(stats=4096)) == -5               # statistics without a workspace
+    assert call(mx.MXFP4, item(stats=4096, ws=1 << 24, wsb=WS),
+                item(stats=8192, ws=(1 << 24) + 4096, wsb=WS)) == -1    # one workspace for two tensors
+    assert call(mx.NVFP4, item(ws=1 << 24, wsb=WS), item(ws=1 << 24, wsb=WS)) == -1
+    assert call(mx.Config(elem=9), item()) == -1
+    assert call(mx.Config(block=16, scale_fmt=mx.SCALE_UE4M3, rule=mx.RULE_NEAREST, tensor_scale=4), item()) == -1
+
+
 def test_element_limit_checked_on_host(mx):
     """Calls take fewer than 2^32 elements (32-bit indices in the kernels)."""
     P = C.c_void_p

@@ -1,12 +1,13 @@
 """GPU parity of the launches the benchmark times, element by element.
 
-Every quantizer launch of the benchmark's step -- MXFP4, NVFP4 (tensor-amax
+Every quantizer call of the benchmark's step -- MXFP4, NVFP4 (tensor-amax
 pass + UE4M3 nearest scales), 32-point Hadamard + MXFP4 without the rotated
 tensor (the TMA-fed quantizer's rotation path) and MBS + OAS(7) MXFP4 -- on
 the full Llama-3-8B layer operands, A 8192 x 4096 and W 14336 x 4096, in the
-configuration the benchmark launches them with: packed codes, scales, macro
-scales, tensor scale and the dequantized tensor bit-exact against the
-oracle, statistics within 1e-4.  Then the same kernels on small ragged
+configuration the benchmark launches them with (one grouped launch over A and
+W per variant): packed codes, scales, macro scales, tensor scale and the
+dequantized tensor of each tensor bit-exact against the oracle, statistics
+within 1e-4; the same tensors quantized alone give the same bits.  Then the same kernels on small ragged
 shapes for every rotation x scale combination, and the UE4M3 / UE5M3
 nearest-scale block-size sweep of "Is Finer Better?" (experimental analysis:
 blocks 8 to 256, with and without the FP32 tensor scale).
@@ -47,20 +48,37 @@ def _step_quantizers(mx):
     return {(name, t): cfg for name, t, cfg, kind in bench.step_plan(mx) if kind == "q"}
 
 
-@pytest.mark.parametrize("tensor", ["A", "W"])
 @pytest.mark.parametrize("name", ["mxfp4_row", "nvfp4_row", "had32_mxfp4", "mbs_oas_mxfp4"])
-def test_step_launch_full_size(mx, orc, name, tensor):
-    """One quantizer launch of the benchmark's step on its full-size operand
-    (no rotated output: the launch configuration the step times), and the
-    step's bf16 dequantizer on the MXFP4 codes."""
-    cfg = _step_quantizers(mx)[(name, tensor)]
-    run_case(mx, orc, _layer()[tensor], cfg, want_rotated=False, bf16_out=(name == "mxfp4_row"))
+def test_step_call_full_size(mx, orc, name):
+    """One quantizer call of the benchmark's step, the grouped launch over the
+    full-size A and W (no rotated output: the launch configuration the step
+    times), and the step's bf16 dequantizer on the MXFP4 codes; then each
+    tensor quantized alone, which must give the same bits."""
+    calls = {n: (ts, cfg) for n, ts, cfg, kind in bench.step_calls(bench.step_plan(mx)) if kind == "q"}
+    ts, cfg = calls[name]
+    assert ts == ("A", "W")
+    L = _layer()
+    xs = [L[t].cuda() for t in ts]
+    qs = mx.quantize_group(xs, cfg)
+    torch.cuda.synchronize()
+    for t, q in zip(ts, qs):
+        run_case(mx, orc, L[t], cfg, want_rotated=False, bf16_out=(name == "mxfp4_row"), q=q)
+    for x, q in zip(xs, qs):
+        a = mx.quantize(x, cfg)
+        torch.cuda.synchronize()
+        assert torch.equal(a.codes, q.codes) and torch.equal(a.scales, q.scales)
+        assert torch.equal(a.tensor_scale, q.tensor_scale)
+        if cfg.macro_block:
+            assert torch.equal(a.macro, q.macro)
 
 
 def test_step_plan_is_covered(mx):
-    """Every quantizer launch of the benchmark's step is one of the cases above."""
+    """Every quantizer launch of the benchmark's step is one of the cases
+    above, and the step issues each variant as one call over A and W."""
     names = {name for name, _ in _step_quantizers(mx)}
     assert names == {"mxfp4_row", "nvfp4_row", "had32_mxfp4", "mbs_oas_mxfp4"}
+    qcalls = [c for c in bench.step_calls(bench.step_plan(mx)) if c[3] == "q"]
+    assert sorted(c[0] for c in qcalls) == sorted(names) and all(c[1] == ("A", "W") for c in qcalls)
 
 
 RAGGED = [(40, 640), (96, 1152), (1, 128), (264, 384)]

@@ -61,20 +61,21 @@ def assert_stats(g, o, n):
     assert g[3] == o[3] and g[4] == o[4] and g[10] == o[10]
 
 
-def run_case(mx, orc, x_cpu, cfg, check_stats=True, given_ts=None, want_rotated=None, bf16_out=False):
+def run_case(mx, orc, x_cpu, cfg, check_stats=True, given_ts=None, want_rotated=None, bf16_out=False, q=None):
     """Quantize on the GPU and with the oracle; compare every output.
     want_rotated: ask the library for the rotated tensor y too (default: when
     the config rotates).  Without it, a rotation with blocks of 16 or 32 runs
     on the TMA-fed quantizer, with it on the lane-per-chunk kernel.
-    bf16_out: also compare the bf16 dequantized tensor."""
+    bf16_out: also compare the bf16 dequantized tensor.  q: outputs the GPU
+    already produced for x_cpu (a grouped call), checked instead of a new call."""
     rows, cols = x_cpu.shape
-    x = x_cpu.cuda()
     ts_in = None
     if given_ts is not None:
         ts_in = torch.tensor([given_ts], dtype=torch.float32, device="cuda")
     if want_rotated is None:
         want_rotated = bool(cfg.hadamard)
-    q = mx.quantize(x, cfg, stats=check_stats, tensor_scale=ts_in, rotated=want_rotated)
+    if q is None:
+        q = mx.quantize(x_cpu.cuda(), cfg, stats=check_stats, tensor_scale=ts_in, rotated=want_rotated)
     xh = mx.dequantize(q, torch.float32)
     torch.cuda.synchronize()
     oc = ocfg(orc, cfg)
