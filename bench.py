@@ -52,7 +52,8 @@ def parse():
                     help="capture the step on one stream (default: two streams, see run_ours)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-case", default=None,
-                    help="run one kernel alone (for ncu captures): quant_mxfp4_row, quant_nvfp4_row, "
+                    help="run one kernel alone (for ncu captures; a group_ prefix on a quant_ case runs it "
+                         "as one grouped call over A- and W-shaped tensors): quant_mxfp4_row, quant_nvfp4_row, "
                          "quant_mxfp4_col, quant_mxfp4_2d, quant_had32_row, quant_mbs_oas_row, "
                          "dequant_mxfp4_row, gemm_mxfp4, gemm_nvfp4, gemm_qsnr_mxfp4, gemm_qsnr_nvfp4")
     ap.add_argument("--rows", type=int, default=16384)
@@ -359,7 +360,7 @@ def run_ours(args, rank, world, device):
     qbytes = sum(rows[n]["bytes"] for n in qnames)
     qus = sum(rows[n]["us"] for n in qnames)
     achieved = round(qbytes / (qus * 1e-6) / 1e9, 1)
-    traffic = traffic_record("mxfp4_row_W")
+    traffic = traffic_record("mxfp4_row_AW")
     roofline = {"bound": "hbm",
                 "kernel": "k_quant_fast (TMA-fed E2M1 quantizer, statistics summed by the last CTA of each "
                           "tensor): the step's 4 grouped launches, MXFP4 / NVFP4 (with its tensor-amax "
@@ -367,9 +368,10 @@ def run_ours(args, rank, world, device):
                 "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk_src,
                 "traffic": traffic,
-                "traffic_launch": "MXFP4 on W (dram read + write per launch, from the ncu capture of the "
-                                  "16384 x 8192 case scaled by elements)",
-                "traffic_launch_algorithmic_bytes": algo_bytes(mx.MXFP4, N_OUT, K_DIM, "q"),
+                "traffic_launch": "the grouped MXFP4 launch on A and W (dram read + write per launch, from the "
+                                  "ncu capture of the 16384 x 8192 case scaled by elements)",
+                "traffic_launch_algorithmic_bytes": algo_bytes(mx.MXFP4, M_TOK, K_DIM, "q")
+                                                    + algo_bytes(mx.MXFP4, N_OUT, K_DIM, "q"),
                 "algorithmic_bytes_per_step": qbytes,
                 "by_variant_frac": {n: round(rows[n]["GB_per_s"] / pk["hbm_gbs"], 4) for n in qnames}}
 
@@ -853,10 +855,12 @@ def kernel_case(args):
             run = lambda: mx.gemm(qa, qw, out=c)
             work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
     else:
+        # group_<case>: the quantizer case as one grouped call over the layer's
+        # A-shaped and W-shaped tensors
+        group = case.startswith("group_")
+        if group:
+            case = case[len("group_"):]
         R, Cc = args.rows, args.cols
-        x = torch.randn(R, Cc, generator=g, device=dev)
-        # gradient-like cases quantize binary32 input, the others bf16
-        x = x * 1e-3 if case.endswith("_grad") else x.to(torch.bfloat16)
         cfg = {"quant_mxfp4_row": mx.MXFP4, "quant_nvfp4_row": mx.NVFP4,
                "quant_mxfp4_col": mx.Config(axis=1), "quant_mxfp4_2d": mx.Config(axis=2),
                "quant_had32_row": mx.Config(hadamard=32), "dequant_mxfp4_row": mx.MXFP4,
@@ -866,15 +870,24 @@ def kernel_case(args):
                "quant_int4_asym_grad": mx.Config(elem=mx.INT4, asymmetric=1, rule=mx.RULE_CEIL),
                "quant_e3m0_ceil_grad": mx.Config(elem=mx.E3M0, rule=mx.RULE_CEIL),
                "quant_nvfp4_mse_row": mx.Config(block=16, scale_fmt=1, rule=mx.RULE_MSE, tensor_scale=1)}[case]
-        q = mx.quantize(x, cfg, stats=not args.no_stats)
-        if case.startswith("dequant"):
-            out = torch.empty(R, Cc, dtype=torch.bfloat16, device=dev)
-            run = lambda: mx.dequantize(q, out=out)
-            kind = "d"
+        if group:
+            xs = [torch.randn(r, K_DIM, generator=g, device=dev).to(torch.bfloat16) for r in (M_TOK, N_OUT)]
+            qs = mx.quantize_group(xs, cfg, stats=not args.no_stats)
+            run = lambda: mx.quantize_group(xs, cfg, outs=qs)
+            nbytes = sum(algo_bytes(cfg, *t.shape, "q") for t in xs)
         else:
-            run = lambda: mx.quantize(x, cfg, out=q)
-            kind = "q"
-        nbytes = algo_bytes(cfg, R, Cc, kind, in_bytes=x.element_size())
+            x = torch.randn(R, Cc, generator=g, device=dev)
+            # gradient-like cases quantize binary32 input, the others bf16
+            x = x * 1e-3 if case.endswith("_grad") else x.to(torch.bfloat16)
+            q = mx.quantize(x, cfg, stats=not args.no_stats)
+            if case.startswith("dequant"):
+                out = torch.empty(R, Cc, dtype=torch.bfloat16, device=dev)
+                run = lambda: mx.dequantize(q, out=out)
+                kind = "d"
+            else:
+                run = lambda: mx.quantize(x, cfg, out=q)
+                kind = "q"
+            nbytes = algo_bytes(cfg, R, Cc, kind, in_bytes=x.element_size())
         work, unit = nbytes / 1e9, "GB/s"
         res["algorithmic_bytes"] = nbytes
     run()
