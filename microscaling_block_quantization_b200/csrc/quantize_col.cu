@@ -659,13 +659,13 @@ __device__ __forceinline__ uint32_t cvt_e2m1x4(const float v[4])
     return r;
 }
 
-template <int AXIS, bool STATS, bool NEAR>
+template <int AXIS, bool STATS, bool NEAR, int RB>
 __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
 {
+    // RB: rows of a block (the column block size, or 32 for 2D tiles)
     constexpr int NS = (AXIS == AX_COL) ? 4 : 1;          // blocks a lane holds per tile
     extern __shared__ uint4 smem[];
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int RB = (AXIS == AX_2D) ? 32 : p.block;
     uint8_t *const bufs = reinterpret_cast<uint8_t *>(smem) + (size_t)w * 2 * kColxBufBytes;
     const int64_t ngc = (p.cols + kColxCols - 1) / kColxCols;
     const int64_t nitems = (p.rows / RB) * ngc;
@@ -699,6 +699,7 @@ __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
     // the tile's RB rows x 256 bytes as 16-byte copies, RB / 2 per lane
     auto issue = [&](int64_t item, uint8_t *buf) {
         const int64_t rg = item / ngc, cg = item - rg * ngc;
+#pragma unroll
         for (int k = 0; k < RB / 2; ++k) {
             const int f = k * 32 + lane, r = f >> 4, ch = f & 15;
             const int64_t cb = cg * (kColxCols * 2) + ch * 16;
@@ -729,7 +730,7 @@ __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
 
         // column statistics on the packed words (two chains per word)
         uint32_t am[4] = {0u, 0u, 0u, 0u}, mn[4] = {0x7f807f80u, 0x7f807f80u, 0x7f807f80u, 0x7f807f80u};
-#pragma unroll 4
+#pragma unroll
         for (int r = 0; r < RB; r += 2) {
             const uint2 u0 = b[r * 32], u1 = b[(r + 1) * 32];
             am[0] = bfx_absmax(am[0], u0.x);
@@ -806,7 +807,7 @@ __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
         }
         int qz = 0;
         uint8_t *const codes = static_cast<uint8_t *>(p.codes) + (r0 * p.cols + c0) / 2;
-#pragma unroll 4
+#pragma unroll 8
         for (int r = 0; r < RB; ++r) {
             const uint2 u = b[r * 32];
             const uint32_t v[2] = {u.x, u.y};
@@ -863,6 +864,7 @@ __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
             for (int j = 0; j < 4; ++j) {
                 int xz = 0;
                 if (mabs[j] == 0.0f)
+#pragma unroll 1
                     for (int r = 0; r < RB; ++r) {
                         const uint2 u = b[r * 32];
                         const uint32_t vv = (j >> 1) ? u.y : u.x;
@@ -878,13 +880,12 @@ __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
     finish_launch(p, acc);
 }
 
-template <int AXIS, bool STATS, bool NEAR>
+template <int AXIS, bool STATS, bool NEAR, int RB>
 int launch_colx_k(const QParams &p, cudaStream_t st, int *grid_out)
 {
-    auto k = k_quant_colx<AXIS, STATS, NEAR>;
+    auto k = k_quant_colx<AXIS, STATS, NEAR, RB>;
     const size_t smem = (size_t)kColxWarps * 2 * kColxBufBytes;
     const int occ = cached_occupancy(reinterpret_cast<const void *>(k), kColxThreads, smem);
-    const int RB = (AXIS == AX_2D) ? 32 : p.block;
     const int64_t items = (p.rows / RB) * ((p.cols + kColxCols - 1) / kColxCols);
     int64_t g = (int64_t)device_sm_count() * occ;
     const int64_t need = (items + kColxWarps - 1) / kColxWarps;
@@ -896,13 +897,30 @@ int launch_colx_k(const QParams &p, cudaStream_t st, int *grid_out)
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
-template <int AXIS>
-int launch_colx(const QParams &p, cudaStream_t st, int *grid_out)
+template <int AXIS, int RB>
+int launch_colx_rb(const QParams &p, cudaStream_t st, int *grid_out)
 {
     const bool near = p.sd.fmt != S_E8M0 && p.sd.rule == R_NEAREST;
     if (p.partials)
-        return near ? launch_colx_k<AXIS, true, true>(p, st, grid_out) : launch_colx_k<AXIS, true, false>(p, st, grid_out);
-    return near ? launch_colx_k<AXIS, false, true>(p, st, grid_out) : launch_colx_k<AXIS, false, false>(p, st, grid_out);
+        return near ? launch_colx_k<AXIS, true, true, RB>(p, st, grid_out)
+                    : launch_colx_k<AXIS, true, false, RB>(p, st, grid_out);
+    return near ? launch_colx_k<AXIS, false, true, RB>(p, st, grid_out)
+                : launch_colx_k<AXIS, false, false, RB>(p, st, grid_out);
+}
+
+template <int AXIS>
+int launch_colx(const QParams &p, cudaStream_t st, int *grid_out)
+{
+    if constexpr (AXIS == AX_2D) {
+        return launch_colx_rb<AXIS, 32>(p, st, grid_out);
+    } else {
+        switch (p.block) {
+        case 8: return launch_colx_rb<AXIS, 8>(p, st, grid_out);
+        case 16: return launch_colx_rb<AXIS, 16>(p, st, grid_out);
+        case 32: return launch_colx_rb<AXIS, 32>(p, st, grid_out);
+        default: return -1;
+        }
+    }
 }
 
 template <typename K>
