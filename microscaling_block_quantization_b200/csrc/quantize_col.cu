@@ -646,19 +646,20 @@ __device__ __forceinline__ float2 bfx_scale2(uint32_t w, uint32_t k0, uint32_t k
         : "=f"(a), "=f"(b) : "r"(w), "r"(k0), "r"(k1));
     return make_float2(a, b);
 }
-// four binary32 values -> four E2M1 nibbles (the first in bits 0..3)
-__device__ __forceinline__ uint32_t cvt_e2m1x4(const float v[4])
+// two rows of four binary32 values -> eight E2M1 nibbles: the first row in
+// bits 0..15 (its first value in bits 0..3), the second in bits 16..31
+__device__ __forceinline__ uint32_t cvt_e2m1x4x2(const float v[8])
 {
     uint32_t r;
-    asm("{\n\t.reg .b8 b0, b1;\n\t.reg .b16 h;\n\t"
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
         "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
         "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-        "mov.b16 h, {b0, b1};\n\t"
-        "cvt.u32.u16 %0, h;\n\t}"
-        : "=r"(r) : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]));
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r) : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
     return r;
 }
-
 template <int AXIS, bool STATS, bool NEAR, int RB>
 __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
 {
@@ -807,42 +808,54 @@ __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
         }
         int qz = 0;
         uint8_t *const codes = static_cast<uint8_t *>(p.codes) + (r0 * p.cols + c0) / 2;
-#pragma unroll 8
-        for (int r = 0; r < RB; ++r) {
-            const uint2 u = b[r * 32];
-            const uint32_t v[2] = {u.x, u.y};
-            float s4[4];
+        const uint32_t zmask2 = zmask | (zmask << 16);
+        // two rows a step: their eight codes share one word (row r in the low
+        // half, row r + 1 in the high half), one mask, one decode and one
+        // zero count
+#pragma unroll 4
+        for (int r = 0; r < RB; r += 2) {
+            float s8[8];
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                float2 sv = bfx_scale2(v[i], kb[2 * i], kb[2 * i + 1]);
-                if (NEAR) {
-                    if (STATS) sx2[i] = __ffma2_rn(sv, sv, sx2[i]);       // reference y
-                    sv = __fmul2_rn(sv, make_float2(inv[2 * i], inv[2 * i + 1]));
-                }
-                s4[2 * i] = sv.x;
-                s4[2 * i + 1] = sv.y;
-            }
-            const uint32_t word = cvt_e2m1x4(s4) & zmask;
-            if (ok) *reinterpret_cast<uint16_t *>(codes + (int64_t)r * (p.cols / 2)) = (uint16_t)word;
-            if (STATS) {
-                uint32_t h0, h1;
-                asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
-                    "mov.b32 {c0, c1, c2, c3}, %2;\n\t"
-                    "cvt.rn.f16x2.e2m1x2 %0, c0;\n\t"
-                    "cvt.rn.f16x2.e2m1x2 %1, c1;\n\t}"
-                    : "=r"(h0), "=r"(h1) : "r"(word));
-                const uint32_t h[2] = {h0, h1};
+            for (int rr = 0; rr < 2; ++rr) {
+                const uint2 u = b[(r + rr) * 32];
+                const uint32_t v[2] = {u.x, u.y};
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
-                    const float2 d = sub_f16x2_from(s4[2 * i], s4[2 * i + 1], h[i]);   // s - q
+                    float2 sv = bfx_scale2(v[i], kb[2 * i], kb[2 * i + 1]);
+                    if (NEAR) {
+                        if (STATS) sx2[i] = __ffma2_rn(sv, sv, sx2[i]);       // reference y
+                        sv = __fmul2_rn(sv, make_float2(inv[2 * i], inv[2 * i + 1]));
+                    }
+                    s8[4 * rr + 2 * i] = sv.x;
+                    s8[4 * rr + 2 * i + 1] = sv.y;
+                }
+            }
+            const uint32_t word = cvt_e2m1x4x2(s8) & zmask2;
+            if (ok) {
+                *reinterpret_cast<uint16_t *>(codes + (int64_t)r * (p.cols / 2)) = (uint16_t)word;
+                *reinterpret_cast<uint16_t *>(codes + (int64_t)(r + 1) * (p.cols / 2)) = (uint16_t)(word >> 16);
+            }
+            if (STATS) {
+                uint32_t h[4];
+                asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
+                    "mov.b32 {c0, c1, c2, c3}, %4;\n\t"
+                    "cvt.rn.f16x2.e2m1x2 %0, c0;\n\t"
+                    "cvt.rn.f16x2.e2m1x2 %1, c1;\n\t"
+                    "cvt.rn.f16x2.e2m1x2 %2, c2;\n\t"
+                    "cvt.rn.f16x2.e2m1x2 %3, c3;\n\t}"
+                    : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(word));
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i = e & 1;                   // column pair
+                    const float2 d = sub_f16x2_from(s8[2 * e], s8[2 * e + 1], h[e]);   // s - q
                     re2[i] = __ffma2_rn(d, d, re2[i]);
                     rb2[i] = __fadd2_rn(rb2[i], d);
                     if (!NEAR) {
-                        const float2 sv = make_float2(s4[2 * i], s4[2 * i + 1]);
+                        const float2 sv = make_float2(s8[2 * e], s8[2 * e + 1]);
                         sx2[i] = __ffma2_rn(sv, sv, sx2[i]);                 // y = R s
                     }
                 }
-                qz += 4 - __popc(((word & 0x7777u) + 0x7777u) & 0x8888u);
+                qz += 8 - __popc(((word & 0x77777777u) + 0x77777777u) & 0x88888888u);
             }
         }
         if (STATS && ok) {
