@@ -265,12 +265,13 @@ typedef struct {
  * statistics: the results are those of n mx_quantize calls (mx_hadamard_quantize
  * without `rotated` when cfg->hadamard), bit for bit ([MXFP4-OAS] Sec.2: every
  * block, and every tensor, is quantized on its own).  Shapes may differ.
- *   For row-axis E2M1 round-to-nearest-even symmetric configurations (not the
- *   MSE rule; with a rotation or a macro scale, blocks of 16 or 32) the
- *   tensors share one quantizer launch, up to 4 tensors a launch, the CTAs
- *   split among the tensors in proportion to their sizes; with a computed
- *   tensor scale one tensor-amax launch comes before it.  Other
- *   configurations run as n calls in order.
+ *   For E2M1 round-to-nearest-even symmetric configurations (not the MSE
+ *   rule) on the row axis (with a rotation or a macro scale, blocks of 16 or
+ *   32), and on the column axis or 2D tiles with bf16 input (no rotation, no
+ *   macro scale), the tensors share one quantizer launch, up to 4 tensors a
+ *   launch, the CTAs split among the tensors in proportion to their sizes;
+ *   with a computed tensor scale one tensor-amax launch comes before it.
+ *   Other configurations run as n calls in order.
  *   Items that need a workspace (stats != NULL, MX_TS_COMPUTE, MX_TS_AMAX)
  *   must each have their own (MX_ERR_INVALID when two overlap).  Every item is
  *   checked before anything is queued; a failing item fails the call with

@@ -282,6 +282,14 @@ bool groupable(const mx_config *cfg)
            ((!cfg->macro_block && !cfg->hadamard) || cfg->block == 16 || cfg->block == 32);
 }
 
+// the configurations launch_quantize_col sends to the double-buffered column /
+// 2D quantizer
+bool col_groupable(const mx_config *cfg, int32_t x_dtype)
+{
+    return cfg->axis != MX_AXIS_ROW && x_dtype == MX_DT_BF16 && fast_elements(cfg) && !cfg->macro_block &&
+           !cfg->hadamard;
+}
+
 }  // namespace
 
 extern "C" {
@@ -360,7 +368,8 @@ int mx_quantize_group(const mx_config *cfg, int32_t x_dtype, const mx_quantize_i
             if (a0 < b0 + (uintptr_t)kWorkspaceBytes && b0 < a0 + (uintptr_t)kWorkspaceBytes) rc = MX_ERR_INVALID;
         }
     const int in_fp32 = x_dtype == MX_DT_FP32;
-    if (rc == MX_OK && !groupable(cfg)) {
+    const bool col = col_groupable(cfg, x_dtype);
+    if (rc == MX_OK && !groupable(cfg) && !col) {
         // other configurations: one call per tensor, in order
         for (int i = 0; i < n && rc == MX_OK; ++i) {
             const mx_quantize_item &it = items[i];
@@ -389,7 +398,11 @@ int mx_quantize_group(const mx_config *cfg, int32_t x_dtype, const mx_quantize_i
                         rc = MX_ERR_CUDA;
                     }
                 }
-                if (rc == MX_OK && launch_quantize_fast_group(chunk, m, in_fp32, st)) rc = MX_ERR_CUDA;
+                if (rc == MX_OK) {
+                    const int e = col ? launch_quantize_colx_group(chunk, m, cfg->axis, st)
+                                      : launch_quantize_fast_group(chunk, m, in_fp32, st);
+                    if (e) rc = MX_ERR_CUDA;
+                }
                 m = 0;
             }
         }

@@ -125,9 +125,35 @@ int launch_amax_col(const QParams &p, int in_fp32, cudaStream_t st);
 // E2M1 round-to-nearest-even, symmetric, row axis, no macro scale, rotation
 // or rotated output: the TMA-fed persistent quantizer.
 int launch_quantize_fast(const QParams &p, int in_fp32, cudaStream_t st, int *grid_out);
+// CTAs of a grouped launch over n tensors with work[i] units each (a CTA
+// takes at least one unit): one CTA per tensor, then one at a time to the
+// tensor with the most units per CTA; cta0 gets the prefix (n + 1 entries)
+inline void split_ctas(const uint64_t *work, int n, uint64_t total, uint32_t *cta0)
+{
+    uint64_t c[kFastGroupMax], sum = 0;
+    for (int i = 0; i < n; ++i) {
+        c[i] = 1;
+        sum += work[i];
+    }
+    if (total > sum) total = sum;
+    for (uint64_t k = n; k < total; ++k) {
+        int best = -1;
+        for (int i = 0; i < n; ++i)
+            if (c[i] < work[i] && (best < 0 || work[i] * c[best] > work[best] * c[i])) best = i;
+        if (best < 0) break;
+        ++c[best];
+    }
+    cta0[0] = 0;
+    for (int i = 0; i < n; ++i) cta0[i + 1] = cta0[i] + (uint32_t)c[i];
+}
+
 // one launch over ps[0..n) (n <= kFastGroupMax, one configuration, every tensor
 // non-empty and eligible for launch_quantize_fast)
 int launch_quantize_fast_group(const QParams *ps, int n, int in_fp32, cudaStream_t st);
+// one launch of the double-buffered column / 2D quantizer over ps[0..n)
+// (bf16 input, E2M1 round-to-nearest-even, symmetric, no macro scale, no
+// rotation; n <= kFastGroupMax, every tensor non-empty)
+int launch_quantize_colx_group(const QParams *ps, int n, int axis, cudaStream_t st);
 // the tensor-amax pre-pass of ps[0..n) without rotation, one launch
 int launch_tensor_amax_group(const QParams *ps, int n, int in_fp32, cudaStream_t st);
 // Other element types / rounding modes / offsets, row axis, blocks of 32, no

@@ -7,6 +7,8 @@
 // every lane works down its own CPT columns: column axis -> CPT blocks per
 // lane; 2D -> one 32 x 32 block per 32 / CPT lanes.  Loads and stores stay
 // coalesced along rows; the reduction runs along columns out of shared memory.
+#include <string.h>
+
 #include "quant_common.cuh"
 
 namespace mxk {
@@ -660,41 +662,60 @@ __device__ __forceinline__ uint32_t cvt_e2m1x4x2(const float v[8])
         : "=r"(r) : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
     return r;
 }
+// A launch over up to kFastGroupMax tensors of one configuration: the CTAs
+// are split among the tensors (cta0 prefix), every CTA works on one tensor;
+// p[0] also carries the shared configuration.
+struct ColxGroup {
+    QParams p[kFastGroupMax];
+    uint32_t cta0[kFastGroupMax + 1];
+    int n;
+};
+
 template <int AXIS, bool STATS, bool NEAR, int RB>
-__global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
+__global__ void __launch_bounds__(kColxThreads) k_quant_colx(const __grid_constant__ ColxGroup g)
 {
     // RB: rows of a block (the column block size, or 32 for 2D tiles)
     constexpr int NS = (AXIS == AX_COL) ? 4 : 1;          // blocks a lane holds per tile
     extern __shared__ uint4 smem[];
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // this CTA's tensor, and its place among the tensor's CTAs
+    int item = 0;
+    while (item + 1 < g.n && blockIdx.x >= g.cta0[item + 1]) ++item;
+    const QParams &pc = g.p[0];
+    const QParams &p = g.p[item];
+    const uint32_t cta = blockIdx.x - g.cta0[item], ncta = g.cta0[item + 1] - g.cta0[item];
     uint8_t *const bufs = reinterpret_cast<uint8_t *>(smem) + (size_t)w * 2 * kColxBufBytes;
-    const int64_t ngc = (p.cols + kColxCols - 1) / kColxCols;
-    const int64_t nitems = (p.rows / RB) * ngc;
-    const int64_t gw = (int64_t)blockIdx.x * kColxWarps + w, nw = (int64_t)gridDim.x * kColxWarps;
-    const float sT = launch_tensor_scale(p);
+    // the tensor's shape and outputs, read once from the launch parameters
+    const int64_t cols = p.cols, rows = p.rows;
+    uint8_t *const codes0 = static_cast<uint8_t *>(p.codes);
+    uint8_t *const scales0 = p.scales;
+    const int64_t ngc = (cols + kColxCols - 1) / kColxCols;
+    const int64_t nitems = (rows / RB) * ngc;
+    const int64_t gw = (int64_t)cta * kColxWarps + w, nw = (int64_t)ncta * kColxWarps;
+    const float sT = launch_tensor_scale(p, cta == 0);
     // nearest scales: s_b s_T and its reciprocal for every scale code, once per CTA
     __shared__ float2 near_tab[NEAR ? 256 : 1];
     if constexpr (NEAR)
         for (int c = threadIdx.x; c < 256; c += blockDim.x) {
-            const float d = __fmul_rn(ue_value(p.sd, (uint32_t)c), sT);
-            near_tab[c] = c < p.sd.ue_nan_code ? make_float2(d, __fdiv_rn(1.0f, d))
+            const float d = __fmul_rn(ue_value(pc.sd, (uint32_t)c), sT);
+            near_tab[c] = c < pc.sd.ue_nan_code ? make_float2(d, __fdiv_rn(1.0f, d))
                                                : make_float2(__uint_as_float(0x7fc00000u), 0.0f);
         }
     __syncthreads();
     NearScale ns;
-    ns.maxv = p.ed.maxv;
-    ns.r_max = __fdiv_rn(1.0f, p.ed.maxv);
+    ns.maxv = pc.ed.maxv;
+    ns.r_max = __fdiv_rn(1.0f, pc.ed.maxv);
     ns.sT = sT;
     ns.r_T = (sT >= 0x1p-125f && sT <= 0x1p125f) ? __fdiv_rn(1.0f, sT) : 0.0f;
     {
-        const float ms = __fmul_rn(p.ed.maxv, sT);
+        const float ms = __fmul_rn(pc.ed.maxv, sT);
         ns.c = (ms >= 0x1p-125f && ms <= 0x1p125f) ? __fdiv_rn(1.0f, ms) : 0.0f;
     }
     ns.tab = near_tab;
-    const bool e8m0 = !NEAR && p.sd.fmt == S_E8M0;
-    const float thr_m = e8m0_threshold(p.ed, p.sd);
+    const bool e8m0 = !NEAR && pc.sd.fmt == S_E8M0;
+    const float thr_m = e8m0_threshold(pc.ed, pc.sd);
     const uint8_t *const xb = static_cast<const uint8_t *>(p.x);
-    const int64_t pitch = p.cols * 2;                        // bytes per row
+    const int64_t pitch = cols * 2;                          // bytes per row
     Acc acc = {0, 0, 0, 0, 0};
 
     // the tile's RB rows x 256 bytes as 16-byte copies, RB / 2 per lane
@@ -726,7 +747,7 @@ __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
         __syncwarp();                    // every lane's copies of this tile have landed
         const int64_t rg = item / ngc, cg = item - rg * ngc;
         const int64_t c0 = cg * kColxCols + lane * 4;
-        const bool ok = c0 < p.cols;
+        const bool ok = c0 < cols;
         const int64_t r0 = rg * RB;
 
         // column statistics on the packed words (two chains per word)
@@ -762,25 +783,25 @@ __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int bad = !(a[j] <= FLT_MAX);
-                bs[j] = NEAR ? near_block_scale(p.sd, ns, bad ? 0.0f : a[j], bad)
-                      : e8m0 ? e8m0_block_scale(bad ? 0.0f : a[j], bad, p.ed.emax, thr_m)
-                             : block_scale(p.ed, p.sd, bad ? 0.0f : a[j], bad, sT);
+                bs[j] = NEAR ? near_block_scale(pc.sd, ns, bad ? 0.0f : a[j], bad)
+                      : e8m0 ? e8m0_block_scale(bad ? 0.0f : a[j], bad, pc.ed.emax, thr_m)
+                             : block_scale(pc.ed, pc.sd, bad ? 0.0f : a[j], bad, sT);
             }
         } else {
             float m = fmax_nan(fmax_nan(a[0], a[1]), fmax_nan(a[2], a[3]));
             int bad = !(m <= FLT_MAX);
             m = grp_max(bad ? 0.0f : m, 8);
             bad = grp_or(bad, 8);
-            bs[0] = NEAR ? near_block_scale(p.sd, ns, m, bad)
-                  : e8m0 ? e8m0_block_scale(m, bad, p.ed.emax, thr_m)
-                         : block_scale(p.ed, p.sd, m, bad, sT);
+            bs[0] = NEAR ? near_block_scale(pc.sd, ns, m, bad)
+                  : e8m0 ? e8m0_block_scale(m, bad, pc.ed.emax, thr_m)
+                         : block_scale(pc.ed, pc.sd, m, bad, sT);
         }
         if (ok) {
             if constexpr (AXIS == AX_COL) {
                 const uint32_t w0 = bs[0].code | (bs[1].code << 8) | (bs[2].code << 16) | (bs[3].code << 24);
-                *reinterpret_cast<uint32_t *>(p.scales + (r0 / RB) * p.cols + c0) = w0;
+                *reinterpret_cast<uint32_t *>(scales0 + (r0 / RB) * cols + c0) = w0;
             } else if ((lane & 7) == 0) {
-                p.scales[(r0 / 32) * (p.cols / 32) + c0 / 32] = (uint8_t)bs[0].code;
+                scales0[(r0 / 32) * (cols / 32) + c0 / 32] = (uint8_t)bs[0].code;
             }
         }
 
@@ -807,7 +828,7 @@ __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
             sx2[i] = re2[i];
         }
         int qz = 0;
-        uint8_t *const codes = static_cast<uint8_t *>(p.codes) + (r0 * p.cols + c0) / 2;
+        uint8_t *const codes = codes0 + (r0 * cols + c0) / 2;
         const uint32_t zmask2 = zmask | (zmask << 16);
         // two rows a step: their eight codes share one word (row r in the low
         // half, row r + 1 in the high half), one mask, one decode and one
@@ -832,8 +853,8 @@ __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
             }
             const uint32_t word = cvt_e2m1x4x2(s8) & zmask2;
             if (ok) {
-                *reinterpret_cast<uint16_t *>(codes + (int64_t)r * (p.cols / 2)) = (uint16_t)word;
-                *reinterpret_cast<uint16_t *>(codes + (int64_t)(r + 1) * (p.cols / 2)) = (uint16_t)(word >> 16);
+                *reinterpret_cast<uint16_t *>(codes + (int64_t)r * (cols / 2)) = (uint16_t)word;
+                *reinterpret_cast<uint16_t *>(codes + (int64_t)(r + 1) * (cols / 2)) = (uint16_t)(word >> 16);
             }
             if (STATS) {
                 uint32_t h[4];
@@ -890,47 +911,54 @@ __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const QParams p)
             acc.ftz += (double)(qz - nanz);
         }
     }
-    finish_launch(p, acc);
+    finish_launch(p, acc, cta, ncta);
 }
 
 template <int AXIS, bool STATS, bool NEAR, int RB>
-int launch_colx_k(const QParams &p, cudaStream_t st, int *grid_out)
+int launch_colx_k(const QParams *ps, int n, cudaStream_t st)
 {
     auto k = k_quant_colx<AXIS, STATS, NEAR, RB>;
     const size_t smem = (size_t)kColxWarps * 2 * kColxBufBytes;
     const int occ = cached_occupancy(reinterpret_cast<const void *>(k), kColxThreads, smem);
-    const int64_t items = (p.rows / RB) * ((p.cols + kColxCols - 1) / kColxCols);
-    int64_t g = (int64_t)device_sm_count() * occ;
-    const int64_t need = (items + kColxWarps - 1) / kColxWarps;
-    if (need < g) g = need;
-    if (g < 1) g = 1;
-    if (g > kMaxPartials) g = kMaxPartials;
-    k<<<(unsigned)g, kColxThreads, smem, st>>>(p);
-    if (grid_out) *grid_out = (int)g;
+    ColxGroup g;
+    memset(&g, 0, sizeof(g));
+    uint64_t need[kFastGroupMax];
+    for (int i = 0; i < n; ++i) {
+        g.p[i] = ps[i];
+        const int64_t items = (ps[i].rows / RB) * ((ps[i].cols + kColxCols - 1) / kColxCols);
+        need[i] = (uint64_t)((items + kColxWarps - 1) / kColxWarps);     // CTAs with work
+    }
+    g.n = n;
+    uint64_t total = (uint64_t)device_sm_count() * occ;
+    if (total > (uint64_t)kMaxPartials) total = kMaxPartials;
+    if (total < (uint64_t)n) total = n;
+    split_ctas(need, n, total, g.cta0);
+    k<<<g.cta0[n], kColxThreads, smem, st>>>(g);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
 template <int AXIS, int RB>
-int launch_colx_rb(const QParams &p, cudaStream_t st, int *grid_out)
+int launch_colx_rb(const QParams *ps, int n, cudaStream_t st)
 {
+    const QParams &p = ps[0];
     const bool near = p.sd.fmt != S_E8M0 && p.sd.rule == R_NEAREST;
-    if (p.partials)
-        return near ? launch_colx_k<AXIS, true, true, RB>(p, st, grid_out)
-                    : launch_colx_k<AXIS, true, false, RB>(p, st, grid_out);
-    return near ? launch_colx_k<AXIS, false, true, RB>(p, st, grid_out)
-                : launch_colx_k<AXIS, false, false, RB>(p, st, grid_out);
+    bool stats = false;
+    for (int i = 0; i < n; ++i) stats = stats || ps[i].partials != nullptr;
+    if (stats)
+        return near ? launch_colx_k<AXIS, true, true, RB>(ps, n, st) : launch_colx_k<AXIS, true, false, RB>(ps, n, st);
+    return near ? launch_colx_k<AXIS, false, true, RB>(ps, n, st) : launch_colx_k<AXIS, false, false, RB>(ps, n, st);
 }
 
 template <int AXIS>
-int launch_colx(const QParams &p, cudaStream_t st, int *grid_out)
+int launch_colx(const QParams *ps, int n, cudaStream_t st)
 {
     if constexpr (AXIS == AX_2D) {
-        return launch_colx_rb<AXIS, 32>(p, st, grid_out);
+        return launch_colx_rb<AXIS, 32>(ps, n, st);
     } else {
-        switch (p.block) {
-        case 8: return launch_colx_rb<AXIS, 8>(p, st, grid_out);
-        case 16: return launch_colx_rb<AXIS, 16>(p, st, grid_out);
-        case 32: return launch_colx_rb<AXIS, 32>(p, st, grid_out);
+        switch (ps[0].block) {
+        case 8: return launch_colx_rb<AXIS, 8>(ps, n, st);
+        case 16: return launch_colx_rb<AXIS, 16>(ps, n, st);
+        case 32: return launch_colx_rb<AXIS, 32>(ps, n, st);
         default: return -1;
         }
     }
@@ -969,7 +997,10 @@ int launch_axis(const QParams &p, int fast, cudaStream_t st, int *grid_out)
     }
     if constexpr (sizeof(InT) == 2) {
         // E2M1 nearest-even without a macro scale: the double-buffered kernel
-        if (fast && !p.mbs && p.ed.elem == 0) return launch_colx<AXIS>(p, st, grid_out);
+        if (fast && !p.mbs && p.ed.elem == 0) {
+            if (grid_out) *grid_out = 0;
+            return launch_colx<AXIS>(&p, 1, st);
+        }
         if (p.ed.code_bits == 4) {
             if (fast) return launch_col_k<InT, 8, AXIS, true, false>(p, st, grid_out);
             return launch_col_k<InT, 8, AXIS, false, false>(p, st, grid_out);
@@ -980,6 +1011,12 @@ int launch_axis(const QParams &p, int fast, cudaStream_t st, int *grid_out)
 }
 
 }  // namespace
+
+int launch_quantize_colx_group(const QParams *ps, int n, int axis, cudaStream_t st)
+{
+    if (n < 1 || n > kFastGroupMax) return -1;
+    return axis == AX_COL ? launch_colx<AX_COL>(ps, n, st) : launch_colx<AX_2D>(ps, n, st);
+}
 
 int launch_quantize_col(const QParams &p, int axis, int in_fp32, int fast, cudaStream_t st,
                         int *grid_out)

@@ -554,27 +554,6 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
     finish_launch(p, acc, cta, ncta);
 }
 
-// CTAs of a grouped launch: one per tensor, then one at a time to the tensor
-// with the most tiles per CTA (as long as it has more tiles than CTAs)
-void split_ctas(const uint64_t *tiles, int n, uint64_t total, uint32_t *cta0)
-{
-    uint64_t c[kFastGroupMax], sum = 0;
-    for (int i = 0; i < n; ++i) {
-        c[i] = 1;
-        sum += tiles[i];
-    }
-    if (total > sum) total = sum;
-    for (uint64_t k = n; k < total; ++k) {
-        int best = -1;
-        for (int i = 0; i < n; ++i)
-            if (c[i] < tiles[i] && (best < 0 || tiles[i] * c[best] > tiles[best] * c[i])) best = i;
-        if (best < 0) break;
-        ++c[best];
-    }
-    cta0[0] = 0;
-    for (int i = 0; i < n; ++i) cta0[i + 1] = cta0[i] + (uint32_t)c[i];
-}
-
 template <typename InT, int B, bool STATS, int HADN, bool MBS, bool NEAR>
 int launch_fast_b(const QParams *ps, int n, cudaStream_t st)
 {

@@ -40,8 +40,12 @@ def _cfgs(mx):
         "ue5m3_b256": mx.Config(block=256, scale_fmt=2, rule=3),
         "e8m0_b8": mx.Config(block=8),
         "ceil_sf_gemm": mx.Config(rule=1, sf_layout=1),       # scales in the tcgen05 chunk layout
-        # configurations outside the shared launch: one call per tensor
         "col": mx.Config(axis=1),
+        "col_b8": mx.Config(axis=1, block=8),
+        "col_nvfp4": mx.Config(axis=1, block=16, scale_fmt=1, rule=3, tensor_scale=1),
+        "2d": mx.Config(axis=2),
+        # configurations outside the shared launch: one call per tensor
+        "col_mbs": mx.Config(axis=1, macro_block=128),
         "int4_asym": mx.Config(elem=mx.INT4, asymmetric=1, rule=1),
         "nvfp4_mse": mx.Config(block=16, scale_fmt=1, rule=4, tensor_scale=1),
     }
@@ -51,8 +55,10 @@ def _tensors(name, dtype=torch.bfloat16):
     """Tensors of different shapes and scales (the tensor amaxes differ)."""
     if name == "ceil_sf_gemm":
         shapes = [(128, 512), (256, 256), (128, 1024)]
-    elif name == "col":
-        shapes = [(64, 256), (32, 512), (96, 128)]
+    elif name.startswith("col") or name == "2d":
+        # column blocks need rows in multiples of the block (and of 128 with MBS),
+        # 2D tiles multiples of 32
+        shapes = [(128, 256), (32, 512), (256, 160), (96, 128)] if name != "col_mbs" else [(128, 256), (256, 512)]
     else:
         shapes = [(40, 768), (264, 512), (1, 256), (96, 1280)]
     out = []
@@ -63,7 +69,8 @@ def _tensors(name, dtype=torch.bfloat16):
 
 
 @pytest.mark.parametrize("name", ["mxfp4", "nvfp4", "had32", "nvfp4_had16", "mbs_oas", "mbs_b16",
-                                  "ue4m3_b64_ts", "ue5m3_b256", "e8m0_b8", "col", "int4_asym", "nvfp4_mse"])
+                                  "ue4m3_b64_ts", "ue5m3_b256", "e8m0_b8", "col", "col_b8", "col_nvfp4", "2d",
+                                  "col_mbs", "int4_asym", "nvfp4_mse"])
 def test_group_matches_oracle(mx, orc, name):
     cfg = _cfgs(mx)[name]
     xs = _tensors(name)
@@ -93,7 +100,7 @@ def test_group_of_six_with_an_empty_tensor(mx, orc, dtype):
         run_case(mx, orc, x, cfg, check_stats=(i != 3), want_rotated=False, q=q)
 
 
-@pytest.mark.parametrize("name", ["mxfp4", "nvfp4", "had32", "mbs_oas", "ceil_sf_gemm"])
+@pytest.mark.parametrize("name", ["mxfp4", "nvfp4", "had32", "mbs_oas", "ceil_sf_gemm", "col", "col_nvfp4", "2d"])
 def test_group_equals_single_calls(mx, name):
     """The same codes, scales (canonical, or the tcgen05 chunk layout the
     oracle does not produce), macro scales and tensor scales as one call per
