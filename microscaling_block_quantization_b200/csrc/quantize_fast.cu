@@ -219,6 +219,11 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
     const QParams &p = g.p[item];
     const uint32_t cta = blockIdx.x - g.cta0[item], ncta = g.cta0[item + 1] - g.cta0[item];
     const uint32_t nch = (uint32_t)(p.rows * p.cols / 32);
+    // the tensor's outputs, read once from the launch parameters
+    uint4 *const codes0 = static_cast<uint4 *>(p.codes);
+    uint8_t *const scales0 = p.scales;
+    uint8_t *const macro0 = p.macro;
+    const int64_t cols = p.cols;
     const uint32_t ntiles = (nch + kConsumers - 1) / kConsumers;
     pdl_trigger();
     if (threadIdx.x == 0) ring.init();
@@ -269,7 +274,7 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
         const float hc = HADN ? hadamard_scale(HADN) : 1.0f;
         const bool e8m0 = !NEAR && pc.sd.fmt == S_E8M0;
         const float thr_m = e8m0_threshold(pc.ed, pc.sd);
-        const uint32_t S = (uint32_t)(p.cols / B);
+        const uint32_t S = (uint32_t)(cols / B);
         const int t = threadIdx.x;
         uint32_t i = 0;
         for (uint32_t tile = cta; tile < ntiles; tile += ncta, ++i) {
@@ -298,7 +303,7 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
                 const float2 mt = macro_tab[mcode];
                 sm = mt.x;
                 const float invm = mt.y;
-                if ((t & 3) == 0 && tile * kConsumers + t < nch) p.macro[(tile * kConsumers + t) >> 2] = (uint8_t)mcode;
+                if ((t & 3) == 0 && tile * kConsumers + t < nch) macro0[(tile * kConsumers + t) >> 2] = (uint8_t)mcode;
                 const float2 invm2 = make_float2(invm, invm);
 #pragma unroll
                 for (int j = 0; j < 32; j += 2) {
@@ -346,7 +351,7 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
                     const float2 mt = macro_tab[mcode];
                     sm = mt.x;
                     invm = mt.y;
-                    if ((t & 3) == 0 && ok) p.macro[c >> 2] = (uint8_t)mcode;
+                    if ((t & 3) == 0 && ok) macro0[c >> 2] = (uint8_t)mcode;
 #pragma unroll
                     for (int k = 0; k < NB; ++k) {
                         a[k] = __fmul_rn(a[k], invm);
@@ -527,21 +532,21 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
             }
             }
             if (ok) {
-                reinterpret_cast<uint4 *>(p.codes)[c] = make_uint4(words[0], words[1], words[2], words[3]);
+                codes0[c] = make_uint4(words[0], words[1], words[2], words[3]);
                 if (G == 1 || (lane & (G - 1)) == 0) {
                     const uint32_t b0 = (G == 1) ? c * NB : c / G;
                     if (pc.sf_gemm) {
                         const uint32_t r = b0 / S, j = b0 - r * S;
 #pragma unroll
-                        for (int k = 0; k < NB; ++k) p.scales[sf_chunk_index(r, j + k, S)] = (uint8_t)scode[k];
+                        for (int k = 0; k < NB; ++k) scales0[sf_chunk_index(r, j + k, S)] = (uint8_t)scode[k];
                     } else if (NB == 4) {
-                        *reinterpret_cast<uint32_t *>(p.scales + b0) =
+                        *reinterpret_cast<uint32_t *>(scales0 + b0) =
                             scode[0] | (scode[NB > 1 ? 1 : 0] << 8) | (scode[NB > 2 ? 2 : 0] << 16) |
                             (scode[NB > 3 ? 3 : 0] << 24);
                     } else if (NB == 2) {
-                        *reinterpret_cast<uint16_t *>(p.scales + b0) = (uint16_t)(scode[0] | (scode[NB > 1 ? 1 : 0] << 8));
+                        *reinterpret_cast<uint16_t *>(scales0 + b0) = (uint16_t)(scode[0] | (scode[NB > 1 ? 1 : 0] << 8));
                     } else {
-                        p.scales[b0] = (uint8_t)scode[0];
+                        scales0[b0] = (uint8_t)scode[0];
                     }
                 }
                 if (STATS) {
