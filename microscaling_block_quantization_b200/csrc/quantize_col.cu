@@ -609,7 +609,8 @@ __global__ void __launch_bounds__(kColThreads) k_amax_col(const QParams p)
 // scaled in one mixed-precision multiply-add (y * 2^-k exactly; nearest
 // scales: widened, then multiplied), and the fidelity sums are formed on the
 // scaled values, s - q with q decoded by the conversion instruction, times
-// the block's scale once per block.
+// the block's scale once per block.  One launch may cover several tensors
+// (a group), the CTAs split among them.
 constexpr int kColxWarps = 12;
 constexpr int kColxThreads = kColxWarps * 32;
 constexpr int kColxTileRows = 32;

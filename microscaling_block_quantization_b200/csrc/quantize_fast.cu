@@ -10,6 +10,9 @@
 // reads of its own chunk are bank-conflict free), each consumer lane
 // quantizes one chunk per tile: all of HBM's latency is covered by the ring,
 // and the registers hold no load buffers.  Every mbarrier wait is bounded.
+// One launch may cover several tensors of one configuration (a group): the
+// CTAs are split among them, and each tensor keeps its own tensor scale,
+// statistics records and ticket.
 #include <string.h>
 
 #include "tma_ring.cuh"
