@@ -141,3 +141,37 @@ def test_group_workspaces_and_repeats(mx):
     with pytest.raises(mx.MXError):
         mx.quantize_group(xs[:2], cfg, workspaces=[wss[0], wss[0]])
     assert mx.mx_device_status() == 0
+
+
+def test_group_given_and_reduced_tensor_scales(mx, orc):
+    """The two other tensor-scale modes in a group: a given s_T per tensor
+    (TS_GIVEN, read from each tensor's own scalar), and an amax word already
+    in each tensor's workspace (TS_AMAX, left there by tensor_amax as the
+    row-sharded path does): each tensor as if quantized alone."""
+    import dataclasses
+    xs = _tensors("nvfp4")
+    dx = [x.cuda() for x in xs]
+    # given: each tensor's own scale, 1/2 and 3 times its computed one
+    alone = [mx.quantize(x, mx.NVFP4) for x in dx]
+    torch.cuda.synchronize()
+    given = dataclasses.replace(mx.NVFP4, tensor_scale=mx.TS_GIVEN)
+    outs = []
+    for i, (x, a) in enumerate(zip(dx, alone)):
+        ts = (a.tensor_scale * (0.5 if i % 2 else 3.0)).clone()
+        outs.append(mx.alloc_outputs(given, *x.shape, "cuda", tensor_scale=ts))
+    qs = mx.quantize_group(dx, given, outs=outs)
+    torch.cuda.synchronize()
+    for x, q in zip(xs, qs):
+        run_case(mx, orc, x, given, given_ts=float(q.tensor_scale.item()), want_rotated=False, q=q)
+    # reduced amax words
+    amax_cfg = dataclasses.replace(mx.NVFP4, tensor_scale=mx.TS_AMAX)
+    wss = [mx.new_workspace(amax_cfg, *x.shape, "cuda") for x in dx]
+    for x, w in zip(dx, wss):
+        mx.tensor_amax(x, amax_cfg, w)
+    qs = mx.quantize_group(dx, amax_cfg, workspaces=wss)
+    torch.cuda.synchronize()
+    for q, a in zip(qs, alone):
+        assert torch.equal(q.codes, a.codes) and torch.equal(q.scales, a.scales)
+        assert torch.equal(q.tensor_scale, a.tensor_scale)
+    for w in wss:
+        assert int(w[:256].count_nonzero()) == 0
