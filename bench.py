@@ -19,6 +19,7 @@ quantizes its own copy of the layer, no data-path collective.)
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -304,6 +305,24 @@ def run_ours(args, rank, world, device):
                     if call[0] == name:
                         run_call(*call)
         pair_graphs[name] = g
+    # NVFP4's quantizer launch alone (k_quant_fast without the tensor-amax
+    # launch before it): the same grouped launch with each tensor's tensor
+    # scale given (the values the step computes), into separate outputs
+    nv_name, nv_ts, nv_cfg, _ = next(c for c in calls if c[0] == "nvfp4_row")
+    nv_given = dataclasses.replace(nv_cfg, tensor_scale=mx.TS_GIVEN)
+    nv_outs = [mx.alloc_outputs(nv_given, *T[t].shape, device, stats=True,
+                                tensor_scale=outs[(nv_name, t)].tensor_scale.clone()) for t in nv_ts]
+    nv_wss = [mx.new_workspace(nv_given, *T[t].shape, device) for t in nv_ts]
+
+    def nv_quantizer_only():
+        mx.quantize_group([T[t] for t in nv_ts], nv_given, outs=nv_outs, workspaces=nv_wss)
+    nv_quantizer_only()
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(R_PAIRS):
+            nv_quantizer_only()
+    pair_graphs["nvfp4_row_quantizer"] = g
     for _ in range(args.warmup):
         step_graph.replay()
     torch.cuda.synchronize(device)
@@ -338,7 +357,7 @@ def run_ours(args, rank, world, device):
 
     # per-variant device time (A + W launches) from its pair graph
     rows = {}
-    for name in variants:
+    for name in variants + ["nvfp4_row_quantizer"]:
         g = pair_graphs[name]
         g.replay()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -347,33 +366,40 @@ def run_ours(args, rank, world, device):
             g.replay()
         e1.record(stream)
         torch.cuda.synchronize(device)
-        nb = sum(algo_bytes(cfg, *T[t].shape, kind) for n, t, cfg, kind in plan if n == name)
+        src = "nvfp4_row" if name == "nvfp4_row_quantizer" else name
+        nb = sum(algo_bytes(cfg, *T[t].shape, kind) for n, t, cfg, kind in plan if n == src)
         ms = e0.elapsed_time(e1) / (args.steps * R_PAIRS)
         rows[name] = {"bytes": nb, "GB_per_s": round(nb / (ms * 1e-3) / 1e9, 1), "us": round(ms * 1e3, 2)}
     del pair_graphs
 
     pk, pk_src = peaks()
     # the dominant kernel of the step: k_quant_fast, the four grouped
-    # quantizer launches over A and W (NVFP4's per-call time includes its
-    # tensor-amax pre-pass)
-    qnames = ["mxfp4_row", "nvfp4_row", "had32_mxfp4", "mbs_oas_mxfp4"]
+    # quantizer launches over A and W, each timed alone (NVFP4's quantizer
+    # launch without the tensor-amax launch, a separate kernel, before it);
+    # the same with NVFP4's whole call (amax launch included) beside it
+    qnames = ["mxfp4_row", "nvfp4_row_quantizer", "had32_mxfp4", "mbs_oas_mxfp4"]
+    qnames_call = ["mxfp4_row", "nvfp4_row", "had32_mxfp4", "mbs_oas_mxfp4"]
     qbytes = sum(rows[n]["bytes"] for n in qnames)
     qus = sum(rows[n]["us"] for n in qnames)
     achieved = round(qbytes / (qus * 1e-6) / 1e9, 1)
+    achieved_call = round(qbytes / (sum(rows[n]["us"] for n in qnames_call) * 1e-6) / 1e9, 1)
     traffic = traffic_record("mxfp4_row_AW")
     roofline = {"bound": "hbm",
                 "kernel": "k_quant_fast (TMA-fed E2M1 quantizer, statistics summed by the last CTA of each "
-                          "tensor): the step's 4 grouped launches, MXFP4 / NVFP4 (with its tensor-amax "
-                          "pre-pass) / rotation-32 / MBS+OAS, each over A and W",
+                          "tensor): the step's 4 grouped launches, MXFP4 / NVFP4 / rotation-32 / MBS+OAS, "
+                          "each over A and W, each launch timed alone (NVFP4's tensor-amax pre-pass is a "
+                          "separate kernel, k_amax_vec: see achieved_with_amax_pass)",
                 "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / pk["hbm_gbs"], 4), "peak_source": pk_src,
+                "achieved_with_amax_pass": achieved_call,
+                "frac_with_amax_pass": round(achieved_call / pk["hbm_gbs"], 4),
                 "traffic": traffic,
                 "traffic_launch": "the grouped MXFP4 launch on A and W (dram read + write per launch, from the "
                                   "ncu capture of the 16384 x 8192 case scaled by elements)",
                 "traffic_launch_algorithmic_bytes": algo_bytes(mx.MXFP4, M_TOK, K_DIM, "q")
                                                     + algo_bytes(mx.MXFP4, N_OUT, K_DIM, "q"),
                 "algorithmic_bytes_per_step": qbytes,
-                "by_variant_frac": {n: round(rows[n]["GB_per_s"] / pk["hbm_gbs"], 4) for n in qnames}}
+                "by_variant_frac": {n: round(rows[n]["GB_per_s"] / pk["hbm_gbs"], 4) for n in qnames_call + ["nvfp4_row_quantizer"]}}
 
     extra = run_extra_rows(mx, A, W, device, args)
     try:
@@ -956,9 +982,10 @@ def main():
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "step": [f"{n}:{t}" for n, t, _, _ in step_plan(__import__("microscaling_block_quantization_b200"))],
                    "step_algorithmic_bytes": r["step_bytes"], "hbm_frac_of_8TBs": round(r["value"] / world / 8000, 4),
-                   "quantize_only_GB_per_s": r["roofline"]["achieved"],
-                   "quantize_only_note": "the step's 4 grouped quantizer calls on A and W (no dequantizer): their "
-                                         "algorithmic bytes over their summed call durations, one stream",
+                   "quantize_only_GB_per_s": r["roofline"]["achieved_with_amax_pass"],
+                   "quantize_only_note": "the step's 4 grouped quantizer calls on A and W (NVFP4's tensor-amax "
+                                         "launch included, no dequantizer): their algorithmic bytes over their "
+                                         "summed call durations, one stream",
                    "per_launch_timing": f"per variant a graph of {R_PAIRS} back-to-back calls over A and W "
                                         "(one grouped quantizer launch each), replayed K times (no graph-launch "
                                         "gap between launches)",

@@ -72,6 +72,27 @@ def test_step_call_full_size(mx, orc, name):
             assert torch.equal(a.macro, q.macro)
 
 
+def test_nvfp4_quantizer_launch_alone_full_size(mx):
+    """The launch the benchmark times for NVFP4's quantizer alone: the grouped
+    NVFP4 launch over the full-size A and W with each tensor's scale given
+    (the values the computed call wrote) gives the computed call's bits."""
+    import dataclasses
+    L = _layer()
+    xs = [L[t].cuda() for t in ("A", "W")]
+    computed = mx.quantize_group(xs, mx.NVFP4)
+    given = dataclasses.replace(mx.NVFP4, tensor_scale=mx.TS_GIVEN)
+    outs = [mx.alloc_outputs(given, *x.shape, "cuda", tensor_scale=q.tensor_scale.clone())
+            for x, q in zip(xs, computed)]
+    qs = mx.quantize_group(xs, given, outs=outs)
+    torch.cuda.synchronize()
+    for a, q in zip(computed, qs):
+        assert torch.equal(a.codes, q.codes) and torch.equal(a.scales, q.scales)
+        assert torch.equal(a.tensor_scale, q.tensor_scale)
+        st_a, st_q = a.stats.cpu().numpy(), q.stats.cpu().numpy()
+        assert np.array_equal(st_a[[3, 4, 9, 10]], st_q[[3, 4, 9, 10]])
+        assert np.allclose(st_a, st_q, rtol=1e-9, atol=0, equal_nan=True)
+
+
 def test_step_plan_is_covered(mx):
     """Every quantizer launch of the benchmark's step is one of the cases
     above, and the step issues each variant as one call over A and W."""
