@@ -421,6 +421,20 @@ def run_ours(args, rank, world, device):
                                                   "and the timed region"), extra=extra)
 
 
+GRAD_ROWS, GRAD_COLS, GRAD_SEED = 4096, 14336, 5      # the fp32 gradient-like tensor of the extra rows
+
+
+def extra_row_cases(mx):
+    """(row name, tensors, config) of the extra rows: "A"/"W" the layer's
+    operands (quantized together in one grouped call), "G" the fp32
+    gradient-like tensor."""
+    return [("mxfp4_col_AW", ("A", "W"), mx.Config(axis=1)), ("mxfp4_2d_AW", ("A", "W"), mx.Config(axis=2)),
+            ("e2m1_sr_grad_fp32", ("G",), mx.Config(round=mx.ROUND_STOCHASTIC, seed=5)),
+            ("e2m3_grad_fp32", ("G",), mx.Config(elem=mx.E2M3)),
+            ("int4_asym_grad_fp32", ("G",), mx.Config(elem=mx.INT4, asymmetric=1, rule=mx.RULE_CEIL)),
+            ("e3m0_ceil_grad_fp32", ("G",), mx.Config(elem=mx.E3M0, rule=mx.RULE_CEIL))]
+
+
 def run_extra_rows(mx, A, W, device, args):
     """The other rows of the path, outside the headline step: column and 2D
     blocks on the layer's A and W (one grouped call over both), and on a
@@ -429,12 +443,9 @@ def run_extra_rows(mx, A, W, device, args):
     R_PAIRS back-to-back calls (A and W together, and the 224 MiB gradient,
     are larger than L2, so no input is served from L2), replayed K times."""
     from microscaling_block_quantization_b200 import inputs
-    G = inputs.gradient_like(4096, 14336, seed=5).to(device)
-    cases = [("mxfp4_col_AW", (A, W), mx.Config(axis=1)), ("mxfp4_2d_AW", (A, W), mx.Config(axis=2)),
-             ("e2m1_sr_grad_fp32", (G,), mx.Config(round=mx.ROUND_STOCHASTIC, seed=5)),
-             ("e2m3_grad_fp32", (G,), mx.Config(elem=mx.E2M3)),
-             ("int4_asym_grad_fp32", (G,), mx.Config(elem=mx.INT4, asymmetric=1, rule=mx.RULE_CEIL)),
-             ("e3m0_ceil_grad_fp32", (G,), mx.Config(elem=mx.E3M0, rule=mx.RULE_CEIL))]
+    G = inputs.gradient_like(GRAD_ROWS, GRAD_COLS, seed=GRAD_SEED).to(device)
+    tens = {"A": A, "W": W, "G": G}
+    cases = [(name, tuple(tens[t] for t in ts), cfg) for name, ts, cfg in extra_row_cases(mx)]
     out = {}
     stream = torch.cuda.current_stream(device)
     for name, xs, cfg in cases:

@@ -93,6 +93,47 @@ def test_nvfp4_quantizer_launch_alone_full_size(mx):
         assert np.allclose(st_a, st_q, rtol=1e-9, atol=0, equal_nan=True)
 
 
+_GRAD = {}
+
+
+def _grad():
+    if not _GRAD:
+        _GRAD["G"] = inputs.gradient_like(bench.GRAD_ROWS, bench.GRAD_COLS, seed=bench.GRAD_SEED)
+    return _GRAD["G"]
+
+
+@pytest.mark.parametrize("name", [n for n, _, _ in bench.extra_row_cases(__import__("microscaling_block_quantization_b200"))])
+def test_extra_row_full_size(mx, orc, name):
+    """Every extra row of the benchmark in the launch it times: column and 2D
+    blocks as one grouped call over the full-size A and W, the fp32 gradient
+    rows on the 4096 x 14336 tensor; codes, scales (and offsets) against the
+    oracle, and the dequantized tensor and statistics (the gradient rows on
+    256 sampled rows of x_hat: the statistics of stochastic rounding are
+    covered by the smaller tests)."""
+    _, ts, cfg = next(c for c in bench.extra_row_cases(mx) if c[0] == name)
+    if ts == ("A", "W"):
+        L = _layer()
+        qs = mx.quantize_group([L[t].cuda() for t in ts], cfg)
+        torch.cuda.synchronize()
+        for t, q in zip(ts, qs):
+            run_case(mx, orc, L[t], cfg, want_rotated=False, q=q)
+        return
+    from .test_gpu_quantize import assert_same_f32, ocfg
+    x = _grad()
+    q = mx.quantize(x.cuda(), cfg)
+    torch.cuda.synchronize()
+    oc = ocfg(orc, cfg)
+    full = orc.quantize(oc, x)
+    assert np.array_equal(q.codes.cpu().numpy(), full["packed"].ravel()), "packed codes"
+    assert np.array_equal(q.scales.cpu().numpy(), full["scales"]), "scales"
+    if cfg.asymmetric:
+        assert np.array_equal(q.offsets.cpu().numpy().view(np.uint16), full["offsets"]), "offsets"
+    rows = np.random.default_rng(1).choice(x.shape[0], 256, replace=False)
+    xh = mx.dequantize(q, torch.float32).cpu().numpy()
+    oxh = orc.dequantize(oc, full["packed"], full["scales"], None, None, full["offsets"], *x.shape)
+    assert_same_f32(xh[rows], oxh[rows], "dequantized sample")
+
+
 def test_step_plan_is_covered(mx):
     """Every quantizer launch of the benchmark's step is one of the cases
     above, and the step issues each variant as one call over A and W."""
