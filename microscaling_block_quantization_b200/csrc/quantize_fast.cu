@@ -355,10 +355,15 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
                     sm = mt.x;
                     invm = mt.y;
                     if ((t & 3) == 0 && ok) macro0[c >> 2] = (uint8_t)mcode;
+                    // a block is non-finite when any of its y' is: a NaN
+                    // macro scale (a non-finite value in the macro block)
+                    // makes every block of it NaN, and y * (1 / S_M) may
+                    // overflow for the largest bf16 values
 #pragma unroll
                     for (int k = 0; k < NB; ++k) {
                         a[k] = __fmul_rn(a[k], invm);
                         mn[k] = __fmul_rn(mn[k], invm);
+                        bad[k] = !(a[k] <= FLT_MAX);
                     }
                 }
 #pragma unroll
@@ -391,13 +396,6 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
                     for (int g = 0; g < L / 8; ++g) {
                         float s8[8];
                         bf16x8_scale(wb + 4 * g, kb, s8);
-                        if (WIDEN && STATS) {
-#pragma unroll
-                            for (int e = 0; e < 8; e += 2) {
-                                const float2 yv = make_float2(s8[e], s8[e + 1]);
-                                sx2 = __ffma2_rn(yv, yv, sx2);
-                            }
-                        }
                         if (WIDEN) {
 #pragma unroll
                             for (int e = 0; e < 8; e += 2) {
@@ -419,24 +417,34 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
                                 const int u = (e >> 1) & 1;
                                 re2[u] = __ffma2_rn(d, d, re2[u]);
                                 rb2[u] = __fadd2_rn(rb2[u], d);
-                                if (!WIDEN) {
-                                    // y = 2^k s exactly: sum s^2, scaled below
-                                    const float2 sv = make_float2(s8[e], s8[e + 1]);
-                                    sx2 = __ffma2_rn(sv, sv, sx2);
-                                }
+                                // reference sum on the scaled values (y = X s,
+                                // exactly for power-of-two scales): sum s^2,
+                                // times X^2 below in binary64
+                                const float2 sv = make_float2(s8[e], s8[e + 1]);
+                                sx2 = __ffma2_rn(sv, sv, sx2);
                             }
                             qz += zero_codes8(word);
                         }
                     }
                     if (STATS) {
                         if (ok) {
-                            // y - x_hat = deqT (s - q); reference sums of y (R = 1)
-                            // or of s with y = 2^k s (R = 2^k; 1 in a flushed block)
+                            // y - x_hat = deqT (s - q); reference sum sum s^2 X^2
+                            // (a flushed block: s = y, X = 1)
                             const double X = (double)deqT;
-                            const double R = (WIDEN || flush) ? 1.0 : (double)bs.deq;
                             acc.e2 += (double)((re2[0].x + re2[1].x) + (re2[0].y + re2[1].y)) * X * X;
                             acc.e -= (double)((rb2[0].x + rb2[1].x) + (rb2[0].y + rb2[1].y)) * X;
-                            acc.x2 += (double)(sx2.x + sx2.y) * R * R;
+                            if (!bs.nan) {
+                                acc.x2 += (double)(sx2.x + sx2.y) * X * X;
+                            } else {
+                                // a non-finite block (rare): sum y^2 of its inputs in binary64
+                                double t2 = 0.0;
+                                for (int j = 0; j < L / 2; ++j) {
+                                    const double y0 = (double)__uint_as_float(wb[j] << 16);
+                                    const double y1 = (double)__uint_as_float(wb[j] & 0xffff0000u);
+                                    t2 += y0 * y0 + y1 * y1;
+                                }
+                                acc.x2 += t2;
+                            }
                         }
                         int xz = 0;
                         if (mn[k] == 0.0f)                 // rare: count exact zeros
@@ -511,19 +519,30 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
                             const int u = (e >> 1) & 1;          // two accumulator chains
                             re2[u] = __ffma2_rn(d, d, re2[u]);
                             rb2[u] = __fadd2_rn(rb2[u], d);
-                            const float2 yv = make_float2(y[jb + e], y[jb + e + 1]);
-                            sx2[u] = __ffma2_rn(yv, yv, sx2[u]);
+                            const float2 sv = make_float2(s8[e], s8[e + 1]);
+                            sx2[u] = __ffma2_rn(sv, sv, sx2[u]);     // reference values X s
                         }
                         qz += zero_codes8(word);
                     }
                 }
                 if (STATS) {
                     if (ok) {
-                        // y - x_hat = deqT (s - q); a NaN block makes the sums NaN
-                        const double X = (double)deqT, R = (double)sxm;
+                        // y - x_hat = deqT (s - q); a NaN block makes the sums NaN;
+                        // reference sum sum s^2 X^2 (a flushed block: s = sxm y, X = 1)
+                        const double X = (double)deqT;
                         acc.e2 += (double)((re2[0].x + re2[1].x) + (re2[0].y + re2[1].y)) * X * X;
                         acc.e -= (double)((rb2[0].x + rb2[1].x) + (rb2[0].y + rb2[1].y)) * X;
-                        acc.x2 += (double)((sx2[0].x + sx2[1].x) + (sx2[0].y + sx2[1].y)) * R * R;
+                        if (!bs.nan) {
+                            acc.x2 += (double)((sx2[0].x + sx2[1].x) + (sx2[0].y + sx2[1].y)) * X * X;
+                        } else {
+                            // a non-finite block (rare): the reference values sxm y in binary64
+                            double t2 = 0.0;
+                            for (int j = j0; j < j0 + L; ++j) {
+                                const double v = (double)y[j] * (double)sxm;
+                                t2 += v * v;
+                            }
+                            acc.x2 += t2;
+                        }
                     }
                     int xz = 0;
                     if (mabs == 0.0f)                      // rare: count exact zeros

@@ -421,6 +421,40 @@ def test_special_values(mx, orc):
         run_case(mx, orc, x16, mx.Config(**cfg), check_stats=False)
 
 
+def test_special_values_mbs(mx, orc):
+    """Every bf16 bit pattern under the macro-block scale (rows of 128, so
+    each 1 x 128 macro block mixes NaN / Inf, huge, subnormal and zero
+    values with ordinary ones): macro codes, codes, scales and x_hat."""
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(512, 128)
+    x = torch.from_numpy(pats.view(np.int16)).view(torch.bfloat16)
+    perm = np.random.default_rng(3).permutation(65536)
+    xp = torch.from_numpy(pats.ravel()[perm].reshape(512, 128).view(np.int16)).view(torch.bfloat16)
+    for t in (x, xp):
+        for cfg in (dict(macro_block=128), dict(macro_block=128, rule=1), dict(macro_block=128, rule=2, oas_tau=7.0),
+                    dict(macro_block=128, block=16), dict(macro_block=128, block=16, rule=2, oas_tau=6.5)):
+            run_case(mx, orc, t, mx.Config(**cfg), check_stats=False)
+
+
+def test_mbs_wide_dynamic_range(mx, orc):
+    """Finite values from 2^-133 to 2^126 (bf16 subnormals included), the
+    magnitudes of a 1 x 128 macro block spread over the whole range or over
+    a narrow band at either end: codes, scales, macro codes, x_hat and the
+    statistics (the squares of values above 2^64 overflow binary32, so the
+    reference sum must be taken on the scaled values).  The largest values
+    stay below 2^126: within a factor 2 of the binary32 maximum a dequantized
+    value can itself overflow, where the oracle's error sum is infinite and
+    the fused sums (formed exactly as X (s - q) in binary64) are not."""
+    rng = np.random.default_rng(11)
+    rows = []
+    for lo, hi in ((-133, 126), (-133, -100), (100, 126), (-20, 20)):
+        e = rng.uniform(lo, hi, size=(64, 256))
+        m = rng.uniform(1.0, 2.0, size=(64, 256))
+        rows.append(np.where(rng.random((64, 256)) < 0.5, -1.0, 1.0) * m * np.exp2(e))
+    x = torch.from_numpy(np.concatenate(rows).astype(np.float32)).to(torch.bfloat16)
+    for cfg in (dict(macro_block=128), dict(macro_block=128, rule=2, oas_tau=7.0), dict(macro_block=128, block=16)):
+        run_case(mx, orc, x, mx.Config(**cfg))
+
+
 def test_zeros_and_empty(mx, orc):
     z = torch.zeros(64, 256, dtype=torch.bfloat16)
     q, _ = run_case(mx, orc, z, mx.MXFP4)
