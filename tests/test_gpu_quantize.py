@@ -435,6 +435,29 @@ def test_special_values_mbs(mx, orc):
             run_case(mx, orc, t, mx.Config(**cfg), check_stats=False)
 
 
+@pytest.mark.parametrize("path", ["had32", "had16", "nvfp4_had16", "had32_mbs", "col", "col_nvfp4", "col_mbs", "2d",
+                                  "2d_nvfp4"])
+def test_special_values_other_paths(mx, orc, path):
+    """Every bf16 bit pattern through the rotation (TMA-fed and lane-per-chunk
+    kernels), column-block and 2D-tile quantizers: NaN / Inf spreading through
+    the butterflies, huge, subnormal and zero values."""
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    perm = np.random.default_rng(5).permutation(65536)
+    shape = (512, 128) if path in ("had32_mbs", "col_mbs") else (2048, 32)
+    x = torch.from_numpy(pats[perm].reshape(shape).view(np.int16)).view(torch.bfloat16)
+    nv = dict(block=16, scale_fmt=1, rule=3, tensor_scale=1)
+    cfg = {"had32": dict(hadamard=32), "had16": dict(hadamard=16, block=16),
+           "nvfp4_had16": dict(hadamard=16, **nv), "had32_mbs": dict(hadamard=32, macro_block=128),
+           "col": dict(axis=1), "col_nvfp4": dict(axis=1, **nv), "col_mbs": dict(axis=1, macro_block=128),
+           "2d": dict(axis=2), "2d_nvfp4": dict(axis=2, block=32, scale_fmt=1, rule=3, tensor_scale=1)}[path]
+    c = mx.Config(**cfg)
+    if c.hadamard:
+        run_case(mx, orc, x, c, check_stats=False, want_rotated=False)
+        run_case(mx, orc, x, c, check_stats=False, want_rotated=True)
+    else:
+        run_case(mx, orc, x, c, check_stats=False)
+
+
 def test_mbs_wide_dynamic_range(mx, orc):
     """Finite values from 2^-133 to 2^126 (bf16 subnormals included), the
     magnitudes of a 1 x 128 macro block spread over the whole range or over
