@@ -320,6 +320,17 @@ __device__ __forceinline__ float deq_value(const QParams &p, float q, const Bloc
     return v;
 }
 
+// A power of two P near 1 / a and 1 / P, both normal (a zero or subnormal a:
+// 1, 1): y P is exact and below 2 in magnitude for |y| <= a, so the residuals
+// of a flushed block (x_hat = 0) can be summed as (y P)^2 (1 / P)^2 without a
+// binary32 overflow.
+__device__ __forceinline__ float2 pow2_near_inv(float a)
+{
+    const uint32_t ef = (__float_as_uint(a) >> 23) & 0xffu;
+    const uint32_t fe = ef == 0u ? 127u : (ef > 253u ? 253u : ef);
+    return make_float2(__uint_as_float((254u - fe) << 23), __uint_as_float(fe << 23));
+}
+
 // Macro-block (MBS) scale code from the macro absmax and a non-finite flag:
 // E4M3 nearest to m / (max_elem / 2^emax), m the mantissa of the absmax.
 __device__ __forceinline__ uint32_t macro_code(const ElemDesc &ed, float amax, int bad)

@@ -814,11 +814,15 @@ __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const __grid_consta
         for (int j = 0; j < 4; ++j) {
             const BlockScale &s = bs[(AXIS == AX_COL) ? j : 0];
             const bool flush = s.zero && !s.nan;
-            inv[j] = flush ? 1.0f : s.inv;
+            // the scaled values s and their reference factor X (y = X s):
+            // a flushed block is scaled by a power of two from its column's
+            // maximum (its codes are zero), a non-finite one not at all
+            const float2 pp = pow2_near_inv(a[j]);
+            inv[j] = s.nan ? 1.0f : flush ? pp.x : s.inv;
             kb[j] = NEAR ? 0x3f80u : (__float_as_uint(inv[j]) >> 16);
             if (s.zero) zmask &= ~(0xfu << (4 * j));
-            X[j] = s.nan ? __uint_as_float(0x7fc00000u) : flush ? 1.0f : s.deq;
-            R[j] = (NEAR || flush) ? 1.0f : s.deq;
+            X[j] = s.nan ? __uint_as_float(0x7fc00000u) : flush ? pp.y : s.deq;
+            R[j] = s.nan ? 1.0f : X[j];
         }
 
         float2 re2[2], rb2[2], sx2[2];
@@ -844,10 +848,7 @@ __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const __grid_consta
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     float2 sv = bfx_scale2(v[i], kb[2 * i], kb[2 * i + 1]);
-                    if (NEAR) {
-                        if (STATS) sx2[i] = __ffma2_rn(sv, sv, sx2[i]);       // reference y
-                        sv = __fmul2_rn(sv, make_float2(inv[2 * i], inv[2 * i + 1]));
-                    }
+                    if (NEAR) sv = __fmul2_rn(sv, make_float2(inv[2 * i], inv[2 * i + 1]));
                     s8[4 * rr + 2 * i] = sv.x;
                     s8[4 * rr + 2 * i + 1] = sv.y;
                 }
@@ -872,16 +873,14 @@ __global__ void __launch_bounds__(kColxThreads) k_quant_colx(const __grid_consta
                     const float2 d = sub_f16x2_from(s8[2 * e], s8[2 * e + 1], h[e]);   // s - q
                     re2[i] = __ffma2_rn(d, d, re2[i]);
                     rb2[i] = __fadd2_rn(rb2[i], d);
-                    if (!NEAR) {
-                        const float2 sv = make_float2(s8[2 * e], s8[2 * e + 1]);
-                        sx2[i] = __ffma2_rn(sv, sv, sx2[i]);                 // y = R s
-                    }
+                    const float2 sv = make_float2(s8[2 * e], s8[2 * e + 1]);
+                    sx2[i] = __ffma2_rn(sv, sv, sx2[i]);                     // y = R s
                 }
                 qz += 8 - __popc(((word & 0x77777777u) + 0x77777777u) & 0x88888888u);
             }
         }
         if (STATS && ok) {
-            // y - x_hat = X (s - q) per column; reference sums R^2 sum s^2 (or sum y^2)
+            // y - x_hat = X (s - q) per column; reference sums R^2 sum s^2
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int i = j >> 1;

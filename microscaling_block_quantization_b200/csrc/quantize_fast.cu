@@ -377,11 +377,14 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
                     if (MBS) deqT = __fmul_rn(deqT, sm);       // X S_M, exact (E4M3 times a power of two)
                     float inv = bs.inv, im = invm;
                     // a flushed block: residuals are the inputs themselves
+                    // (scaled by a power of two from the block maximum, so that
+                    // their squares stay within binary32)
                     const bool flush = bs.zero && !bs.nan;
                     if (flush) {
-                        inv = 1.0f;
+                        const float2 pp = pow2_near_inv(a[k]);
+                        inv = pp.x;
                         im = 1.0f;
-                        deqT = 1.0f;
+                        deqT = pp.y;
                     }
                     // power-of-two rules: s = y 2^-k straight from the packed
                     // words (exact); nearest scales and MBS: widen, then
@@ -487,10 +490,13 @@ __global__ void __launch_bounds__(kFastThreads, (HADN || ((MBS || STATS) && size
                     }
                 }
                 // a flushed block (x_hat = 0, not NaN): residuals are the
-                // reference values themselves, s = sxm * y with factor 1
+                // reference values themselves, s = sxm y P with factor 1 / P
+                // (P a power of two from the block maximum: no binary32
+                // overflow of the squares)
                 if (bs.zero && !bs.nan) {
-                    inv = sxm;
-                    deqT = 1.0f;
+                    const float2 pp = pow2_near_inv(__fmul_rn(a, MBS ? sm : 1.0f));
+                    inv = __fmul_rn(sxm, pp.x);
+                    deqT = pp.y;
                 }
                 const float2 inv2 = make_float2(inv, inv);
                 float2 sx2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};

@@ -458,12 +458,13 @@ def test_special_values_other_paths(mx, orc, path):
         run_case(mx, orc, x, c, check_stats=False)
 
 
-def test_mbs_wide_dynamic_range(mx, orc):
+def test_wide_dynamic_range(mx, orc):
     """Finite values from 2^-133 to 2^126 (bf16 subnormals included), the
-    magnitudes of a 1 x 128 macro block spread over the whole range or over
-    a narrow band at either end: codes, scales, macro codes, x_hat and the
-    statistics (the squares of values above 2^64 overflow binary32, so the
-    reference sum must be taken on the scaled values).  The largest values
+    magnitudes of a row spread over the whole range or over a narrow band at
+    either end, through MBS, MXFP4, NVFP4 (blocks far below the tensor's
+    maximum flush to a zero scale), rotation, column and 2D blocks: codes,
+    scales, macro codes, x_hat and the statistics (the squares of values
+    above 2^64 overflow binary32, so the sums must be taken on scaled values).  The largest values
     stay below 2^126: within a factor 2 of the binary32 maximum a dequantized
     value can itself overflow, where the oracle's error sum is infinite and
     the fused sums (formed exactly as X (s - q) in binary64) are not."""
@@ -474,8 +475,18 @@ def test_mbs_wide_dynamic_range(mx, orc):
         m = rng.uniform(1.0, 2.0, size=(64, 256))
         rows.append(np.where(rng.random((64, 256)) < 0.5, -1.0, 1.0) * m * np.exp2(e))
     x = torch.from_numpy(np.concatenate(rows).astype(np.float32)).to(torch.bfloat16)
-    for cfg in (dict(macro_block=128), dict(macro_block=128, rule=2, oas_tau=7.0), dict(macro_block=128, block=16)):
-        run_case(mx, orc, x, mx.Config(**cfg))
+    # scales that span the range: E8M0, or UE4M3 with the FP32 tensor scale
+    # (UE scales without one saturate for blocks far above their range, and
+    # a rotation of values near the binary32 maximum overflows)
+    for cfg in (dict(macro_block=128), dict(macro_block=128, rule=2, oas_tau=7.0), dict(macro_block=128, block=16),
+                dict(), dict(rule=1), dict(block=16, scale_fmt=1, rule=3, tensor_scale=1),
+                dict(axis=1), dict(axis=2), dict(axis=1, block=16, scale_fmt=1, rule=3, tensor_scale=1),
+                dict(axis=2, scale_fmt=1, rule=3, tensor_scale=1)):
+        c = mx.Config(**cfg)
+        run_case(mx, orc, x, c, want_rotated=False if c.hadamard else None)
+    # the same values as fp32 input (the lane-per-chunk path of the fast quantizer)
+    run_case(mx, orc, x.float(), mx.Config(macro_block=128))
+    run_case(mx, orc, x.float(), mx.Config(block=16, scale_fmt=1, rule=3, tensor_scale=1))
 
 
 def test_zeros_and_empty(mx, orc):
