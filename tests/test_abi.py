@@ -216,3 +216,14 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(m, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError):
         m.lib()
+
+
+def test_group_binding_checks_on_host(mx):
+    """The grouped binding rejects CPU tensors and mixed dtypes before any
+    library call, and an empty group is an empty result."""
+    import torch
+    assert mx.quantize_group([], mx.MXFP4) == []
+    with pytest.raises(ValueError):
+        mx.quantize_group([torch.zeros(32, 64, dtype=torch.bfloat16)], mx.MXFP4)
+    with pytest.raises(ValueError):
+        mx.quantize_group([torch.zeros(2, 32, 64, dtype=torch.bfloat16)], mx.MXFP4)
